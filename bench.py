@@ -1,0 +1,327 @@
+#!/usr/bin/env python
+"""Benchmark of one batched exact Lloyd iteration (FlashAssign + Sort-Inverse Update) on B200.
+
+A step is one full Lloyd iteration -- centroid preparation, FlashAssign, label
+argsort, segmented gather-reduce, centroid finalisation -- over the workload
+B=32 independent problems x N=65536 points x d=128, K=1024 centroids, fp16
+inputs with fp32 accumulation (Gaussian mixture, 1024 components, sigma 0.3).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on stdout (rank 0).  Multi-GPU runs (torchrun) are replicas:
+every rank solves its own 32 problems (weak scaling, no data-path collective);
+the barrier and the max over ranks use NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per Lloyd iter at B32·N65536·K1024·d128 fp16; assign/update % of roofline"
+UNIT = "ms/iter"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", type=int, default=2, help="workload id (2 = the metric's configuration)")
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---- algorithmic work per launch (method's own, not the avoided N x K matrix) ----
+
+def work(w):
+    s = w.elem_bytes
+    B, N, K, d = w.B, w.N, w.K, w.d
+    flops_assign = 2.0 * B * N * K * d
+    bytes_assign = B * N * (d * s + 8) + B * K * (d * s + 4)
+    bytes_update = B * N * (d * s + 8) + 2 * B * K * d * 4 + 4 * B * K
+    passes = 2 if K > 256 else 1
+    bytes_sort = passes * B * N * 16 + B * N * 4
+    bytes_finalize = B * K * d * (4 + 4 + s) + B * K * 8
+    return dict(flops_assign=flops_assign, bytes_assign=bytes_assign, bytes_update=bytes_update,
+                bytes_sort=bytes_sort, bytes_finalize=bytes_finalize)
+
+
+# ---- clocks sampled during the timed region ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if uuid:
+            cmd += ["-i", uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---- CPU oracle baseline ----
+
+def cpu_oracle_ms_per_iter(w, X, C, rows: int):
+    """Time the oracle's assign + update over `rows` points of batch 0; extrapolate to one full iteration."""
+    import numpy as np
+    import oracle
+    sample_X = np.ascontiguousarray(X[:1, :rows])
+    t0 = time.perf_counter()
+    lab, _, _ = oracle.assign(sample_X, C[:1])
+    oracle.update(sample_X, lab, C[:1])
+    dt = time.perf_counter() - t0
+    scale = (w.B * w.N) / rows
+    return dt * scale * 1e3, dt, oracle.threads()
+
+
+def run_reference(args, w):
+    """The oracle arm: plain C++ CPU Lloyd on bounded samples of the same workload."""
+    import numpy as np
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = 4096
+    wx = w.with_(B=1)
+    X = synth.points(wx, 0, rows)  # batch 0, first rows: same distribution as the full workload
+    rng = np.random.default_rng(0)
+    C = X[:, rng.choice(rows, w.K, replace=False)].astype(np.float32)
+    times = []
+    for i in range(args.warmup + args.steps):
+        ms, dt, cores = cpu_oracle_ms_per_iter(w, X, C, rows)
+        if i >= args.warmup:
+            times.append(ms)
+    v = statistics.mean(times)
+    sample = (f"each step: oracle assign+update of {rows} of the {w.B * w.N} points (batch 0) against all "
+              f"K={w.K} centroids, extrapolated linearly to the full iteration")
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+           "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "parallelism": "replicas"},
+           "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import flashassign_b200 as km
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def allmax(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wr = w if rank == 0 else w.with_(seed=w.seed + 0x100 * rank)  # independent replicas
+    X_host = synth.points(wr)
+    C_init = synth.init_centroids(wr, X_host)
+    X = torch.from_numpy(X_host).cuda()
+    C = torch.from_numpy(C_init).cuda()
+    labels = torch.empty((w.B, w.N), dtype=torch.int32, device="cuda")
+    C_out = torch.empty_like(C)
+    stream = torch.cuda.current_stream()
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(local).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+
+    # warm-up: W iterations (also the first-call set-up)
+    km.lloyd(X, C, args.warmup, labels=labels, C_out=C_out)
+    C.copy_(C_out)
+    torch.cuda.synchronize()
+    assert km.device_fault() == 0
+
+    # timed: K iterations, one call, device-resident inputs (X = 512 MiB > L2)
+    km.trace_read()
+    km.trace_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    km.lloyd(X, C, args.steps, labels=labels, C_out=C_out)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    km.trace_enable(False)
+    phases = km.trace_read()
+    total_ms = allmax(ev0.elapsed_time(ev1))
+    ms_iter = total_ms / args.steps
+    C.copy_(C_out)
+    fault = km.device_fault()
+
+    # end to end: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        Xp = torch.from_numpy(X_host).pin_memory()
+        Cp = torch.from_numpy(C_init).pin_memory()
+        lab_h = torch.empty((w.B, w.N), dtype=torch.int32).pin_memory()
+        C_h = torch.empty_like(Cp).pin_memory()
+        Xd = torch.empty_like(X)
+        Cd = torch.empty_like(C)
+        steps_e = max(1, args.e2e_steps)
+
+        def e2e_step():
+            Xd.copy_(Xp, non_blocking=True)
+            Cd.copy_(Cp, non_blocking=True)
+            km.lloyd(Xd, Cd, 1, labels=labels, C_out=C_out)
+            lab_h.copy_(labels, non_blocking=True)
+            C_h.copy_(C_out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps_e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = allmax(e0.elapsed_time(e1)) / steps_e
+        e2e = {"value": round(e_ms, 4), "unit": UNIT, "steps": steps_e,
+               "h2d_bytes_per_step": int(Xp.numel() * Xp.element_size() + Cp.numel() * 4),
+               "d2h_bytes_per_step": int(lab_h.numel() * 4 + C_h.numel() * 4),
+               "path": "pinned host X and C copied in, km_lloyd(iters=1), labels and C copied out"}
+    clocks = sampler.stop()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    wk = work(w)
+    t_assign = phases["assign"][0] / args.steps
+    t_update = phases["update"][0] / args.steps
+    t_sort = phases["sort"][0] / args.steps
+    t_fin = phases["finalize"][0] / args.steps
+    t_other = phases["other"][0] / args.steps
+    tflops = wk["flops_assign"] / (t_assign * 1e-3) / 1e12
+    upd_gbs = wk["bytes_update"] / (t_update * 1e-3) / 1e9
+    peak_tf = peaks["bf16_tflops"]  # fp16 dense rate equals bf16; burst figure (short timed region)
+    peak_bw = peaks["hbm_gbs"]
+    t_roof = (max(wk["flops_assign"] / (peak_tf * 1e12), wk["bytes_assign"] / (peak_bw * 1e9)) +
+              (wk["bytes_update"] + wk["bytes_sort"] + wk["bytes_finalize"]) / (peak_bw * 1e9)) * 1e3
+    launches = sum(c for _, c in phases.values())
+
+    cpu = None
+    if not args.no_cpu and world == 1:
+        rows = 65536
+        ms_cpu, dt, cores = cpu_oracle_ms_per_iter(w, X_host, C_init, rows)
+        cpu = {"value": round(ms_cpu, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"oracle assign+update of batch 0 ({rows} points, K={w.K}, d={w.d}) took {dt:.2f} s; "
+                         f"extrapolated x{w.B} to the full {w.B}-problem iteration"}
+
+    out = {
+        "metric": METRIC, "value": round(ms_iter, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_iter, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "global_problems": w.B * world,
+                   "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (X is 512 MiB)"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(tflops / peak_tf, 4), "traffic": None, "kernel": "assign_tc_kernel",
+                     "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)",
+                     "ms_per_launch": round(t_assign, 4)},
+        "roofline_update": {"bound": "hbm", "achieved": round(upd_gbs, 1), "peak": peak_bw, "unit": "GB/s",
+                            "frac": round(upd_gbs / peak_bw, 4), "kernel": "update_kernel",
+                            "ms_per_launch": round(t_update, 4), "peak_source": peak_src},
+        "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4)},
+        "phases_ms_per_iter": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "device_fault": fault,
+    }
+    print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,444 @@
+// The extern "C" entry points of libkm.so (declared in include/km.h):
+// argument validation, stream-ordered scratch, and the composition of the
+// kernels into the assignment, sort, update and full Lloyd iterations
+// (papernotes.org "Flash-KMeans" page, 方法详解: 整体框架 and 关键设计 1-3).
+#include "km_internal.cuh"
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+namespace km {
+
+namespace {
+thread_local char g_err[512] = "";
+__device__ int32_t g_fault;  // device fault word (see km_device_fault)
+
+bool inject(const char* what) {
+    const char* f = std::getenv("KM_FAULT");
+    return f && std::strcmp(f, what) == 0;
+}
+
+// Scratch taken stream-ordered on one stream, released on scope exit.
+class Scratch {
+  public:
+    explicit Scratch(cudaStream_t st) : st_(st) {}
+    ~Scratch() {
+        for (void* p : ptrs_) cudaFreeAsync(p, st_);
+    }
+    template <typename T>
+    km_status get(T** out, size_t count, const char* what) {
+        *out = nullptr;
+        if (count == 0) return KM_OK;
+        void* p = nullptr;
+        cudaError_t e = inject("alloc") ? cudaErrorMemoryAllocation : cudaMallocAsync(&p, count * sizeof(T), st_);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            set_error("scratch allocation of %zu bytes for %s failed: %s", count * sizeof(T), what,
+                      cudaGetErrorString(e));
+            return KM_E_NOMEM;
+        }
+        ptrs_.push_back(p);
+        *out = static_cast<T*>(p);
+        return KM_OK;
+    }
+
+  private:
+    cudaStream_t st_;
+    std::vector<void*> ptrs_;
+};
+
+// ---- tracing: CUDA event pairs around each kernel phase ----
+std::atomic<bool> g_trace_on{false};
+std::mutex g_trace_mu;
+struct TraceRec {
+    int phase;
+    cudaEvent_t a, b;
+    int launches;
+};
+std::vector<TraceRec> g_trace;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return e;
+}
+
+class PhaseScope {
+  public:
+    PhaseScope(cudaStream_t st, int phase, int launches) : st_(st), phase_(phase), launches_(launches) {
+        if (g_trace_on.load(std::memory_order_relaxed)) {
+            a_ = take_event();
+            if (a_) cudaEventRecord(a_, st_);
+        }
+    }
+    ~PhaseScope() {
+        if (!a_) return;
+        cudaEvent_t b = take_event();
+        if (!b) return;
+        cudaEventRecord(b, st_);
+        std::lock_guard<std::mutex> lk(g_trace_mu);
+        g_trace.push_back({phase_, a_, b, launches_});
+    }
+
+  private:
+    cudaStream_t st_;
+    int phase_, launches_;
+    cudaEvent_t a_ = nullptr;
+};
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+km_status check_shape(int64_t B, int64_t N, int64_t K, int64_t d, int dtype) {
+    if (B < 1 || N < 1 || K < 1 || d < 1) {
+        set_error("sizes must be positive (B=%lld N=%lld K=%lld d=%lld)", (long long)B, (long long)N, (long long)K,
+                  (long long)d);
+        return KM_E_INVALID;
+    }
+    if (dtype != KM_F32 && dtype != KM_F16) {
+        set_error("unknown dtype %d", dtype);
+        return KM_E_INVALID;
+    }
+    if (B > 65535 || B * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 24) || d > 512) {
+        set_error("outside the supported range: B <= 65535, B*N < 2^31, K < 2^24, d <= 512");
+        return KM_E_UNSUPPORTED;
+    }
+    const int64_t s = dtype == KM_F16 ? 2 : 4;
+    if ((d * s) % 16 != 0) {
+        set_error("d * sizeof(dtype) = %lld bytes is not a multiple of 16", (long long)(d * s));
+        return KM_E_UNSUPPORTED;
+    }
+    return KM_OK;
+}
+
+km_status check_device(DeviceInfo* info) {
+    km_status st = device_info(info);
+    if (st != KM_OK) return st;
+    if (info->cc_major != 10 || info->cc_minor != 0) {
+        set_error("device %d has compute capability %d.%d; this library is built for sm_100a (10.0)", info->device,
+                  info->cc_major, info->cc_minor);
+        return KM_E_UNSUPPORTED;
+    }
+    return KM_OK;
+}
+
+km_status launched(cudaError_t e, const char* what) {
+    if (inject("launch")) e = cudaErrorLaunchFailure;
+    if (e != cudaSuccess) return cuda_error(e, what);
+    return KM_OK;
+}
+
+#define KM_TRY(expr)                       \
+    do {                                   \
+        km_status _s = (expr);             \
+        if (_s != KM_OK) return _s;        \
+    } while (0)
+
+// The assignment for one iteration, given prepared centroids.
+km_status run_assign(const void* X, int dtype, const float* C, const __half* chat, const float* cnh, int64_t B,
+                     int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, const DeviceInfo& dev,
+                     cudaStream_t st) {
+    PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
+    if (dtype == KM_F16 && assign_tc_supported(d, dtype))
+        return launched(launch_assign_tc((const __half*)X, chat, cnh, B, N, K, d, labels, mindist, dev.sms, st),
+                        "assign (tensor cores)");
+    return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, st), "assign (CUDA cores)");
+}
+
+bool uses_tc(int dtype, int64_t d) { return dtype == KM_F16 && assign_tc_supported(d, dtype); }
+
+}  // namespace
+
+void set_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+
+km_status cuda_error(cudaError_t e, const char* what) {
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return e == cudaErrorMemoryAllocation ? KM_E_NOMEM : KM_E_CUDA;
+}
+
+int32_t* fault_word() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fault) != cudaSuccess) return nullptr;
+    return static_cast<int32_t*>(p);
+}
+
+km_status device_info(DeviceInfo* out) {
+    static DeviceInfo cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) {
+        set_error("device ordinal %d out of range", dev);
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo& c = cache[dev];
+    if (c.device != dev) {
+        DeviceInfo n;
+        n.device = dev;
+        if ((e = cudaDeviceGetAttribute(&n.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&n.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&n.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+            return cuda_error(e, "cudaDeviceGetAttribute");
+        c = n;
+    }
+    *out = c;
+    return KM_OK;
+}
+
+}  // namespace km
+
+using namespace km;
+
+extern "C" {
+
+const char* km_status_string(km_status s) {
+    switch (s) {
+        case KM_OK: return "ok";
+        case KM_E_INVALID: return "invalid argument";
+        case KM_E_UNSUPPORTED: return "unsupported shape, alignment or device";
+        case KM_E_NOMEM: return "out of device memory";
+        case KM_E_CUDA: return "CUDA error";
+        case KM_E_TIMEOUT: return "bounded wait expired";
+    }
+    return "unknown status";
+}
+
+const char* km_last_error(void) { return g_err; }
+
+km_status km_assign(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                    int32_t* labels, float* mindist, void* stream) {
+    g_err[0] = 0;
+    if (!X || !C || !labels) {
+        set_error("km_assign: X, C and labels must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (!aligned(X, 16) || !aligned(C, 16) || !aligned(labels, 4) || (mindist && !aligned(mindist, 4))) {
+        set_error("km_assign: X and C must be 16-byte aligned, labels and mindist 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    Scratch scratch(st);
+    __half* chat = nullptr;
+    float* cnh = nullptr;
+    if (uses_tc(dtype, d)) {
+        KM_TRY(scratch.get(&chat, (size_t)(B * K * d), "rounded centroids"));
+        KM_TRY(scratch.get(&cnh, (size_t)(B * padded_k(K)), "centroid half norms"));
+        PhaseScope ph(st, KM_PHASE_PREP, 1);
+        KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, chat, cnh, st), "centroid preparation"));
+    }
+    return run_assign(X, dtype, C, chat, cnh, B, N, K, d, labels, mindist, dev, st);
+}
+
+km_status km_sort_labels(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* sorted_idx,
+                         int32_t* counts, int32_t* offsets, void* stream) {
+    g_err[0] = 0;
+    if (!labels || !sorted_idx || !counts) {
+        set_error("km_sort_labels: labels, sorted_idx and counts must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, 16, KM_F16));
+    if (!aligned(labels, 4) || !aligned(sorted_idx, 4) || !aligned(counts, 4) || (offsets && !aligned(offsets, 4))) {
+        set_error("km_sort_labels: arrays must be 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    Scratch scratch(st);
+    int32_t* a_sorted = nullptr;
+    unsigned char* work = nullptr;
+    KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
+    KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
+    PhaseScope ph(st, KM_PHASE_SORT, sort_kernel_launches(N, K, true));
+    return launched(launch_sort(labels, B, N, K, a_sorted, sorted_idx, counts, offsets, work, st), "label sort");
+}
+
+km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                    float* sums, int32_t* counts, float* C_out, void* stream) {
+    g_err[0] = 0;
+    if (!X || !labels || !sums || !counts || !C_out) {
+        set_error("km_update: X, labels, sums, counts and C_out must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (!aligned(X, 16) || !aligned(sums, 16) || !aligned(C_out, 4) || !aligned(labels, 4) || !aligned(counts, 4)) {
+        set_error("km_update: X and sums must be 16-byte aligned, the other arrays 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    Scratch scratch(st);
+    int32_t *a_sorted = nullptr, *sidx = nullptr;
+    unsigned char* work = nullptr;
+    KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
+    KM_TRY(scratch.get(&sidx, (size_t)(B * N), "sorted indices"));
+    KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
+    {
+        PhaseScope ph(st, KM_PHASE_OTHER, 0);
+        KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * (size_t)(B * K * d), st), "zero sums"));
+    }
+    {
+        PhaseScope ph(st, KM_PHASE_SORT, sort_kernel_launches(N, K, true));
+        KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, counts, nullptr, work, st), "label sort"));
+    }
+    {
+        PhaseScope ph(st, KM_PHASE_UPDATE, 1);
+        KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, st), "segmented update"));
+    }
+    PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
+    return launched(launch_finalize(sums, counts, B, K, d, C_out, dtype, nullptr, nullptr, st), "centroid finalize");
+}
+
+km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                   int iters, int32_t* labels, float* C_out, float* objective, void* stream) {
+    g_err[0] = 0;
+    if (!X || !C_init || !labels || !C_out) {
+        set_error("km_lloyd: X, C_init, labels and C_out must be non-null");
+        return KM_E_INVALID;
+    }
+    if (iters < 0) {
+        set_error("km_lloyd: iters must be >= 0");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (!aligned(X, 16) || !aligned(C_init, 16) || !aligned(C_out, 16) || !aligned(labels, 4) ||
+        (objective && !aligned(objective, 4))) {
+        set_error("km_lloyd: X, C_init and C_out must be 16-byte aligned, labels and objective 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaPointerAttributes pa;
+    cudaError_t e = cudaPointerGetAttributes(&pa, X);
+    if (e != cudaSuccess) return cuda_error(e, "cudaPointerGetAttributes(X)");
+    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged) {
+        set_error("km_lloyd: X must be device memory (host-resident X is not available in this build)");
+        return KM_E_UNSUPPORTED;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t ckd = (size_t)(B * K * d);
+    if (C_out != C_init)
+        KM_TRY(launched(cudaMemcpyAsync(C_out, C_init, sizeof(float) * ckd, cudaMemcpyDeviceToDevice, st),
+                        "copy C_init"));
+    if (iters == 0) return KM_OK;
+
+    Scratch scratch(st);
+    const bool tc = uses_tc(dtype, d);
+    __half* chat = nullptr;
+    float *cnh = nullptr, *mindist = nullptr, *sums = nullptr;
+    int32_t *a_sorted = nullptr, *sidx = nullptr, *counts = nullptr;
+    unsigned char* work = nullptr;
+    if (tc) {
+        KM_TRY(scratch.get(&chat, ckd, "rounded centroids"));
+        KM_TRY(scratch.get(&cnh, (size_t)(B * padded_k(K)), "centroid half norms"));
+    }
+    KM_TRY(scratch.get(&mindist, (size_t)(B * N), "minimum distances"));
+    KM_TRY(scratch.get(&sums, ckd, "cluster sums"));
+    KM_TRY(scratch.get(&counts, (size_t)(B * K), "cluster counts"));
+    KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
+    KM_TRY(scratch.get(&sidx, (size_t)(B * N), "sorted indices"));
+    KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
+
+    if (tc) {
+        PhaseScope ph(st, KM_PHASE_PREP, 1);
+        KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, chat, cnh, st), "centroid preparation"));
+    }
+    const int sort_launches = sort_kernel_launches(N, K, true);
+    for (int t = 0; t < iters; ++t) {
+        KM_TRY(run_assign(X, dtype, C_out, chat, cnh, B, N, K, d, labels, mindist, dev, st));
+        {
+            PhaseScope ph(st, KM_PHASE_OTHER, objective ? 1 : 0);
+            if (objective)
+                KM_TRY(launched(launch_objective(mindist, B, N, objective + (size_t)t * B, st), "objective"));
+            KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * ckd, st), "zero sums"));
+        }
+        {
+            PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
+            KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, counts, nullptr, work, st), "label sort"));
+        }
+        {
+            PhaseScope ph(st, KM_PHASE_UPDATE, 1);
+            KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, st), "segmented update"));
+        }
+        const bool prep_next = tc && t + 1 < iters;
+        PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
+        KM_TRY(launched(launch_finalize(sums, counts, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
+                                        prep_next ? cnh : nullptr, st),
+                        "centroid finalize"));
+    }
+    return KM_OK;
+}
+
+void km_set_chunk_rows(int64_t rows) { (void)rows; }
+
+void km_trace_enable(int on) { g_trace_on.store(on != 0); }
+
+km_status km_trace_read(double* ms, int64_t* launches, int nphases) {
+    g_err[0] = 0;
+    std::vector<TraceRec> recs;
+    {
+        std::lock_guard<std::mutex> lk(g_trace_mu);
+        recs.swap(g_trace);
+    }
+    for (int p = 0; p < nphases; ++p) {
+        if (ms) ms[p] = 0.0;
+        if (launches) launches[p] = 0;
+    }
+    km_status st = KM_OK;
+    for (const TraceRec& r : recs) {
+        float t = 0.f;
+        cudaError_t e = cudaEventSynchronize(r.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+        if (e != cudaSuccess && st == KM_OK) st = cuda_error(e, "trace event");
+        if (r.phase < nphases) {
+            if (ms) ms[r.phase] += t;
+            if (launches) launches[r.phase] += r.launches;
+        }
+    }
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    for (const TraceRec& r : recs) {
+        g_event_pool.push_back(r.a);
+        g_event_pool.push_back(r.b);
+    }
+    return st;
+}
+
+km_status km_device_fault(int32_t* code, void* stream) {
+    g_err[0] = 0;
+    if (!code) {
+        set_error("km_device_fault: code must be non-null");
+        return KM_E_INVALID;
+    }
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_error(e, "cudaStreamSynchronize");
+    int32_t v = 0, zero = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_fault, sizeof(v))) != cudaSuccess) return cuda_error(e, "read fault word");
+    if ((e = cudaMemcpyToSymbol(g_fault, &zero, sizeof(zero))) != cudaSuccess) return cuda_error(e, "clear fault word");
+    *code = v;
+    return KM_OK;
+}
+
+}  // extern "C"

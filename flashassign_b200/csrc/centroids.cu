@@ -1,0 +1,120 @@
+// Centroid-side kernels of the Lloyd iteration:
+//  * preparation for the assignment: round the fp32 centroids to the dtype of
+//    X and take half their squared norms (the ||c||^2 term of the expansion
+//    ||x - c||^2 = ||x||^2 + ||c||^2 - 2 x.c, papernotes.org "Flash-KMeans"
+//    page, 关键设计 1);
+//  * finalisation of the update: c_k = s_k / n_k, an empty cluster keeping its
+//    previous centroid (the flowchart's C_new on the same page, 整体框架);
+//  * the per-batch objective sum of the minimum distances.
+// All three are tiny next to the assignment and the gather; one warp per
+// centroid row keeps them coalesced.
+#include "km_internal.cuh"
+
+#include <cmath>
+
+namespace km {
+namespace {
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, int64_t Kp, int64_t d, int dtype,
+                            __half* __restrict__ chat, float* __restrict__ cnh) {
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    if (row >= B * Kp) return;
+    const int64_t b = row / Kp, k = row % Kp;
+    if (k >= K) {
+        if (lane == 0) cnh[row] = INFINITY;
+        return;
+    }
+    const int64_t base = (b * K + k) * d;
+    double acc = 0.0;
+    for (int64_t j = lane; j < d; j += 32) {
+        float v = C[base + j];
+        if (dtype == KM_F16) {
+            const __half h = __float2half_rn(v);
+            if (chat) chat[base + j] = h;
+            v = __half2float(h);
+        }
+        acc += (double)v * (double)v;
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) cnh[row] = (float)(0.5 * acc);
+}
+
+__global__ void finalize_kernel(const float* __restrict__ sums, const int32_t* __restrict__ counts, int64_t B,
+                                int64_t K, int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype,
+                                __half* __restrict__ chat, float* __restrict__ cnh) {
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    if (row >= B * K) return;
+    const int64_t b = row / K, k = row % K;
+    const int32_t n = counts[row];
+    const float fn = (float)n;
+    const int64_t base = row * d;
+    double acc = 0.0;
+    for (int64_t j = lane; j < d; j += 32) {
+        float v;
+        if (n > 0) {
+            v = sums[base + j] / fn;
+            C_out[base + j] = v;
+        } else {
+            v = C_out[base + j];
+        }
+        if (dtype == KM_F16) {
+            const __half h = __float2half_rn(v);
+            if (chat) chat[base + j] = h;
+            v = __half2float(h);
+        }
+        acc += (double)v * (double)v;
+    }
+    if (cnh) {
+        acc = warp_sum(acc);
+        if (lane == 0) cnh[b * Kp + k] = (float)(0.5 * acc);
+    }
+}
+
+__global__ void objective_kernel(const float* __restrict__ mindist, int64_t N, float* __restrict__ objective) {
+    const int64_t b = blockIdx.x;
+    double acc = 0.0;
+    for (int64_t i = threadIdx.x; i < N; i += blockDim.x) acc += (double)mindist[b * N + i];
+    acc = warp_sum(acc);
+    __shared__ double part[32];
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x / 32] = acc;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        double v = threadIdx.x < blockDim.x / 32 ? part[threadIdx.x] : 0.0;
+        v = warp_sum(v);
+        if (threadIdx.x == 0) objective[b] = (float)v;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
+                                  float* cnh, cudaStream_t st) {
+    const int64_t Kp = padded_k(K);
+    const int64_t rows = B * Kp;
+    const int warps = 8;
+    prep_kernel<<<(unsigned)ceil_div(rows, warps), warps * 32, 0, st>>>(C, B, K, Kp, d, dtype, chat, cnh);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float* sums, const int32_t* counts, int64_t B, int64_t K, int64_t d, float* C_out,
+                            int dtype, __half* chat, float* cnh, cudaStream_t st) {
+    const int warps = 8;
+    finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(sums, counts, B, K, padded_k(K), d,
+                                                                            C_out, dtype, chat, cnh);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_objective(const float* mindist, int64_t B, int64_t N, float* objective, cudaStream_t st) {
+    objective_kernel<<<(unsigned)B, 1024, 0, st>>>(mindist, N, objective);
+    return cudaGetLastError();
+}
+
+}  // namespace km

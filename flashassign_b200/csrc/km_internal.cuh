@@ -1,0 +1,72 @@
+// Internal declarations shared by the libkm translation units: launchers,
+// the per-thread error detail, and the device fault word.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/km.h"
+
+namespace km {
+
+// Per-thread error detail (km_last_error).
+void set_error(const char* fmt, ...);
+km_status cuda_error(cudaError_t e, const char* what);
+
+// Device fault word: kernels write a non-zero code when a bounded wait expires.
+enum : int32_t { FAULT_NONE = 0, FAULT_PIPELINE_TIMEOUT = 1 };
+int32_t* fault_word();  // device address of the word on the current device
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Tile width of the assignment kernels along K; the half-norm array is padded
+// to a multiple of it with +inf so that padded columns never win.
+constexpr int kAssignTileK = 128;
+inline int64_t padded_k(int64_t K) { return ceil_div(K, kAssignTileK) * kAssignTileK; }
+
+struct DeviceInfo {
+    int device = -1;
+    int sms = 0;
+    int cc_major = 0, cc_minor = 0;
+};
+km_status device_info(DeviceInfo* out);
+
+// ---- launchers (all asynchronous on `st`) ----
+// Centroid preparation for the assignment: chat = fp16(C) (RNE) and
+// cnh[b][k] = 0.5 * ||chat_k||^2 for k < K, +inf for K <= k < padded_k(K).
+// For fp32 runs chat may be null (the fp32 kernel reads C directly) and cnh
+// holds 0.5 * ||C_k||^2.
+cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
+                                  float* cnh, cudaStream_t st);
+
+// C_out[b][k] = sums / counts where counts > 0 (else unchanged); when chat or
+// cnh is non-null, also prepares the next assignment's centroids from C_out.
+cudaError_t launch_finalize(const float* sums, const int32_t* counts, int64_t B, int64_t K, int64_t d,
+                            float* C_out, int dtype, __half* chat, float* cnh, cudaStream_t st);
+
+// Tensor-core assignment (fp16, 64 <= d <= 128).  Returns cudaErrorNotSupported
+// for shapes it does not take.
+bool assign_tc_supported(int64_t d, int dtype);
+cudaError_t launch_assign_tc(const __half* X, const __half* chat, const float* cnh, int64_t B, int64_t N, int64_t K,
+                             int64_t d, int32_t* labels, float* mindist, int sms, cudaStream_t st);
+
+// CUDA-core assignment for every supported shape (fp32 inputs, and fp16
+// shapes outside the tensor-core kernel's range): direct-difference distances.
+cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
+                               int32_t* labels, float* mindist, cudaStream_t st);
+
+// Stable LSD radix argsort of labels in [0, K).  Scratch: sort_scratch_bytes().
+size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K);
+int sort_kernel_launches(int64_t N, int64_t K, bool with_counts);
+cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* a_sorted,
+                        int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st);
+
+// Segmented gather-reduce over the sorted order (sums must be zeroed first).
+cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
+                               int64_t B, int64_t N, int64_t K, int64_t d, float* sums, cudaStream_t st);
+
+// objective[b] = sum_i mindist[b][i] (fp32, one block per batch).
+cudaError_t launch_objective(const float* mindist, int64_t B, int64_t N, float* objective, cudaStream_t st);
+
+}  // namespace km

@@ -1,0 +1,219 @@
+// Device argsort of the 1-D label vector, the first half of Sort-Inverse
+// Update (papernotes.org "Flash-KMeans" page, 关键设计 2: only the labels are
+// sorted -- a radix sort giving sorted_idx and the sorted labels -- and the
+// point matrix X is never moved).
+//
+// Stable least-significant-digit radix sort, batched over B (grid.y), with
+// digits of at most 8 bits: ceil(log2 K) bits in ceil(bits/8) passes (K=1024:
+// two 5-bit passes; K=65536: two 8-bit passes).  Each pass is
+//   1. a per-tile digit histogram (2048 keys per CTA),
+//   2. an exclusive scan over (digit, tile) per batch,
+//   3. a scatter in which each warp ranks its keys with __match_any_sync and
+//      the warps of a tile are combined by a per-digit scan, so equal digits
+//      keep their input order (stability).
+// The segment offsets and counts then follow from the sorted labels without
+// any atomics: position p starts label k exactly when a[p-1] < k <= a[p].
+#include "km_internal.cuh"
+
+namespace km {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kItems = 8;
+constexpr int kTile = kThreads * kItems;  // 2048 keys per CTA
+constexpr int kWarps = kThreads / 32;
+
+struct Plan {
+    int passes = 0;
+    int shift[4] = {0, 0, 0, 0};
+    int bits[4] = {0, 0, 0, 0};
+    int64_t tiles = 0;
+};
+
+Plan make_plan(int64_t N, int64_t K) {
+    int total = 1;
+    while (total < 31 && (int64_t(1) << total) < K) ++total;
+    Plan p;
+    p.passes = (total + 7) / 8;
+    const int per = (total + p.passes - 1) / p.passes;
+    int shift = 0;
+    for (int i = 0; i < p.passes; ++i) {
+        p.shift[i] = shift;
+        p.bits[i] = (total - shift < per) ? total - shift : per;
+        shift += p.bits[i];
+    }
+    p.tiles = ceil_div(N, kTile);
+    return p;
+}
+
+__global__ void __launch_bounds__(kThreads) radix_hist_kernel(const int32_t* __restrict__ keys, int64_t N, int shift,
+                                                              int bits, int64_t T, int32_t* __restrict__ hist) {
+    __shared__ int s[256];
+    const int64_t b = blockIdx.y, tile = blockIdx.x;
+    const int bins = 1 << bits, mask = bins - 1;
+    for (int t = threadIdx.x; t < bins; t += kThreads) s[t] = 0;
+    __syncthreads();
+    const int32_t* kb = keys + b * N;
+#pragma unroll
+    for (int k = 0; k < kItems; ++k) {
+        const int64_t i = tile * kTile + k * kThreads + threadIdx.x;
+        if (i < N) atomicAdd(&s[(kb[i] >> shift) & mask], 1);
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < bins; t += kThreads) hist[(b * bins + t) * T + tile] = s[t];
+}
+
+// In-place exclusive scan of `len` ints per batch (one 1024-thread block per batch).
+__global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t* __restrict__ data, int64_t len) {
+    __shared__ int warp_tot[32];
+    __shared__ int carry_s;
+    int32_t* p = data + (int64_t)blockIdx.x * len;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    if (threadIdx.x == 0) carry_s = 0;
+    __syncthreads();
+    for (int64_t base = 0; base < len; base += 1024) {
+        const int64_t idx = base + threadIdx.x;
+        const int v = idx < len ? p[idx] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_tot[w] = incl;
+        __syncthreads();
+        if (w == 0) {
+            int t = warp_tot[lane];
+            int ti = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, ti, o);
+                if (lane >= o) ti += y;
+            }
+            warp_tot[lane] = ti - t;  // exclusive prefix of the warp totals
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        if (idx < len) p[idx] = carry + warp_tot[w] + incl - v;
+        __syncthreads();
+        if (threadIdx.x == 1023) carry_s = carry + warp_tot[w] + incl;
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* __restrict__ keys_in,
+                                                                 const int32_t* __restrict__ vals_in,
+                                                                 int32_t* __restrict__ keys_out,
+                                                                 int32_t* __restrict__ vals_out, int64_t N, int shift,
+                                                                 int bits, int64_t T,
+                                                                 const int32_t* __restrict__ offs) {
+    __shared__ int wh[kWarps][256];
+    const int64_t b = blockIdx.y, tile = blockIdx.x;
+    const int bins = 1 << bits, mask = bins - 1;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int t = threadIdx.x; t < kWarps * 256; t += kThreads) (&wh[0][0])[t] = 0;
+    __syncthreads();
+
+    const uint32_t lt = (1u << lane) - 1u;
+    const int64_t base = tile * kTile + (int64_t)w * (kItems * 32);
+    int key[kItems], val[kItems], rank[kItems];
+#pragma unroll
+    for (int s = 0; s < kItems; ++s) {
+        const int64_t i = base + s * 32 + lane;
+        const bool valid = i < N;
+        key[s] = valid ? keys_in[b * N + i] : 0;
+        val[s] = valid ? (vals_in ? vals_in[b * N + i] : (int)i) : 0;
+        const int dig = valid ? ((key[s] >> shift) & mask) : 256;  // 256: never a real digit
+        const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+        const int cnt = valid ? wh[w][dig] : 0;
+        rank[s] = cnt + __popc(peers & lt);
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) wh[w][dig] = cnt + __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    if (threadIdx.x < bins) {
+        int run = 0;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) {
+            const int t = wh[ww][threadIdx.x];
+            wh[ww][threadIdx.x] = run;
+            run += t;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int s = 0; s < kItems; ++s) {
+        const int64_t i = base + s * 32 + lane;
+        if (i < N) {
+            const int dig = (key[s] >> shift) & mask;
+            const int64_t pos = (int64_t)offs[(b * bins + dig) * T + tile] + wh[w][dig] + rank[s];
+            keys_out[b * N + pos] = key[s];
+            vals_out[b * N + pos] = val[s];
+        }
+    }
+}
+
+// offsets[b][k] = first sorted position holding a label >= k (offsets[b][K] = N).
+__global__ void seg_bounds_kernel(const int32_t* __restrict__ a, int64_t N, int64_t K, int32_t* __restrict__ offsets) {
+    const int64_t b = blockIdx.y;
+    const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p > N) return;
+    // clamped so that out-of-range labels cannot write outside offsets
+    const int64_t prev = p == 0 ? -1 : min(max((int64_t)a[b * N + p - 1], (int64_t)-1), K);
+    const int64_t cur = p == N ? K : min(max((int64_t)a[b * N + p], (int64_t)-1), K);
+    for (int64_t k = prev + 1; k <= cur; ++k) offsets[b * (K + 1) + k] = (int32_t)p;
+}
+
+__global__ void counts_kernel(const int32_t* __restrict__ offsets, int64_t B, int64_t K, int32_t* __restrict__ counts) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= B * K) return;
+    const int64_t b = t / K, k = t % K;
+    counts[t] = offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
+}
+
+}  // namespace
+
+int sort_kernel_launches(int64_t N, int64_t K, bool with_counts) {
+    return 3 * make_plan(N, K).passes + 1 + (with_counts ? 1 : 0);
+}
+
+size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K) {
+    const Plan p = make_plan(N, K);
+    size_t bytes = 0;
+    bytes += 2 * sizeof(int32_t) * (size_t)(B * N);     // ping-pong keys and values
+    bytes += sizeof(int32_t) * (size_t)(B * 256 * p.tiles);  // tile histograms
+    bytes += sizeof(int32_t) * (size_t)(B * (K + 1));   // offsets when the caller passes none
+    return bytes;
+}
+
+cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* a_sorted,
+                        int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st) {
+    const Plan p = make_plan(N, K);
+    int32_t* tmp_k = (int32_t*)scratch;
+    int32_t* tmp_v = tmp_k + B * N;
+    int32_t* hist = tmp_v + B * N;
+    int32_t* offs_scratch = hist + B * 256 * p.tiles;
+    if (!offsets) offsets = offs_scratch;
+
+    const int32_t* in_k = labels;
+    const int32_t* in_v = nullptr;
+    const dim3 grid((unsigned)p.tiles, (unsigned)B);
+    for (int i = 0; i < p.passes; ++i) {
+        const bool to_final = ((p.passes - 1 - i) % 2) == 0;
+        int32_t* out_k = to_final ? a_sorted : tmp_k;
+        int32_t* out_v = to_final ? sorted_idx : tmp_v;
+        const int bins = 1 << p.bits[i];
+        radix_hist_kernel<<<grid, kThreads, 0, st>>>(in_k, N, p.shift[i], p.bits[i], p.tiles, hist);
+        exclusive_scan_kernel<<<(unsigned)B, 1024, 0, st>>>(hist, (int64_t)bins * p.tiles);
+        radix_scatter_kernel<<<grid, kThreads, 0, st>>>(in_k, in_v, out_k, out_v, N, p.shift[i], p.bits[i], p.tiles,
+                                                        hist);
+        in_k = out_k;
+        in_v = out_v;
+    }
+    seg_bounds_kernel<<<dim3((unsigned)ceil_div(N + 1, 256), (unsigned)B), 256, 0, st>>>(a_sorted, N, K, offsets);
+    if (counts) counts_kernel<<<(unsigned)ceil_div(B * K, 256), 256, 0, st>>>(offsets, B, K, counts);
+    return cudaGetLastError();
+}
+
+}  // namespace km

@@ -1,0 +1,201 @@
+// Sort-Inverse Update, the gather-reduce half (papernotes.org "Flash-KMeans"
+// page, 关键设计 2).  After the labels are argsorted, each CTA takes a fixed run
+// of B_N consecutive sorted positions, splits it where the sorted label
+// changes (the intervals [u, v) of the page), gathers the rows of X through
+// sorted_idx, reduces each interval on chip, and touches global memory
+// atomically only for intervals that may continue into a neighbouring CTA.
+// The page's count of O((K + ceil(N / B_N)) d) atomic additions is met
+// exactly: at most two intervals per CTA are added atomically; every other
+// interval is a whole cluster owned by this CTA and is written with a plain
+// store.  Cluster counts come from the sort's segment offsets (exact
+// integers), so no counter atomics are needed at all.
+//
+// Layout of a CTA (16-byte chunks of a row per thread):
+//   tpr = d * sizeof(T) / 16 threads cover one row; G = 256 / tpr row-lanes;
+//   row-lane g walks 16 consecutive sorted positions (B_N = 16 G), issuing
+//   four independent 16-byte gathers at a time and keeping a running fp32
+//   partial sum in registers.  A label change inside the walk ends a piece:
+//   pieces strictly inside the walk are whole clusters and are stored at once;
+//   the first and last piece of each walk go to shared memory, where one pass
+//   in position order joins equal labels across row-lanes and decides, from
+//   the labels just outside the CTA's run, whether each joined interval is the
+//   whole cluster (plain store) or a part of it (fp32 vector atomic add).
+#include "km_internal.cuh"
+
+namespace km {
+namespace {
+
+constexpr int kRowsPerLane = 16;
+constexpr int kUnroll = 4;
+
+template <typename T>
+struct Chunk;
+template <>
+struct Chunk<__half> {
+    static constexpr int kElems = 8;
+    static __device__ __forceinline__ void add(float* acc, const uint4& v) {
+        const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            acc[2 * e] += f.x;
+            acc[2 * e + 1] += f.y;
+        }
+    }
+};
+template <>
+struct Chunk<float> {
+    static constexpr int kElems = 4;
+    static __device__ __forceinline__ void add(float* acc, const uint4& v) {
+        acc[0] += __uint_as_float(v.x);
+        acc[1] += __uint_as_float(v.y);
+        acc[2] += __uint_as_float(v.z);
+        acc[3] += __uint_as_float(v.w);
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, const int32_t* __restrict__ a_sorted,
+                                                     const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
+                                                     int64_t d, int tpr, int G, float* __restrict__ sums) {
+    constexpr int E = Chunk<T>::kElems;
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int BN = G * kRowsPerLane;
+    float* head_vec = reinterpret_cast<float*>(smem);    // [G][d]
+    float* tail_vec = head_vec + (size_t)G * d;          // [G][d]
+    int* s_lab = reinterpret_cast<int*>(tail_vec + (size_t)G * d);  // [BN]
+    int* s_idx = s_lab + BN;                             // [BN]
+    int* head_lab = s_idx + BN;                          // [G]
+    int* tail_lab = head_lab + G;                        // [G]
+
+    const int64_t b = blockIdx.y;
+    const int64_t p0 = (int64_t)blockIdx.x * BN;
+    const int64_t pend = min(p0 + BN, N);
+    const int n = (int)(pend - p0);
+    const int32_t* ab = a_sorted + b * N;
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+        s_lab[t] = ab[p0 + t];
+        s_idx[t] = sorted_idx[b * N + p0 + t];
+    }
+    __syncthreads();
+
+    const int g = threadIdx.x / tpr, c = threadIdx.x % tpr;
+    const int r0 = g * kRowsPerLane, r1 = min(r0 + kRowsPerLane, n);
+    float* sums_b = sums + b * K * d + (int64_t)c * E;
+    if (r0 >= r1) {
+        if (c == 0) head_lab[g] = tail_lab[g] = -1;
+    } else {
+        const T* xb = X + b * N * d + (int64_t)c * E;
+        float acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
+        int cur = s_lab[r0];
+        int piece = 0;
+        for (int r = r0; r < r1; r += kUnroll) {
+            uint4 v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u)
+                if (r + u < r1) v[u] = __ldg(reinterpret_cast<const uint4*>(xb + (int64_t)s_idx[r + u] * d));
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (r + u >= r1) break;
+                const int lab = s_lab[r + u];
+                if (lab != cur) {
+                    if (piece == 0) {
+                        if (c == 0) head_lab[g] = cur;
+#pragma unroll
+                        for (int e = 0; e < E; ++e) head_vec[(size_t)g * d + c * E + e] = acc[e];
+                    } else if (cur >= 0 && cur < K) {  // a whole cluster inside this walk
+#pragma unroll
+                        for (int e = 0; e < E; e += 4)
+                            *reinterpret_cast<float4*>(sums_b + (int64_t)cur * d + e) =
+                                make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                    }
+                    ++piece;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+                    cur = lab;
+                }
+                Chunk<T>::add(acc, v[u]);
+            }
+        }
+        if (piece == 0) {  // the whole walk is one label: a head piece with no tail
+            if (c == 0) {
+                head_lab[g] = cur;
+                tail_lab[g] = -1;
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) head_vec[(size_t)g * d + c * E + e] = acc[e];
+        } else {
+            if (c == 0) tail_lab[g] = cur;
+#pragma unroll
+            for (int e = 0; e < E; ++e) tail_vec[(size_t)g * d + c * E + e] = acc[e];
+        }
+    }
+    __syncthreads();
+
+    // Join the boundary pieces in position order; one thread per 4 dims.
+    const int j4 = threadIdx.x * 4;
+    if (j4 >= d) return;
+    const int before = p0 > 0 ? ab[p0 - 1] : -1;   // label just before the run
+    const int after = pend < N ? ab[pend] : -1;    // label just after it
+    int run_lab = -1;
+    bool run_first = false;
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    bool seen = false;
+    auto emit = [&](int lab, float4 v, bool first, bool last) {
+        if (lab < 0 || lab >= K) return;
+        const bool shared_left = first && before == lab;
+        const bool shared_right = last && after == lab;
+        float* dst = sums + (b * K + lab) * d + j4;
+        if (shared_left || shared_right) {
+            atomicAdd(reinterpret_cast<float4*>(dst), v);
+        } else {
+            *reinterpret_cast<float4*>(dst) = v;
+        }
+    };
+    for (int gg = 0; gg < G; ++gg) {
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const int lab = which == 0 ? head_lab[gg] : tail_lab[gg];
+            if (lab < 0) continue;
+            const float4 v = *reinterpret_cast<const float4*>((which == 0 ? head_vec : tail_vec) + (size_t)gg * d + j4);
+            if (seen && lab == run_lab) {
+                run.x += v.x; run.y += v.y; run.z += v.z; run.w += v.w;
+            } else {
+                if (seen) emit(run_lab, run, run_first, false);
+                run_first = !seen;
+                seen = true;
+                run_lab = lab;
+                run = v;
+            }
+        }
+    }
+    if (seen) emit(run_lab, run, run_first, true);
+}
+
+template <typename T>
+cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sorted_idx, int64_t B, int64_t N,
+                     int64_t K, int64_t d, float* sums, cudaStream_t st) {
+    const int tpr = (int)(d * (int64_t)sizeof(T) / 16);
+    const int G = 256 / tpr;
+    const int BN = G * kRowsPerLane;
+    const size_t smem = sizeof(float) * 2 * (size_t)G * d + sizeof(int) * (2 * (size_t)BN + 2 * (size_t)G);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(update_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B);
+    update_kernel<T><<<grid, G * tpr, smem, st>>>((const T*)X, a_sorted, sorted_idx, N, K, d, tpr, G, sums);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
+                               int64_t B, int64_t N, int64_t K, int64_t d, float* sums, cudaStream_t st) {
+    if (dtype == KM_F16) return launch_t<__half>(X, a_sorted, sorted_idx, B, N, K, d, sums, st);
+    return launch_t<float>(X, a_sorted, sorted_idx, B, N, K, d, sums, st);
+}
+
+}  // namespace km

@@ -1,0 +1,169 @@
+/*
+ * km.h -- C ABI of libkm.so: one batched exact Lloyd k-means iteration on an
+ * NVIDIA B200 (sm_100a), in hand-written CUDA.
+ *
+ * The method is Flash-KMeans as described on the papernotes.org page
+ * "Flash-KMeans: Fast and Memory-Efficient Exact K-Means" (method section
+ * 方法详解): an iteration is an assignment step (FlashAssign, 关键设计 1) and
+ * an update step (Sort-Inverse Update, 关键设计 2), repeated (整体框架 and its
+ * flowchart).  The result is exactly Lloyd's k-means; only the data movement
+ * differs (7minutos.es article, opening section).
+ *
+ * Conventions shared by every entry point
+ *   - All arrays are dense and row-major.  X is [B, N, d] in `dtype`;
+ *     centroids C, C_init, C_out and sums are [B, K, d] fp32; labels, mindist
+ *     and sorted_idx are [B, N]; counts is [B, K]; offsets is [B, K + 1].
+ *     Labels and sorted indices are 0-based and index within their batch.
+ *   - The B problems are independent; each has its own K centroids.
+ *   - Pointers are device pointers unless stated otherwise; the caller owns
+ *     (allocates and frees) every array it passes.  Scratch memory is taken
+ *     stream-ordered (cudaMallocAsync) on `stream` and released before return
+ *     on the same stream.  No state survives a call except a per-device cache
+ *     of the capability check.
+ *   - `stream` is a cudaStream_t (NULL means the legacy default stream).
+ *     Every call is asynchronous on it: results are ready once the stream is
+ *     synchronised.  Argument errors return before any work is enqueued.
+ *   - Supported: B >= 1, N >= 1, K >= 1, B*N < 2^31, K < 2^24, 1 <= d <= 512,
+ *     d * sizeof(dtype) a multiple of 16 bytes, X and C 16-byte aligned,
+ *     every other array 4-byte aligned, a device of compute capability 10.0.
+ *     Anything else returns KM_E_UNSUPPORTED (KM_E_INVALID for null pointers
+ *     and non-positive sizes).  There is no CPU fallback.
+ *   - Inputs must be finite; non-finite values are outside the contract.
+ */
+#ifndef KM_H
+#define KM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KM_API __attribute__((visibility("default")))
+#else
+#define KM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { KM_F32 = 0, KM_F16 = 1 } km_dtype;
+
+typedef enum {
+    KM_OK = 0,
+    KM_E_INVALID = 1,     /* null pointer, non-positive size, unknown dtype */
+    KM_E_UNSUPPORTED = 2, /* shape, alignment or device outside the supported range */
+    KM_E_NOMEM = 3,       /* scratch allocation failed */
+    KM_E_CUDA = 4,        /* a CUDA call or kernel launch failed */
+    KM_E_TIMEOUT = 5      /* a bounded wait expired (see km_device_fault) */
+} km_status;
+
+/*
+ * Assignment step (FlashAssign; papernotes.org page, 关键设计 1).
+ * For every point x_i of every batch:
+ *     labels[b][i]  = argmin_k ||x_i - c_k||^2, the lowest k among equal distances,
+ *     mindist[b][i] = that minimum squared distance (clamped at 0).
+ * The distance is expanded as ||x||^2 + ||c||^2 - 2 x.c; the N x K distance
+ * matrix is never written to memory.  The centroids are first rounded
+ * (round-to-nearest-even) to `dtype`, and x.c is accumulated in fp32 on the
+ * tensor cores (fp16) or in fp32 on the CUDA cores (fp32 inputs).
+ *   X       [B, N, d] dtype, device.     C [B, K, d] fp32, device.
+ *   labels  [B, N] int32, device, written.
+ *   mindist [B, N] fp32, device, written; may be NULL.
+ */
+KM_API km_status km_assign(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                    int32_t* labels, float* mindist, void* stream);
+
+/*
+ * Label argsort (papernotes.org page, 关键设计 2: the labels alone are sorted;
+ * X is never permuted).  A stable device LSD radix sort of each batch's labels:
+ *   sorted_idx[b][p] = index of the point at sorted position p (ascending
+ *                      label, ties by ascending point index; unique),
+ *   counts[b][k]     = number of points with label k,
+ *   offsets[b][k]    = first sorted position of label k (offsets[b][K] = N).
+ * Labels must lie in [0, K); others give undefined (but in-bounds) output.
+ *   labels [B, N] int32, device.  sorted_idx [B, N] int32, device, written.
+ *   counts [B, K] int32, device, written.  offsets [B, K+1] int32, device,
+ *   written; may be NULL.
+ */
+KM_API km_status km_sort_labels(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* sorted_idx,
+                         int32_t* counts, int32_t* offsets, void* stream);
+
+/*
+ * Update step (Sort-Inverse Update; papernotes.org page, 关键设计 2).
+ * Sorts the labels, then each CTA walks a fixed run of sorted positions,
+ * gathers the rows of X through the sorted indices, reduces each cluster's
+ * rows on chip, and adds to global memory atomically only for the clusters
+ * that cross its run boundaries:
+ *   sums[b][k]   = sum of the rows labelled k (fp32 accumulation),
+ *   counts[b][k] = their number,
+ *   C_out[b][k]  = sums / counts if counts > 0, else unchanged.
+ * C_out is in/out: on entry it holds the previous centroids (an empty cluster
+ * keeps its centroid, bit for bit); it must not alias X, sums or labels.
+ *   X [B, N, d] dtype, device.  labels [B, N] int32 in [0, K), device.
+ *   sums [B, K, d] fp32, device, written.  counts [B, K] int32, device, written.
+ *   C_out [B, K, d] fp32, device, read and written.
+ */
+KM_API km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                    float* sums, int32_t* counts, float* C_out, void* stream);
+
+/*
+ * `iters` Lloyd iterations (assign, sort, update), all enqueued on `stream`
+ * with no host synchronisation inside the loop (papernotes.org page, 整体框架:
+ * the loop returns to the assignment until the iteration budget is spent).
+ *   X        [B, N, d] dtype, device memory; or pinned host memory
+ *            (cudaHostAlloc / cudaHostRegister), in which case it is streamed
+ *            to the device in chunks of rows with copies overlapped with the
+ *            computation (papernotes.org page, 关键设计 3).
+ *   C_init   [B, K, d] fp32, device.  C_out [B, K, d] fp32, device, written
+ *            (may equal C_init).
+ *   labels   [B, N] int32: the assignment of the LAST iteration, made against
+ *            the centroids before its update; device memory, or pinned host
+ *            memory when X is host memory.
+ *   objective [iters, B] fp32, device, may be NULL: per iteration and batch,
+ *            the sum of the assignment's minimum distances.
+ * iters = 0 copies C_init to C_out.
+ */
+KM_API km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                   int iters, int32_t* labels, float* C_out, float* objective, void* stream);
+
+/* Rows per chunk used by km_lloyd for host-resident X (0 restores the default, 2^23). */
+KM_API void km_set_chunk_rows(int64_t rows);
+
+/*
+ * Tracing.  While enabled (process-wide), every call records a CUDA event pair
+ * on its stream around each kernel phase it enqueues and counts the kernels it
+ * launches.  km_trace_read waits for the recorded events, returns for each
+ * phase the summed GPU time in milliseconds and the number of kernel
+ * launches, and clears the record.  Phases: see km_phase.  Arrays have
+ * `nphases` entries (at most KM_NUM_PHASES are filled); either may be NULL.
+ */
+typedef enum {
+    KM_PHASE_PREP = 0,     /* centroid rounding and half norms */
+    KM_PHASE_ASSIGN = 1,   /* FlashAssign */
+    KM_PHASE_SORT = 2,     /* label argsort, segment offsets, counts */
+    KM_PHASE_UPDATE = 3,   /* segmented gather-reduce of the sums */
+    KM_PHASE_FINALIZE = 4, /* centroid division (and next preparation) */
+    KM_PHASE_OTHER = 5,    /* zeroing of sums, objective, copies */
+    KM_NUM_PHASES = 6
+} km_phase;
+KM_API void km_trace_enable(int on);
+KM_API km_status km_trace_read(double* ms, int64_t* launches, int nphases);
+
+/* Static description of a status code. */
+KM_API const char* km_status_string(km_status s);
+
+/* Detail of the last error on the calling host thread ("" if none). */
+KM_API const char* km_last_error(void);
+
+/*
+ * Reads and clears the device fault word of the current device: a kernel
+ * whose bounded wait expired records a non-zero code there instead of hanging
+ * (1: a TMA or MMA pipeline wait timed out).  Synchronises `stream`.
+ * Returns KM_OK with *code = 0 when no fault was recorded.
+ */
+KM_API km_status km_device_fault(int32_t* code, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KM_H */

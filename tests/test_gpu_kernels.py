@@ -1,0 +1,227 @@
+"""Parity of each CUDA kernel with the CPU oracle on small seeded inputs, through the C ABI.
+
+Sizes span several tiles with ragged tails: point units of 256 rows, centroid
+tiles of 128 columns, 16-byte row chunks; shapes at and around those edges,
+plus the degenerate cases of the method (K = 1, one cluster holding every
+point, empty clusters, duplicate centroids, exact distance ties).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import check_centroids, check_labels, check_sort
+
+torch = pytest.importorskip("torch")
+import flashassign_b200 as km  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+def cuda(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def run_assign(X, C):
+    lab, md = km.assign(cuda(X), cuda(C))
+    torch.cuda.synchronize()
+    assert km.device_fault() == 0
+    return lab.cpu().numpy(), md.cpu().numpy()
+
+
+ASSIGN_SHAPES = [
+    # (B, N, K, d, dtype)
+    (1, 1, 1, 128, "f16"),
+    (1, 127, 2, 128, "f16"),
+    (2, 128, 8, 128, "f16"),
+    (1, 129, 127, 128, "f16"),
+    (3, 255, 128, 128, "f16"),
+    (2, 256, 129, 128, "f16"),
+    (2, 257, 255, 128, "f16"),
+    (3, 1000, 300, 128, "f16"),
+    (2, 777, 257, 64, "f16"),
+    (2, 600, 200, 96, "f16"),
+    (2, 500, 100, 16, "f16"),    # below the tensor-core range: CUDA-core kernel
+    (2, 300, 50, 256, "f16"),    # above it
+    (1, 4096, 8, 16, "f32"),
+    (2, 1000, 300, 128, "f32"),
+    (2, 129, 33, 4, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,N,K,d,dt", ASSIGN_SHAPES)
+def test_assign_matches_oracle(B, N, K, d, dt):
+    w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, ncomp=max(1, K // 2), sigma=0.3, seed=1000 + N + K + d)
+    X = synth.points(w)
+    C = synth.init_centroids(w, X) if K <= N else np.random.default_rng(1).standard_normal((B, K, d)).astype(
+        np.float32)
+    lab, md = run_assign(X, C)
+    check_labels(X, C, lab, md)
+
+
+@pytest.mark.parametrize("dt", ["f16", "f32"])
+def test_assign_ties_go_to_the_lowest_index(dt):
+    # integer coordinates and duplicate centroids give exact ties in every precision
+    rng = np.random.default_rng(11)
+    B, N, K, d = 2, 700, 260, 128 if dt == "f16" else 16
+    npdt = np.float16 if dt == "f16" else np.float32
+    X = rng.integers(-2, 3, (B, N, d)).astype(npdt)
+    base = rng.integers(-2, 3, (B, 40, d)).astype(np.float32)
+    C = base[:, rng.integers(0, 40, K)]  # many duplicates, at indices far apart
+    lab, md = run_assign(X, C)
+    ref, d1, d2 = oracle.assign(X, C)
+    assert np.array_equal(lab, ref)
+    assert np.array_equal(md, d1.astype(np.float32))
+
+
+def test_assign_single_centroid_and_far_centroids():
+    rng = np.random.default_rng(12)
+    X = rng.standard_normal((2, 300, 128)).astype(np.float16)
+    C = rng.standard_normal((2, 1, 128)).astype(np.float32)
+    lab, md = run_assign(X, C)
+    assert (lab == 0).all()
+    check_labels(X, C, lab, md)
+
+
+@pytest.mark.parametrize("case", ["random", "all_equal", "k1", "sorted", "skewed", "big_k", "ragged"])
+def test_sort_is_bit_exact(case):
+    rng = np.random.default_rng(13)
+    B, N, K = 3, 5000, 1024
+    if case == "random":
+        lab = rng.integers(0, K, (B, N))
+    elif case == "all_equal":
+        lab = np.full((B, N), 517)
+    elif case == "k1":
+        K = 1
+        lab = np.zeros((B, N))
+    elif case == "sorted":
+        lab = np.sort(rng.integers(0, K, (B, N)), axis=1)
+    elif case == "skewed":
+        lab = np.minimum(rng.zipf(1.2, (B, N)) - 1, K - 1)
+    elif case == "big_k":
+        K = 65536
+        lab = rng.integers(0, K, (B, N))
+    else:
+        B, N, K = 2, 2049, 3000  # one key past a 2048-key tile; 12-bit keys
+        lab = rng.integers(0, K, (B, N))
+    lab = lab.astype(np.int32)
+    sidx, counts, offsets = km.sort_labels(cuda(lab), K)
+    torch.cuda.synchronize()
+    check_sort(lab, K, sidx.cpu().numpy(), counts.cpu().numpy(), offsets.cpu().numpy())
+
+
+@pytest.mark.parametrize("B,N,K,d,dt,case", [
+    (2, 1000, 40, 128, "f16", "random"),
+    (2, 5000, 300, 128, "f16", "zipf"),
+    (1, 3000, 7, 128, "f16", "one_cluster"),
+    (2, 2000, 500, 128, "f16", "empty"),
+    (1, 4096, 8, 16, "f32", "random"),
+    (2, 1500, 100, 128, "f32", "zipf"),
+    (2, 999, 64, 64, "f16", "random"),
+    (1, 700, 30, 512, "f32", "random"),
+    (1, 700, 30, 512, "f16", "zipf"),
+])
+def test_update_matches_oracle(B, N, K, d, dt, case):
+    rng = np.random.default_rng(14)
+    w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, seed=77 + K)
+    X = synth.points(w)
+    if case == "random":
+        lab = rng.integers(0, K, (B, N))
+    elif case == "zipf":
+        lab = np.minimum(rng.zipf(1.2, (B, N)) - 1, K - 1)
+    elif case == "one_cluster":
+        lab = np.full((B, N), 3)
+    else:
+        lab = rng.integers(0, K // 3, (B, N)) * 3  # two thirds of the clusters empty
+    lab = lab.astype(np.int32)
+    C_prev = rng.standard_normal((B, K, d)).astype(np.float32)
+    C_out, sums, counts = km.update(cuda(X), cuda(lab), cuda(C_prev))
+    torch.cuda.synchronize()
+    check_centroids(X, lab, C_prev, C_out.cpu().numpy(), counts.cpu().numpy(), sums.cpu().numpy())
+
+
+@pytest.mark.parametrize("B,N,K,d,dt", [(2, 3000, 50, 128, "f16"), (1, 4096, 8, 16, "f32"), (2, 1000, 300, 64, "f16")])
+def test_lloyd_lockstep_with_oracle(B, N, K, d, dt):
+    """Each iteration: the oracle takes the GPU's centroids and checks that iteration's labels and update."""
+    w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=5 + K)
+    X = synth.points(w)
+    C = synth.init_centroids(w, X)
+    Xg = cuda(X)
+    near = 0
+    for t in range(5):
+        lab, C_next, obj = km.lloyd(Xg, cuda(C), 1)
+        torch.cuda.synchronize()
+        lab, C_next, obj = lab.cpu().numpy(), C_next.cpu().numpy(), obj.cpu().numpy()
+        near += check_labels(X, C, lab)
+        check_sort(lab, K, *[a.cpu().numpy() for a in km.sort_labels(cuda(lab), K)])
+        check_centroids(X, lab, C, C_next)
+        _, d1, _ = oracle.assign(X, C)
+        np.testing.assert_allclose(obj[0], d1.sum(axis=1), rtol=1e-4)
+        C = C_next
+    assert km.device_fault() == 0
+
+
+def test_lloyd_many_iterations_equal_one_at_a_time():
+    w = synth.small(B=2, N=2000, d=128, K=64, dtype="f16", seed=21)
+    X = synth.points(w)
+    C0 = synth.init_centroids(w, X)
+    Xg = cuda(X)
+    lab6, C6, obj6 = km.lloyd(Xg, cuda(C0), 6)
+    C = cuda(C0)
+    objs = []
+    for t in range(6):
+        lab1, C, o = km.lloyd(Xg, C, 1)
+        objs.append(o)
+    torch.cuda.synchronize()
+    # resuming from saved centroids reproduces the run (sums may differ in the last bits
+    # through the order of boundary atomics, hence the tolerance)
+    np.testing.assert_allclose(C6.cpu().numpy(), C.cpu().numpy(), rtol=1e-5, atol=1e-5)
+    assert (lab6.cpu().numpy() == lab1.cpu().numpy()).mean() > 0.999
+    np.testing.assert_allclose(obj6.cpu().numpy(), torch.cat(objs).cpu().numpy(), rtol=1e-5)
+
+
+def test_labels_counts_and_sort_are_deterministic():
+    w = synth.small(B=2, N=5000, d=128, K=200, dtype="f16", seed=22)
+    X = cuda(synth.points(w))
+    C = cuda(synth.init_centroids(w, X.cpu().numpy()))
+    outs = []
+    for _ in range(3):
+        lab, md = km.assign(X, C)
+        sidx, counts, offs = km.sort_labels(lab, w.K)
+        outs.append([t.cpu().numpy() for t in (lab, md, sidx, counts, offs)])
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert np.array_equal(a, b)
+
+
+def test_objective_never_increases_beyond_rounding():
+    w = synth.small(B=2, N=4000, d=128, K=100, dtype="f16", ncomp=100, seed=23)
+    X = synth.points(w)
+    C0 = synth.init_centroids(w, X)
+    _, _, obj = km.lloyd(cuda(X), cuda(C0), 12)
+    obj = obj.cpu().numpy().astype(np.float64)
+    # fp16 rounding of the centroids can add a little; it must stay tiny relative to J
+    assert (np.diff(obj, axis=0) <= 1e-3 * obj[:-1]).all()
+    assert (obj[-1] < obj[0]).all()
+
+
+def test_injected_allocation_failure_is_reported_and_leaks_nothing(monkeypatch):
+    w = synth.small(B=1, N=1000, d=128, K=50, dtype="f16", seed=24)
+    X = cuda(synth.points(w))
+    C = cuda(synth.init_centroids(w, X.cpu().numpy()))
+    km.lloyd(X, C, 1)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    monkeypatch.setenv("KM_FAULT", "alloc")
+    with pytest.raises(km.KMError) as e:
+        km.lloyd(X, C, 2)
+    assert e.value.status == 3
+    monkeypatch.setenv("KM_FAULT", "launch")
+    with pytest.raises(km.KMError) as e:
+        km.assign(X, C)
+    assert e.value.status == 4
+    monkeypatch.delenv("KM_FAULT")
+    torch.cuda.synchronize()
+    assert abs(torch.cuda.mem_get_info()[0] - free0) < (64 << 20)
+    km.lloyd(X, C, 1)  # still works
+    torch.cuda.synchronize()
