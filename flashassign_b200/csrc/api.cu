@@ -291,25 +291,27 @@ km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, 
     KM_TRY(check_device(&dev));
     cudaStream_t st = (cudaStream_t)stream;
     Scratch scratch(st);
-    int32_t *a_sorted = nullptr, *sidx = nullptr;
+    int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
     unsigned char* work = nullptr;
     KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
     KM_TRY(scratch.get(&sidx, (size_t)(B * N), "sorted indices"));
+    KM_TRY(scratch.get(&offs, (size_t)(B * (K + 1)), "segment offsets"));
     KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
     {
         PhaseScope ph(st, KM_PHASE_OTHER, 0);
         KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * (size_t)(B * K * d), st), "zero sums"));
     }
     {
-        PhaseScope ph(st, KM_PHASE_SORT, sort_kernel_launches(N, K, true));
-        KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, counts, nullptr, work, st), "label sort"));
+        PhaseScope ph(st, KM_PHASE_SORT, sort_kernel_launches(N, K, false));
+        KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, offs, work, st), "label sort"));
     }
     {
         PhaseScope ph(st, KM_PHASE_UPDATE, 1);
         KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, st), "segmented update"));
     }
     PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
-    return launched(launch_finalize(sums, counts, B, K, d, C_out, dtype, nullptr, nullptr, st), "centroid finalize");
+    return launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, nullptr, nullptr, counts, false, st),
+                    "centroid finalize");
 }
 
 km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
@@ -349,7 +351,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     const bool tc = uses_tc(dtype, d);
     __half* chat = nullptr;
     float *cnh = nullptr, *mindist = nullptr, *sums = nullptr;
-    int32_t *a_sorted = nullptr, *sidx = nullptr, *counts = nullptr;
+    int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
     unsigned char* work = nullptr;
     if (tc) {
         KM_TRY(scratch.get(&chat, ckd, "rounded centroids"));
@@ -357,7 +359,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     }
     KM_TRY(scratch.get(&mindist, (size_t)(B * N), "minimum distances"));
     KM_TRY(scratch.get(&sums, ckd, "cluster sums"));
-    KM_TRY(scratch.get(&counts, (size_t)(B * K), "cluster counts"));
+    KM_TRY(scratch.get(&offs, (size_t)(B * (K + 1)), "segment offsets"));
     KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
     KM_TRY(scratch.get(&sidx, (size_t)(B * N), "sorted indices"));
     KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
@@ -366,18 +368,20 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         PhaseScope ph(st, KM_PHASE_PREP, 1);
         KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, chat, cnh, st), "centroid preparation"));
     }
-    const int sort_launches = sort_kernel_launches(N, K, true);
+    {
+        PhaseScope ph(st, KM_PHASE_OTHER, 0);
+        KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * ckd, st), "zero sums"));
+    }
+    const int sort_launches = sort_kernel_launches(N, K, false);
     for (int t = 0; t < iters; ++t) {
         KM_TRY(run_assign(X, dtype, C_out, chat, cnh, B, N, K, d, labels, mindist, dev, st));
-        {
-            PhaseScope ph(st, KM_PHASE_OTHER, objective ? 1 : 0);
-            if (objective)
-                KM_TRY(launched(launch_objective(mindist, B, N, objective + (size_t)t * B, st), "objective"));
-            KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * ckd, st), "zero sums"));
+        if (objective) {
+            PhaseScope ph(st, KM_PHASE_OTHER, 1);
+            KM_TRY(launched(launch_objective(mindist, B, N, objective + (size_t)t * B, st), "objective"));
         }
         {
             PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
-            KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, counts, nullptr, work, st), "label sort"));
+            KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, offs, work, st), "label sort"));
         }
         {
             PhaseScope ph(st, KM_PHASE_UPDATE, 1);
@@ -385,8 +389,9 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         }
         const bool prep_next = tc && t + 1 < iters;
         PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
-        KM_TRY(launched(launch_finalize(sums, counts, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
-                                        prep_next ? cnh : nullptr, st),
+        // the finalize zeroes the consumed sums, so the next update starts from 0
+        KM_TRY(launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
+                                        prep_next ? cnh : nullptr, nullptr, true, st),
                         "centroid finalize"));
     }
     return KM_OK;

@@ -52,12 +52,17 @@ constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+constexpr int kNStages = 3;                      // half-norm tiles in flight
+constexpr int kNBytesPerStage = kTileK * 4;      // 128 fp32 half norms
+
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kXBytes = kXBufs * kRowTiles * kMaxBoxes * kBoxBytes;  // 128 KB
 constexpr int kCBytes = kCStages * kMaxBoxes * kBoxBytes;            // 96 KB
-constexpr int kBarOff = kXBytes + kCBytes;
-constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets;
+constexpr int kNOff = kXBytes + kCBytes;
+constexpr int kBarOff = kNOff + kNStages * kNBytesPerStage;
+constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 2 * kNStages;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + tmem slot, flags, alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA exceeded");
 
 // ---- PTX wrappers -------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -111,6 +116,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
 }
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
 // UMMA shared-memory descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row core groups 1024 bytes apart (SBO), LBO unused (1),
 // descriptor version 1 (sm_100).
@@ -140,21 +150,27 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// 32 consecutive fp32 columns of this thread's TMEM lane, waited on.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
+// 64 consecutive fp32 columns of this thread's TMEM lane, waited on.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+    uint32_t r[64];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
         : "r"(taddr)
         : "memory");
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(r[j]);
 }
 
 struct Params {
@@ -181,6 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_x_full = bars, bar_x_empty = bars + 8 * kXBufs;
     const uint32_t bar_c_full = bars + 16 * kXBufs, bar_c_empty = bar_c_full + 8 * kCStages;
     const uint32_t bar_acc_full = bar_c_empty + 8 * kCStages, bar_acc_empty = bar_acc_full + 8 * kAccSets;
+    const uint32_t bar_n_full = bar_acc_empty + 8 * kAccSets, bar_n_empty = bar_n_full + 8 * kNStages;
+    const uint32_t n_base = sbase + kNOff;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + kNumBars * 8 + 4);
 
@@ -197,6 +215,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kAccSets; ++i) {
             mbar_init(bar_acc_full + 8 * i, 1);
             mbar_init(bar_acc_empty + 8 * i, kEpiWarps);
+        }
+        for (int i = 0; i < kNStages; ++i) {
+            mbar_init(bar_n_full + 8 * i, 1);
+            mbar_init(bar_n_empty + 8 * i, kEpiWarps);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -273,6 +295,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) umma_commit(bar_x_empty + 8 * xb);
             }
         }
+    } else if (warp == 2) {
+        // ------------------------------ half-norm producer ------------------------------
+        if (lane == 0) {
+            uint32_t it_n = 0;
+            bool ok = true;
+            for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
+                const float* cnh_b = P.cnh + (u / P.units_per_batch) * (int64_t)P.ktiles * kTileK;
+                for (int kt = 0; kt < P.ktiles; ++kt, ++it_n) {
+                    const uint32_t ns = it_n % kNStages;
+                    if (!(ok = mbar_wait(bar_n_empty + 8 * ns, ((it_n / kNStages) & 1) ^ 1, abort_flag, P.fault)))
+                        break;
+                    mbar_expect_tx(bar_n_full + 8 * ns, kNBytesPerStage);
+                    bulk_load(n_base + ns * kNBytesPerStage, cnh_b + kt * kTileK, kNBytesPerStage, bar_n_full + 8 * ns);
+                }
+            }
+        }
     } else if (warp >= kEpiWarp0) {
         // ------------------------------ epilogue ------------------------------
         const int e = warp - kEpiWarp0;
@@ -295,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     smem + ((xb * kRowTiles + rt) * kMaxBoxes + kb) * kBoxBytes + row_in_tile * 128);
 #pragma unroll
                 for (int cch = 0; cch < 8; ++cch) {
-                    const uint4 v = rowp[cch];
+                    const uint4 v = rowp[(cch + lane) & 7];  // lanes start on different banks
                     const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
@@ -308,7 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
 
-            const float* cnh_b = P.cnh + b * (int64_t)P.ktiles * kTileK;
             float best = INFINITY;
             int gbest = -1;
             float kept[32];
@@ -316,38 +353,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) kept[j] = INFINITY;
             for (int kt = 0; kt < P.ktiles; ++kt, ++it_a) {
                 const uint32_t s = it_a % kAccSets;
+                const uint32_t ns = it_a % kNStages;
+                if (!(ok = mbar_wait(bar_n_full + 8 * ns, (it_a / kNStages) & 1, abort_flag, P.fault))) break;
                 if (!(ok = mbar_wait(bar_acc_full + 8 * s, (it_a / kAccSets) & 1, abort_flag, P.fault))) break;
                 __syncwarp();  // tcgen05.ld below is warp-collective
                 tc_fence_after();
                 const uint32_t tcol = tmem_base + ((uint32_t)(q * 32) << 16) + s * (kRowTiles * kTileK) + rt * kTileK;
+                const float4* cn = reinterpret_cast<const float4*>(smem + kNOff + ns * kNBytesPerStage);
 #pragma unroll 1
-                for (int ch = 0; ch < kTileK / 32; ++ch) {
-                    float v[32];
-                    tmem_ld32(tcol + ch * 32, v);
-                    const float4* cn4 = reinterpret_cast<const float4*>(cnh_b + kt * kTileK + ch * 32);
-                    float gmin = INFINITY;
-#pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 c = __ldg(cn4 + j4);
-                        v[4 * j4 + 0] = c.x - v[4 * j4 + 0];
-                        v[4 * j4 + 1] = c.y - v[4 * j4 + 1];
-                        v[4 * j4 + 2] = c.z - v[4 * j4 + 2];
-                        v[4 * j4 + 3] = c.w - v[4 * j4 + 3];
-                        gmin = fminf(gmin, fminf(fminf(v[4 * j4], v[4 * j4 + 1]), fminf(v[4 * j4 + 2], v[4 * j4 + 3])));
+                for (int half = 0; half < kTileK / 64; ++half) {
+                    float v[64];
+                    tmem_ld64(tcol + half * 64, v);
+                    if (half == kTileK / 64 - 1) {
+                        // every column of this tile is in registers: hand the accumulator back
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_acc_empty + 8 * s);
                     }
-                    const bool better = gmin < best;  // strict: an earlier group keeps ties
-                    if (__any_sync(0xffffffffu, better)) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) kept[j] = better ? v[j] : kept[j];
-                    }
-                    if (better) {
-                        best = gmin;
-                        gbest = kt * (kTileK / 32) + ch;
+                    for (int g = 0; g < 2; ++g) {
+                        float* w = v + 32 * g;
+                        float gmin = INFINITY;
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 c = cn[half * 16 + g * 8 + j4];
+                            w[4 * j4 + 0] = c.x - w[4 * j4 + 0];
+                            w[4 * j4 + 1] = c.y - w[4 * j4 + 1];
+                            w[4 * j4 + 2] = c.z - w[4 * j4 + 2];
+                            w[4 * j4 + 3] = c.w - w[4 * j4 + 3];
+                            gmin = fminf(gmin, fminf(fminf(w[4 * j4], w[4 * j4 + 1]), fminf(w[4 * j4 + 2], w[4 * j4 + 3])));
+                        }
+                        const bool better = gmin < best;  // strict: an earlier group keeps ties
+                        if (__any_sync(0xffffffffu, better)) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) kept[j] = better ? w[j] : kept[j];
+                        }
+                        if (better) {
+                            best = gmin;
+                            gbest = kt * (kTileK / 32) + half * 2 + g;
+                        }
                     }
                 }
-                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_acc_empty + 8 * s);
+                if (lane == 0) mbar_arrive(bar_n_empty + 8 * ns);
             }
             if (!ok) break;
             // resolve the column: first position in the kept group equal to the minimum

@@ -46,14 +46,18 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
     if (lane == 0) cnh[row] = (float)(0.5 * acc);
 }
 
-__global__ void finalize_kernel(const float* __restrict__ sums, const int32_t* __restrict__ counts, int64_t B,
-                                int64_t K, int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype,
-                                __half* __restrict__ chat, float* __restrict__ cnh) {
+// n_k comes from the sort's segment offsets (offsets[k+1] - offsets[k]); it is
+// also written to counts when that is non-null.  With zero_sums the consumed
+// sums are reset to 0, ready for the next iteration's boundary atomics.
+__global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t B, int64_t K,
+                                int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype, __half* __restrict__ chat,
+                                float* __restrict__ cnh, int32_t* __restrict__ counts, int zero_sums) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (row >= B * K) return;
     const int64_t b = row / K, k = row % K;
-    const int32_t n = counts[row];
+    const int32_t n = offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
+    if (counts && lane == 0) counts[row] = n;
     const float fn = (float)n;
     const int64_t base = row * d;
     double acc = 0.0;
@@ -62,6 +66,7 @@ __global__ void finalize_kernel(const float* __restrict__ sums, const int32_t* _
         if (n > 0) {
             v = sums[base + j] / fn;
             C_out[base + j] = v;
+            if (zero_sums) sums[base + j] = 0.f;
         } else {
             v = C_out[base + j];
         }
@@ -80,8 +85,22 @@ __global__ void finalize_kernel(const float* __restrict__ sums, const int32_t* _
 
 __global__ void objective_kernel(const float* __restrict__ mindist, int64_t N, float* __restrict__ objective) {
     const int64_t b = blockIdx.x;
+    const float* m = mindist + b * N;
     double acc = 0.0;
-    for (int64_t i = threadIdx.x; i < N; i += blockDim.x) acc += (double)mindist[b * N + i];
+    // 16-byte loads where the batch row is aligned (N % 4 == 0), with four
+    // independent partial sums to keep several loads in flight
+    if ((N & 3) == 0) {
+        const float4* m4 = reinterpret_cast<const float4*>(m);
+        const int64_t n4 = N / 4;
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+        for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
+            const float4 v = __ldg(m4 + i);
+            a0 += v.x; a1 += v.y; a2 += v.z; a3 += v.w;
+        }
+        acc = (a0 + a1) + (a2 + a3);
+    } else {
+        for (int64_t i = threadIdx.x; i < N; i += blockDim.x) acc += (double)m[i];
+    }
     acc = warp_sum(acc);
     __shared__ double part[32];
     if ((threadIdx.x & 31) == 0) part[threadIdx.x / 32] = acc;
@@ -104,11 +123,11 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
     return cudaGetLastError();
 }
 
-cudaError_t launch_finalize(const float* sums, const int32_t* counts, int64_t B, int64_t K, int64_t d, float* C_out,
-                            int dtype, __half* chat, float* cnh, cudaStream_t st) {
+cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
+                            int dtype, __half* chat, float* cnh, int32_t* counts, bool zero_sums, cudaStream_t st) {
     const int warps = 8;
-    finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(sums, counts, B, K, padded_k(K), d,
-                                                                            C_out, dtype, chat, cnh);
+    finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(
+        sums, offsets, B, K, padded_k(K), d, C_out, dtype, chat, cnh, counts, zero_sums ? 1 : 0);
     return cudaGetLastError();
 }
 

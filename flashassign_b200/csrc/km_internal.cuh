@@ -40,10 +40,12 @@ km_status device_info(DeviceInfo* out);
 cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
                                   float* cnh, cudaStream_t st);
 
-// C_out[b][k] = sums / counts where counts > 0 (else unchanged); when chat or
-// cnh is non-null, also prepares the next assignment's centroids from C_out.
-cudaError_t launch_finalize(const float* sums, const int32_t* counts, int64_t B, int64_t K, int64_t d,
-                            float* C_out, int dtype, __half* chat, float* cnh, cudaStream_t st);
+// C_out[b][k] = sums / n_k where n_k > 0 (else unchanged), n_k taken from the
+// segment offsets [B, K+1] (and written to counts when non-null); when chat
+// or cnh is non-null, also prepares the next assignment's centroids from
+// C_out; with zero_sums the sums are reset to 0 once consumed.
+cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
+                            int dtype, __half* chat, float* cnh, int32_t* counts, bool zero_sums, cudaStream_t st);
 
 // Tensor-core assignment (fp16, 64 <= d <= 128).  Returns cudaErrorNotSupported
 // for shapes it does not take.
