@@ -149,12 +149,12 @@ km_status launched(cudaError_t e, const char* what) {
     } while (0)
 
 // The assignment for one iteration, given prepared centroids.
-km_status run_assign(const void* X, int dtype, const float* C, const __half* chat, const float* cnh, int64_t B,
+km_status run_assign(const void* X, int dtype, const float* C, const __half* chat, const __half* cext, int64_t B,
                      int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, const DeviceInfo& dev,
                      cudaStream_t st) {
     PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
     if (dtype == KM_F16 && assign_tc_supported(d, dtype))
-        return launched(launch_assign_tc((const __half*)X, chat, cnh, B, N, K, d, labels, mindist, dev.sms, st),
+        return launched(launch_assign_tc((const __half*)X, chat, cext, B, N, K, d, labels, mindist, dev.sms, st),
                         "assign (tensor cores)");
     return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, st), "assign (CUDA cores)");
 }
@@ -240,15 +240,14 @@ km_status km_assign(const void* X, const float* C, int64_t B, int64_t N, int64_t
     KM_TRY(check_device(&dev));
     cudaStream_t st = (cudaStream_t)stream;
     Scratch scratch(st);
-    __half* chat = nullptr;
-    float* cnh = nullptr;
+    __half *chat = nullptr, *cext = nullptr;
     if (uses_tc(dtype, d)) {
         KM_TRY(scratch.get(&chat, (size_t)(B * K * d), "rounded centroids"));
-        KM_TRY(scratch.get(&cnh, (size_t)(B * padded_k(K)), "centroid half norms"));
+        KM_TRY(scratch.get(&cext, (size_t)(B * padded_k(K) * 16), "centroid norm slices"));
         PhaseScope ph(st, KM_PHASE_PREP, 1);
-        KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, chat, cnh, st), "centroid preparation"));
+        KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, chat, cext, st), "centroid preparation"));
     }
-    return run_assign(X, dtype, C, chat, cnh, B, N, K, d, labels, mindist, dev, st);
+    return run_assign(X, dtype, C, chat, cext, B, N, K, d, labels, mindist, dev, st);
 }
 
 km_status km_sort_labels(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* sorted_idx,
@@ -349,13 +348,13 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
 
     Scratch scratch(st);
     const bool tc = uses_tc(dtype, d);
-    __half* chat = nullptr;
-    float *cnh = nullptr, *mindist = nullptr, *sums = nullptr;
+    __half *chat = nullptr, *cext = nullptr;
+    float *mindist = nullptr, *sums = nullptr;
     int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
     unsigned char* work = nullptr;
     if (tc) {
         KM_TRY(scratch.get(&chat, ckd, "rounded centroids"));
-        KM_TRY(scratch.get(&cnh, (size_t)(B * padded_k(K)), "centroid half norms"));
+        KM_TRY(scratch.get(&cext, (size_t)(B * padded_k(K) * 16), "centroid norm slices"));
     }
     KM_TRY(scratch.get(&mindist, (size_t)(B * N), "minimum distances"));
     KM_TRY(scratch.get(&sums, ckd, "cluster sums"));
@@ -366,7 +365,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
 
     if (tc) {
         PhaseScope ph(st, KM_PHASE_PREP, 1);
-        KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, chat, cnh, st), "centroid preparation"));
+        KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, chat, cext, st), "centroid preparation"));
     }
     {
         PhaseScope ph(st, KM_PHASE_OTHER, 0);
@@ -374,7 +373,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     }
     const int sort_launches = sort_kernel_launches(N, K, false);
     for (int t = 0; t < iters; ++t) {
-        KM_TRY(run_assign(X, dtype, C_out, chat, cnh, B, N, K, d, labels, mindist, dev, st));
+        KM_TRY(run_assign(X, dtype, C_out, chat, cext, B, N, K, d, labels, mindist, dev, st));
         if (objective) {
             PhaseScope ph(st, KM_PHASE_OTHER, 1);
             KM_TRY(launched(launch_objective(mindist, B, N, objective + (size_t)t * B, st), "objective"));
@@ -391,7 +390,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
         // the finalize zeroes the consumed sums, so the next update starts from 0
         KM_TRY(launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
-                                        prep_next ? cnh : nullptr, nullptr, true, st),
+                                        prep_next ? cext : nullptr, nullptr, true, st),
                         "centroid finalize"));
     }
     return KM_OK;

@@ -1,31 +1,45 @@
-// FlashAssign on the fifth-generation tensor cores (sm_100a).
+// FlashAssign on the fifth-generation tensor cores (sm_100a), two SMs per MMA.
 //
 // What it computes (papernotes.org "Flash-KMeans" page, 关键设计 1): for every
-// point, the nearest centroid under ||x - c||^2 = ||x||^2 + ||c||^2 - 2 x.c,
-// with the N x K distances reduced on chip as they are produced (running
-// minimum m_i from +inf and index a_i from -1, a strict "<" so the lowest
-// index keeps ties) -- the distance matrix never reaches HBM, so the kernel
-// reads O(N d + K d) bytes instead of writing and re-reading O(N K).
+// point the nearest centroid under ||x - c||^2 = ||x||^2 + ||c||^2 - 2 x.c, the
+// N x K distances reduced on chip as they are produced -- a running extremum
+// per point from its initial value and index -1, replaced only on strict
+// improvement, so the lowest index keeps ties -- so that the distance matrix
+// never reaches HBM and the kernel reads O(N d + K d) bytes, not O(N K).
 //
-// How, on a B200 (the page's design is Triton on an H200 with cp.async double
-// buffering; this is a re-design for tcgen05/TMEM/TMA):
-//   * persistent grid, one CTA per SM; a work unit is 256 consecutive points of
-//     one batch (two 128-row MMA tiles), units strided over the grid so that
-//     concurrently running CTAs share their batch's centroids in L2;
-//   * warp 0 issues TMA loads: the unit's X tile (kept for all K) into one of
-//     two X buffers, and 128-centroid tiles of C (fp16, pre-rounded) into a
-//     3-stage ring, all 128-byte swizzled;
-//   * warp 1 (one thread) issues tcgen05.mma kind::f16, M=128 N=128 K=16, fp32
-//     accumulation in TMEM: for each C tile, both row tiles of the unit into
-//     one of two 256-column accumulator sets, so the epilogue of tile t
-//     overlaps the MMAs of tile t+1;
-//   * warps 4..11 (one thread per point row, TMEM lane = row) read their row
-//     32 columns at a time with tcgen05.ld, form s = ||c||^2/2 - x.c, and keep
-//     the running minimum with a per-32-column group test: the group minimum is
-//     compared with the running best, and only when it improves is the group's
-//     32 scores kept in registers; the winning column is resolved once per
-//     unit from the kept group (first column equal to the minimum).
-//     mindist = ||x||^2 + 2 * min s, with ||x||^2 summed from the staged X tile.
+// How, on a B200 (the page's kernel is Triton on an H200 with cp.async double
+// buffering; this is a re-design for tcgen05 / TMEM / TMA / CTA pairs):
+//   * The score of centroid k for point x is s = x.c_k - ||c_k||^2 / 2, and
+//     argmin_k ||x - c_k||^2 = argmax_k s.  The whole score comes out of the
+//     tensor cores: each point row gets one extra 16-wide K slice of ones and
+//     each centroid row the matching slice holding -||c||^2/2 split into fp16
+//     pieces (exact to ~2^-33 relative), so one more K=16 MMA step adds the
+//     norm term in fp32 and the epilogue only tracks maxima.
+//   * CTA pairs (a cluster of 2) run tcgen05.mma.cta_group::2 with M=256,
+//     N=128, K=16: each CTA stages its own 128 point rows and its own half
+//     (64) of each 128-centroid tile, so each SM reads only half of the B
+//     operand.  Four 128-column accumulator sets fill the 512 TMEM columns:
+//     the MMAs may run three tiles ahead of the epilogue, which hides the
+//     completion -> epilogue -> release -> issue round trip (measured at
+//     more than one 256-column tile of MMA work, the reason for N=128).
+//   * Persistent grid of pairs; a work unit is 256 consecutive points of one
+//     batch; units are strided over the pairs so that pairs running at the
+//     same time share their batch's centroids in L2.
+//   * Warp roles per CTA: warp 0 issues TMA loads (one thread: X tiles of the
+//     units into two buffers; another: centroid tiles plus their norm slices
+//     into an 8-stage ring), completing on the leader CTA's barriers; warp 1 allocates TMEM
+//     for the pair; in the leader CTA, warps 1 and 18 issue the MMAs
+//     (alternate tiles: one thread issues at most ~1 MMA per 100 cycles) and
+//     commit them to both CTAs' barriers; warps 2..17 are the epilogue: TMEM lane = point
+//     row, four warps per row split each tile's 128 columns in 32-column
+//     slices; each reads its slice with one TMEM load and releases the
+//     accumulator before doing any arithmetic on it.
+//   * Epilogue: per 32-column group, the group maximum (3-input max) is
+//     compared with the running best; when it improves for any lane of the
+//     warp, the first column equal to the group maximum is found by an
+//     equality scan and kept with it.  The four column slices of a row are
+//     joined in shared memory (larger score, then lower index).  mindist = ||x||^2 - 2 * best, ||x||^2 summed from the
+//     staged X tile.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records a fault code in the device fault word, stops issuing work, frees
 // its TMEM and returns.
@@ -36,37 +50,60 @@
 namespace km {
 namespace {
 
-constexpr int kRowsPerTile = 128;               // MMA M and TMEM lanes
-constexpr int kRowTiles = 2;                    // row tiles per unit
-constexpr int kUnitRows = kRowsPerTile * kRowTiles;
-constexpr int kTileK = kAssignTileK;            // centroids per C tile (MMA N)
+constexpr int kRows = 128;                      // point rows per CTA per unit (TMEM lanes)
+constexpr int kUnitRows = 2 * kRows;            // points per unit (per CTA pair)
+constexpr int kTileK = kAssignTileK;            // centroids per K tile (MMA N) = 128
+constexpr int kHalfTile = kTileK / 2;           // centroids staged per CTA per tile (64)
 constexpr int kBoxK = 64;                       // fp16 elements per 128-byte swizzle row
 constexpr int kMaxBoxes = 2;                    // d <= 128
-constexpr int kCStages = 3;
+constexpr int kCStages = 8;
 constexpr int kXBufs = 2;
-constexpr int kAccSets = 2;
-constexpr int kBoxBytes = kRowsPerTile * 128;   // one [128 rows x 64 fp16] swizzled box: 16 KB
-constexpr int kThreads = 384;                   // 12 warps
-constexpr int kEpiWarp0 = 4;
-constexpr int kEpiWarps = 8;
+constexpr int kAccSets = 4;                     // 4 x 128 TMEM columns: the MMA may run 3 tiles ahead
+constexpr int kBoxBytes = 128 * 128;            // X: [128 rows x 64 fp16], 128-byte swizzled
+constexpr int kCBoxBytes = kHalfTile * 128;     // C: [64 centroids x 64 fp16], 128-byte swizzled
+constexpr int kExtBytes = 128 * 32;             // ones: [128 rows x 16 fp16], 32-byte swizzled
+constexpr int kCExtBytes = kHalfTile * 32;      // norm slice: [64 centroids x 16 fp16], 32-byte swizzled
+constexpr int kThreads = 608;                   // 19 warps: producers, MMA issuer A, 16 epilogue, MMA issuer B
+constexpr int kEpiWarp0 = 2;
+constexpr int kMmaWarpB = 18;                   // second issuer, on another SMSP than warp 1
+constexpr int kEpiWarps = 16;
+constexpr int kColParts = kEpiWarps / 4;        // warps per TMEM lane quarter, each with a column slice
+constexpr int kPartCols = kTileK / kColParts;   // 32 columns of each tile per epilogue warp
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
-constexpr int kNStages = 3;                      // half-norm tiles in flight
-constexpr int kNBytesPerStage = kTileK * 4;      // 128 fp32 half norms
-
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kXBytes = kXBufs * kRowTiles * kMaxBoxes * kBoxBytes;  // 128 KB
-constexpr int kCBytes = kCStages * kMaxBoxes * kBoxBytes;            // 96 KB
-constexpr int kNOff = kXBytes + kCBytes;
-constexpr int kBarOff = kNOff + kNStages * kNBytesPerStage;
-constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 2 * kNStages;
-constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + tmem slot, flags, alignment slack
+constexpr int kXOff = 0;
+constexpr int kXBytes = kXBufs * kMaxBoxes * kBoxBytes;             // 64 KB
+constexpr int kCOff = kXOff + kXBytes;
+constexpr int kCStageBytes = kMaxBoxes * kCBoxBytes + kCExtBytes;  // 18 KB: centroid boxes + norm slice
+constexpr int kCBytes = kCStages * kCStageBytes;                    // 144 KB
+constexpr int kAOnesOff = kCOff + kCBytes;                          // 4 KB of ones (the points' extra slice)
+constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 3 parts x 128 x (score, label)
+constexpr int kMergeBytes = 2 * (kColParts - 1) * kRows * 8;
+constexpr int kBarOff = kMergeOff + kMergeBytes;
+constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 4;  // + merge handoff (2 slots x full/empty)
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;      // + tmem slot, flag, alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA exceeded");
+static_assert(kCStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 
 // ---- PTX wrappers -------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t cta_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
@@ -79,6 +116,14 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// Arrive on a barrier given by its shared::cluster address (own or peer CTA).
+// Used to hand an accumulator back: the TMEM reads are already ordered by
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync, and nothing this
+// thread wrote needs to be seen by the MMA thread, so no cluster-scope
+// release (which would wait for this thread's outstanding global stores).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
@@ -87,7 +132,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -109,40 +154,47 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         }
     }
 }
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+// TMA tile load into this CTA's shared memory, completing on a barrier that
+// may live in either CTA of the pair (cluster address).
+__device__ __forceinline__ void tma_load_pair(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                              uint32_t bar_cluster) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-        "[%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+        "%4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
         : "memory");
 }
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-// UMMA shared-memory descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes, 8-row core groups 1024 bytes apart (SBO), LBO unused (1),
-// descriptor version 1 (sm_100).
+// UMMA shared-memory descriptors, K-major operands, descriptor version 1.
+//  128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+//  32-byte swizzle:  rows of 32 bytes (one K=16 fp16 slice), 8-row groups 256 bytes apart.
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-// Instruction descriptor, kind::f16: D fp32, A and B fp16, both K-major, N, M.
+__device__ __forceinline__ uint64_t umma_desc_sw32(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
+}
+// Instruction descriptor, kind::f16: D fp32, A and B fp16, both K-major, N=256, M=256.
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kTileK >> 3) << 17) |
-                            ((uint32_t)(kRowsPerTile >> 4) << 24);
+                            ((uint32_t)(kUnitRows >> 4) << 24);
 
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_pair_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
         : "memory");
 }
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+// Arrive on the barrier at this offset in both CTAs of the pair once every
+// MMA issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+    const uint16_t both = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"(both)
+        : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -150,63 +202,61 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// 64 consecutive fp32 columns of this thread's TMEM lane, waited on.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
-    uint32_t r[64];
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane, waited on.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
-          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
-          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
 #pragma unroll
-    for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(r[j]);
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
 struct Params {
     int64_t B, N, K, d;
-    int64_t units_per_batch, units;
+    int64_t units_per_batch, units, pairs;
     int ktiles, ksteps, boxes;
-    const float* cnh;  // [B, padded K] half squared norms, +inf padding
     int32_t* labels;
     float* mindist;
     int32_t* fault;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
-                     const Params P) {
+                     const __grid_constant__ CUtensorMap tmap_e, const Params P) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t x_base = sbase;
-    const uint32_t c_base = sbase + kXBytes;
+    const uint32_t x_base = sbase + kXOff;
+    const uint32_t c_base = sbase + kCOff;
+    const uint32_t ones_base = sbase + kAOnesOff;
     const uint32_t bars = sbase + kBarOff;
-    // barrier indices
     const uint32_t bar_x_full = bars, bar_x_empty = bars + 8 * kXBufs;
     const uint32_t bar_c_full = bars + 16 * kXBufs, bar_c_empty = bar_c_full + 8 * kCStages;
     const uint32_t bar_acc_full = bar_c_empty + 8 * kCStages, bar_acc_empty = bar_acc_full + 8 * kAccSets;
-    const uint32_t bar_n_full = bar_acc_empty + 8 * kAccSets, bar_n_empty = bar_n_full + 8 * kNStages;
-    const uint32_t n_base = sbase + kNOff;
+    const uint32_t bar_m_full = bar_acc_empty + 8 * kAccSets, bar_m_empty = bar_m_full + 16;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + kNumBars * 8 + 4);
+    float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                 // [2][parts-1][128]
+    int* merge_label = reinterpret_cast<int*>(smem + kMergeOff + kMergeBytes / 2);  // [2][parts-1][128]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cta_rank();         // 0: leader CTA of the pair (issues the MMAs)
+    const int64_t pair = blockIdx.x / 2;
+
     if (threadIdx.x == 0) {
         for (int i = 0; i < kXBufs; ++i) {
-            mbar_init(bar_x_full + 8 * i, 1);
-            mbar_init(bar_x_empty + 8 * i, 1 + kEpiWarps);  // last MMA commit + every epilogue warp
+            mbar_init(bar_x_full + 8 * i, 1);               // leader: its expect_tx; bytes from both CTAs
+            mbar_init(bar_x_empty + 8 * i, 2 + kEpiWarps);  // both issuers' end-of-unit commits + local epilogue warps
         }
         for (int i = 0; i < kCStages; ++i) {
             mbar_init(bar_c_full + 8 * i, 1);
@@ -214,210 +264,232 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < kAccSets; ++i) {
             mbar_init(bar_acc_full + 8 * i, 1);
-            mbar_init(bar_acc_empty + 8 * i, kEpiWarps);
+            mbar_init(bar_acc_empty + 8 * i, 2 * kEpiWarps);  // leader: epilogue warps of both CTAs
         }
-        for (int i = 0; i < kNStages; ++i) {
-            mbar_init(bar_n_full + 8 * i, 1);
-            mbar_init(bar_n_empty + 8 * i, kEpiWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_m_full + 8 * i, kEpiWarps - 4);  // the warps of column slices 1..3
+            mbar_init(bar_m_empty + 8 * i, 4);             // the warps of column slice 0
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    // the points' extra K slice: all ones (any layout of it reads as ones)
+    for (int i = threadIdx.x; i < kExtBytes / 16; i += kThreads) {
+        const uint32_t one2 = 0x3C003C00u;  // two fp16 1.0
+        reinterpret_cast<uint4*>(smem + kAOnesOff)[i] = make_uint4(one2, one2, one2, one2);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes visible to the MMA
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kTmemCols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     const int boxes = P.boxes;
-    const uint32_t x_tile_bytes = (uint32_t)(kRowTiles * boxes * kBoxBytes);
-    const uint32_t c_tile_bytes = (uint32_t)(boxes * kBoxBytes);
+    const uint32_t x_bytes_pair = (uint32_t)(2 * boxes * kBoxBytes);
+    const uint32_t c_bytes_pair = (uint32_t)(2 * (boxes * kCBoxBytes + kCExtBytes));
 
     if (warp == 0) {
-        // ------------------------------ TMA producer ------------------------------
-        if (lane == 0) {
-            uint32_t it_x = 0, it_c = 0;
-            bool ok = true;
-            for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++it_x) {
+        // ------------------------------ TMA producers (both CTAs) ------------------------------
+        // lane 16 streams the units' X tiles (a unit ahead, so HBM latency is
+        // hidden behind a whole unit of MMAs); lane 0 streams the centroid
+        // tiles and their norm slices through the 4-stage ring.
+        if (lane == 16) {
+            uint32_t it_x = 0;
+            for (int64_t u = pair; u < P.units; u += P.pairs, ++it_x) {
                 const int b = (int)(u / P.units_per_batch);
-                const int n0 = (int)((u % P.units_per_batch) * kUnitRows);
+                const int n0 = (int)((u % P.units_per_batch) * kUnitRows) + (int)rank * kRows;
                 const uint32_t xb = it_x % kXBufs;
-                if (!(ok = mbar_wait(bar_x_empty + 8 * xb, ((it_x / kXBufs) & 1) ^ 1, abort_flag, P.fault))) break;
-                mbar_expect_tx(bar_x_full + 8 * xb, x_tile_bytes);
-                for (int rt = 0; rt < kRowTiles; ++rt)
-                    for (int kb = 0; kb < boxes; ++kb)
-                        tma_load_3d(x_base + ((xb * kRowTiles + rt) * kMaxBoxes + kb) * kBoxBytes, &tmap_x,
-                                    kb * kBoxK, n0 + rt * kRowsPerTile, b, bar_x_full + 8 * xb);
+                if (!mbar_wait(bar_x_empty + 8 * xb, ((it_x / kXBufs) & 1) ^ 1, abort_flag, P.fault)) break;
+                if (rank == 0) mbar_expect_tx(bar_x_full + 8 * xb, x_bytes_pair);
+                const uint32_t xfull_leader = map_to_rank(bar_x_full + 8 * xb, 0);
+                for (int kb = 0; kb < boxes; ++kb)
+                    tma_load_pair(x_base + (xb * kMaxBoxes + kb) * kBoxBytes, &tmap_x, kb * kBoxK, n0, b, xfull_leader);
+            }
+        } else if (lane == 0) {
+            uint32_t it_c = 0;
+            bool ok = true;
+            for (int64_t u = pair; u < P.units && ok; u += P.pairs) {
+                const int b = (int)(u / P.units_per_batch);
                 for (int kt = 0; kt < P.ktiles; ++kt, ++it_c) {
                     const uint32_t cs = it_c % kCStages;
                     if (!(ok = mbar_wait(bar_c_empty + 8 * cs, ((it_c / kCStages) & 1) ^ 1, abort_flag, P.fault)))
                         break;
-                    mbar_expect_tx(bar_c_full + 8 * cs, c_tile_bytes);
+                    if (rank == 0) mbar_expect_tx(bar_c_full + 8 * cs, c_bytes_pair);
+                    const uint32_t cfull_leader = map_to_rank(bar_c_full + 8 * cs, 0);
+                    const int k0 = kt * kTileK + (int)rank * kHalfTile;
+                    const uint32_t stage = c_base + cs * kCStageBytes;
                     for (int kb = 0; kb < boxes; ++kb)
-                        tma_load_3d(c_base + (cs * kMaxBoxes + kb) * kBoxBytes, &tmap_c, kb * kBoxK, kt * kTileK, b,
-                                    bar_c_full + 8 * cs);
+                        tma_load_pair(stage + kb * kCBoxBytes, &tmap_c, kb * kBoxK, k0, b, cfull_leader);
+                    tma_load_pair(stage + kMaxBoxes * kCBoxBytes, &tmap_e, 0, k0, b, cfull_leader);
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
+    } else if (warp == 1 || warp == kMmaWarpB) {
+        // ------------------------------ MMA issuers (leader CTA) ------------------------------
+        // One thread issues at most about one tcgen05.mma per ~100 cycles, so
+        // two threads on different SMSPs share the work: issuer A takes the
+        // even tiles (accumulator set 0), issuer B the odd ones (set 1).  Each
+        // C stage is only ever used by one of them (4 stages, 2 issuers).
+        const uint32_t mine = warp == 1 ? 0u : 1u;
+        if (rank == 0 && lane == 0) {
             uint32_t it_x = 0, it_c = 0, it_a = 0;
             bool ok = true;
-            for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++it_x) {
+            for (int64_t u = pair; u < P.units && ok; u += P.pairs, ++it_x) {
                 const uint32_t xb = it_x % kXBufs;
                 if (!(ok = mbar_wait(bar_x_full + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
+                const uint64_t a_desc0 = umma_desc_sw128(x_base + xb * kMaxBoxes * kBoxBytes);
                 for (int kt = 0; kt < P.ktiles; ++kt, ++it_c, ++it_a) {
+                    if ((it_a & 1u) != mine) continue;
                     const uint32_t cs = it_c % kCStages;
                     const uint32_t s = it_a % kAccSets;
                     if (!(ok = mbar_wait(bar_c_full + 8 * cs, (it_c / kCStages) & 1, abort_flag, P.fault))) break;
                     if (!(ok = mbar_wait(bar_acc_empty + 8 * s, ((it_a / kAccSets) & 1) ^ 1, abort_flag, P.fault)))
                         break;
                     tc_fence_after();
-                    for (int rt = 0; rt < kRowTiles; ++rt) {
-                        const uint32_t d_tmem = tmem_base + s * (kRowTiles * kTileK) + rt * kTileK;
-                        for (int ks = 0; ks < P.ksteps; ++ks) {
-                            const int kb = ks / 4;
-                            const uint32_t koff = (uint32_t)(ks % 4) * 32;
-                            const uint32_t a_addr = x_base + ((xb * kRowTiles + rt) * kMaxBoxes + kb) * kBoxBytes + koff;
-                            const uint32_t b_addr = c_base + (cs * kMaxBoxes + kb) * kBoxBytes + koff;
-                            umma_f16(d_tmem, umma_desc_sw128(a_addr), umma_desc_sw128(b_addr), ks > 0 ? 1u : 0u);
-                        }
+                    const uint32_t d_tmem = tmem_base + s * kTileK;
+                    const uint32_t stage = c_base + cs * kCStageBytes;
+                    const uint64_t b_desc0 = umma_desc_sw128(stage);
+                    for (int ks = 0; ks < P.ksteps; ++ks) {
+                        // start-address field advance (16-byte units): box, then 32 bytes per K=16 step
+                        const uint64_t a_off = (uint64_t)(((ks >> 2) * kBoxBytes + (ks & 3) * 32) >> 4);
+                        const uint64_t b_off = (uint64_t)(((ks >> 2) * kCBoxBytes + (ks & 3) * 32) >> 4);
+                        umma_pair_f16(d_tmem, a_desc0 + a_off, b_desc0 + b_off, ks > 0 ? 1u : 0u);
                     }
-                    umma_commit(bar_c_empty + 8 * cs);
-                    umma_commit(bar_acc_full + 8 * s);
+                    // the norm slice: ones (points) x (-||c||^2/2 pieces) (centroids)
+                    umma_pair_f16(d_tmem, umma_desc_sw32(ones_base), umma_desc_sw32(stage + kMaxBoxes * kCBoxBytes),
+                                  1u);
+                    umma_commit_pair(bar_c_empty + 8 * cs);
+                    umma_commit_pair(bar_acc_full + 8 * s);
                 }
-                if (ok) umma_commit(bar_x_empty + 8 * xb);
+                if (ok) umma_commit_pair(bar_x_empty + 8 * xb);
             }
         }
-    } else if (warp == 2) {
-        // ------------------------------ half-norm producer ------------------------------
-        if (lane == 0) {
-            uint32_t it_n = 0;
-            bool ok = true;
-            for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x) {
-                const float* cnh_b = P.cnh + (u / P.units_per_batch) * (int64_t)P.ktiles * kTileK;
-                for (int kt = 0; kt < P.ktiles; ++kt, ++it_n) {
-                    const uint32_t ns = it_n % kNStages;
-                    if (!(ok = mbar_wait(bar_n_empty + 8 * ns, ((it_n / kNStages) & 1) ^ 1, abort_flag, P.fault)))
-                        break;
-                    mbar_expect_tx(bar_n_full + 8 * ns, kNBytesPerStage);
-                    bulk_load(n_base + ns * kNBytesPerStage, cnh_b + kt * kTileK, kNBytesPerStage, bar_n_full + 8 * ns);
-                }
-            }
-        }
-    } else if (warp >= kEpiWarp0) {
-        // ------------------------------ epilogue ------------------------------
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
+        // ------------------------------ epilogue (both CTAs) ------------------------------
         const int e = warp - kEpiWarp0;
-        const int q = warp % 4;            // TMEM lane quarter this warp may access
-        const int rt = e / 4;              // row tile of the unit
-        const int row_in_unit = rt * kRowsPerTile + q * 32 + lane;
-        const int row_in_tile = q * 32 + lane;
+        const int q = warp % 4;   // TMEM lane quarter this warp may access
+        const int h = e / 4;      // which 32-column slice of each 128-column tile
+        const int row = q * 32 + lane;
+        const uint32_t acc_empty_leader0 = map_to_rank(bar_acc_empty, 0);
         uint32_t it_x = 0, it_a = 0;
         bool ok = true;
-        for (int64_t u = blockIdx.x; u < P.units && ok; u += gridDim.x, ++it_x) {
+        for (int64_t u = pair; u < P.units && ok; u += P.pairs, ++it_x) {
             const int64_t b = u / P.units_per_batch;
-            const int64_t n = (u % P.units_per_batch) * kUnitRows + row_in_unit;
+            const int64_t n = (u % P.units_per_batch) * kUnitRows + (int64_t)rank * kRows + row;
             const uint32_t xb = it_x % kXBufs;
-            if (!(ok = mbar_wait(bar_x_full + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
-            // ||x||^2 from the staged tile: the swizzle permutes 16-byte chunks
-            // within a 128-byte row, so the row's bytes are all in place.
             float xnorm = 0.f;
-            for (int kb = 0; kb < boxes; ++kb) {
-                const uint4* rowp = reinterpret_cast<const uint4*>(
-                    smem + ((xb * kRowTiles + rt) * kMaxBoxes + kb) * kBoxBytes + row_in_tile * 128);
-#pragma unroll
-                for (int cch = 0; cch < 8; ++cch) {
-                    const uint4 v = rowp[(cch + lane) & 7];  // lanes start on different banks
-                    const __half2* h = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float2 f = __half22float2(h[t]);
-                        xnorm = fmaf(f.x, f.x, xnorm);
-                        xnorm = fmaf(f.y, f.y, xnorm);
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
-
-            float best = INFINITY;
-            int gbest = -1;
-            float kept[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) kept[j] = INFINITY;
+            float best = -INFINITY;
+            int label = -1;
             for (int kt = 0; kt < P.ktiles; ++kt, ++it_a) {
                 const uint32_t s = it_a % kAccSets;
-                const uint32_t ns = it_a % kNStages;
-                if (!(ok = mbar_wait(bar_n_full + 8 * ns, (it_a / kNStages) & 1, abort_flag, P.fault))) break;
                 if (!(ok = mbar_wait(bar_acc_full + 8 * s, (it_a / kAccSets) & 1, abort_flag, P.fault))) break;
                 __syncwarp();  // tcgen05.ld below is warp-collective
                 tc_fence_after();
-                const uint32_t tcol = tmem_base + ((uint32_t)(q * 32) << 16) + s * (kRowTiles * kTileK) + rt * kTileK;
-                const float4* cn = reinterpret_cast<const float4*>(smem + kNOff + ns * kNBytesPerStage);
-#pragma unroll 1
-                for (int half = 0; half < kTileK / 64; ++half) {
-                    float v[64];
-                    tmem_ld64(tcol + half * 64, v);
-                    if (half == kTileK / 64 - 1) {
-                        // every column of this tile is in registers: hand the accumulator back
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bar_acc_empty + 8 * s);
+                // this warp's 64 columns of the tile, then hand the accumulator
+                // straight back so the MMA of tile t+2 is not held up by the math
+                float v[kPartCols];
+                tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + s * kTileK + h * kPartCols, v);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
+                if (kt == 0) {
+                    // The MMA has consumed this unit's X tile, so it is in place.
+                    // ||x||^2 from it: the swizzle permutes 16-byte chunks within a
+                    // 128-byte row, so each row's bytes are all in that row.
+                    if (h == 0) {
+                        for (int kb = 0; kb < boxes; ++kb) {
+                            const uint4* rowp =
+                                reinterpret_cast<const uint4*>(smem + kXOff + (xb * kMaxBoxes + kb) * kBoxBytes + row * 128);
+#pragma unroll
+                            for (int cch = 0; cch < 8; ++cch) {
+                                const uint4 xv = rowp[(cch + lane) & 7];  // lanes start on different banks
+                                const __half2* hh = reinterpret_cast<const __half2*>(&xv);
+#pragma unroll
+                                for (int t = 0; t < 4; ++t) {
+                                    const float2 f = __half22float2(hh[t]);
+                                    xnorm = fmaf(f.x, f.x, xnorm);
+                                    xnorm = fmaf(f.y, f.y, xnorm);
+                                }
+                            }
+                        }
                     }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
+                }
 #pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        float* w = v + 32 * g;
-                        float gmin = INFINITY;
+                for (int g = 0; g < kPartCols / 32; ++g) {
+                    const float* w = v + 32 * g;
+                    // two interleaved 3-input chains: few live temporaries
+                    float ga = max3(w[0], w[1], w[2]), gb = max3(w[3], w[4], w[5]);
 #pragma unroll
-                        for (int j4 = 0; j4 < 8; ++j4) {
-                            const float4 c = cn[half * 16 + g * 8 + j4];
-                            w[4 * j4 + 0] = c.x - w[4 * j4 + 0];
-                            w[4 * j4 + 1] = c.y - w[4 * j4 + 1];
-                            w[4 * j4 + 2] = c.z - w[4 * j4 + 2];
-                            w[4 * j4 + 3] = c.w - w[4 * j4 + 3];
-                            gmin = fminf(gmin, fminf(fminf(w[4 * j4], w[4 * j4 + 1]), fminf(w[4 * j4 + 2], w[4 * j4 + 3])));
-                        }
-                        const bool better = gmin < best;  // strict: an earlier group keeps ties
-                        if (__any_sync(0xffffffffu, better)) {
+                    for (int t = 6; t < 30; t += 4) {
+                        ga = max3(ga, w[t], w[t + 1]);
+                        gb = max3(gb, w[t + 2], w[t + 3]);
+                    }
+                    const float gmax = max3(max3(ga, w[30], w[31]), gb, gb);
+                    const bool better = gmax > best;  // strict: an earlier group keeps ties
+                    if (__any_sync(0xffffffffu, better)) {
+                        // first column of the group holding the maximum
+                        int j0 = 31;
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) kept[j] = better ? w[j] : kept[j];
-                        }
+                        for (int j = 31; j >= 0; --j) j0 = (w[j] == gmax) ? j : j0;
                         if (better) {
-                            best = gmin;
-                            gbest = kt * (kTileK / 32) + half * 2 + g;
+                            best = gmax;
+                            label = kt * kTileK + h * kPartCols + g * 32 + j0;
                         }
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_n_empty + 8 * ns);
             }
             if (!ok) break;
-            // resolve the column: first position in the kept group equal to the minimum
-            int jbest = 31;
+            // join the column slices of each row (larger score, then lower
+            // index) through a double-buffered shared slot with bounded handoffs
+            const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
+            if (h > 0) {
+                if (!(ok = mbar_wait(bar_m_empty + 8 * ms, mph ^ 1, abort_flag, P.fault))) break;
+                const int slot = ((int)ms * (kColParts - 1) + (h - 1)) * kRows + row;
+                merge_score[slot] = best;
+                merge_label[slot] = label;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_m_full + 8 * ms);
+            } else {
+                if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
+                float fb = best;
+                int fl = label;
 #pragma unroll
-            for (int j = 31; j >= 0; --j) jbest = (kept[j] == best) ? j : jbest;
-            if (n < P.N) {
-                P.labels[b * P.N + n] = gbest < 0 ? -1 : gbest * 32 + jbest;
-                if (P.mindist) P.mindist[b * P.N + n] = fmaxf(fmaf(2.f, best, xnorm), 0.f);
+                for (int part = 0; part < kColParts - 1; ++part) {
+                    const int slot = ((int)ms * (kColParts - 1) + part) * kRows + row;
+                    const float ob = merge_score[slot];
+                    const int ol = merge_label[slot];
+                    if (ob > fb || (ob == fb && ol >= 0 && (fl < 0 || ol < fl))) {
+                        fb = ob;
+                        fl = ol;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
+                if (n < P.N) {
+                    P.labels[b * P.N + n] = fl;
+                    if (P.mindist) P.mindist[b * P.N + n] = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
+                }
             }
         }
     }
 
-    // teardown: every role is done (or aborted); free TMEM
+    // teardown: every role of both CTAs is done (or aborted); free the pair's TMEM
     tc_fence_before();
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) __nanosleep(1000000);  // let in-flight async copies land
-    __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                      : "memory");
     }
 }
@@ -439,16 +511,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [B, rows, d] fp16, boxes of [1, 128 rows, 64 cols], 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* base, int64_t B, int64_t rows, int64_t d) {
+// [B, rows, cols] fp16 with boxes of [1, box_rows, box_cols], zero fill outside.
+bool make_map(CUtensorMap* m, const void* base, int64_t B, int64_t rows, int64_t cols, int box_cols, int box_rows,
+              CUtensorMapSwizzle swz) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)B};
-    cuuint64_t strides[2] = {(cuuint64_t)(d * 2), (cuuint64_t)(rows * d * 2)};
-    cuuint32_t box[3] = {(cuuint32_t)kBoxK, (cuuint32_t)kRowsPerTile, 1};
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(rows * cols * 2)};
+    cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -456,11 +529,14 @@ bool make_map(CUtensorMap* m, const void* base, int64_t B, int64_t rows, int64_t
 
 bool assign_tc_supported(int64_t d, int dtype) { return dtype == KM_F16 && d >= 64 && d <= 128 && d % 8 == 0; }
 
-cudaError_t launch_assign_tc(const __half* X, const __half* chat, const float* cnh, int64_t B, int64_t N, int64_t K,
+cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
                              int64_t d, int32_t* labels, float* mindist, int sms, cudaStream_t st) {
     if (!assign_tc_supported(d, KM_F16)) return cudaErrorNotSupported;
-    CUtensorMap mx, mc;
-    if (!make_map(&mx, X, B, N, d) || !make_map(&mc, chat, B, K, d)) return cudaErrorInvalidValue;
+    CUtensorMap mx, mc, me;
+    if (!make_map(&mx, X, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mc, chat, B, K, d, kBoxK, kHalfTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&me, cext, B, padded_k(K), 16, 16, kHalfTile, CU_TENSOR_MAP_SWIZZLE_32B))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     Params P;
@@ -470,12 +546,29 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const float* c
     P.ktiles = (int)ceil_div(K, kTileK);
     P.ksteps = (int)ceil_div(d, 16);
     P.boxes = (int)ceil_div(d, kBoxK);
-    P.cnh = cnh;
     P.labels = labels;
     P.mindist = mindist;
     P.fault = fault_word();
-    const int64_t grid = P.units < sms ? P.units : sms;
-    assign_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mx, mc, P);
+    // co-resident CTA pairs (a GPC with an odd number of free SMs cannot host a whole pair)
+    static int pair_cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int max_pairs = (dev >= 0 && dev < 64) ? pair_cache[dev] : 0;
+    if (max_pairs <= 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(sms & ~1), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, (void*)assign_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = sms / 2;
+        }
+        max_pairs = n < sms / 2 ? n : sms / 2;
+        if (dev >= 0 && dev < 64) pair_cache[dev] = max_pairs;
+    }
+    P.pairs = P.units < max_pairs ? P.units : max_pairs;
+    assign_tc_kernel<<<(unsigned)(2 * P.pairs), kThreads, kSmemBytes, st>>>(mx, mc, me, P);
     return cudaGetLastError();
 }
 

@@ -1,8 +1,8 @@
 // Centroid-side kernels of the Lloyd iteration:
 //  * preparation for the assignment: round the fp32 centroids to the dtype of
-//    X and take half their squared norms (the ||c||^2 term of the expansion
-//    ||x - c||^2 = ||x||^2 + ||c||^2 - 2 x.c, papernotes.org "Flash-KMeans"
-//    page, 关键设计 1);
+//    X and write -||c||^2/2 as a 16-wide fp16 slice that the tensor cores
+//    add to x.c (the ||c||^2 term of the expansion ||x - c||^2 = ||x||^2 +
+//    ||c||^2 - 2 x.c, papernotes.org "Flash-KMeans" page, 关键设计 1);
 //  * finalisation of the update: c_k = s_k / n_k, an empty cluster keeping its
 //    previous centroid (the flowchart's C_new on the same page, 整体框架);
 //  * the per-batch objective sum of the minimum distances.
@@ -21,14 +21,28 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
+// The centroid's norm slice for the tensor-core assignment: 16 fp16 values
+// whose sum is -v to within ~2^-33 relative (greedy pieces, each the
+// nearest fp16 to what is left, clamped to the fp16 range).
+__device__ __forceinline__ void write_norm_slice(__half* out, double v) {
+    double r = -v;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const double c = fmin(fmax(r, -65504.0), 65504.0);
+        const __half p = __float2half_rn((float)c);
+        out[i] = p;
+        r -= (double)__half2float(p);
+    }
+}
+
 __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, int64_t Kp, int64_t d, int dtype,
-                            __half* __restrict__ chat, float* __restrict__ cnh) {
+                            __half* __restrict__ chat, __half* __restrict__ cext) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (row >= B * Kp) return;
     const int64_t b = row / Kp, k = row % Kp;
-    if (k >= K) {
-        if (lane == 0) cnh[row] = INFINITY;
+    if (k >= K) {  // padding centroid: score -inf, never the maximum
+        if (lane < 16) cext[row * 16 + lane] = lane == 0 ? __ushort_as_half((unsigned short)0xFC00) : __float2half(0.f);
         return;
     }
     const int64_t base = (b * K + k) * d;
@@ -43,7 +57,7 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
         acc += (double)v * (double)v;
     }
     acc = warp_sum(acc);
-    if (lane == 0) cnh[row] = (float)(0.5 * acc);
+    if (lane == 0) write_norm_slice(cext + row * 16, 0.5 * acc);
 }
 
 // n_k comes from the sort's segment offsets (offsets[k+1] - offsets[k]); it is
@@ -51,7 +65,7 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
 // sums are reset to 0, ready for the next iteration's boundary atomics.
 __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t B, int64_t K,
                                 int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype, __half* __restrict__ chat,
-                                float* __restrict__ cnh, int32_t* __restrict__ counts, int zero_sums) {
+                                __half* __restrict__ cext, int32_t* __restrict__ counts, int zero_sums) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (row >= B * K) return;
@@ -77,9 +91,9 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
         }
         acc += (double)v * (double)v;
     }
-    if (cnh) {
+    if (cext) {
         acc = warp_sum(acc);
-        if (lane == 0) cnh[b * Kp + k] = (float)(0.5 * acc);
+        if (lane == 0) write_norm_slice(cext + (b * Kp + k) * 16, 0.5 * acc);
     }
 }
 
@@ -115,19 +129,19 @@ __global__ void objective_kernel(const float* __restrict__ mindist, int64_t N, f
 }  // namespace
 
 cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
-                                  float* cnh, cudaStream_t st) {
+                                  __half* cext, cudaStream_t st) {
     const int64_t Kp = padded_k(K);
     const int64_t rows = B * Kp;
     const int warps = 8;
-    prep_kernel<<<(unsigned)ceil_div(rows, warps), warps * 32, 0, st>>>(C, B, K, Kp, d, dtype, chat, cnh);
+    prep_kernel<<<(unsigned)ceil_div(rows, warps), warps * 32, 0, st>>>(C, B, K, Kp, d, dtype, chat, cext);
     return cudaGetLastError();
 }
 
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
-                            int dtype, __half* chat, float* cnh, int32_t* counts, bool zero_sums, cudaStream_t st) {
+                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, cudaStream_t st) {
     const int warps = 8;
     finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(
-        sums, offsets, B, K, padded_k(K), d, C_out, dtype, chat, cnh, counts, zero_sums ? 1 : 0);
+        sums, offsets, B, K, padded_k(K), d, C_out, dtype, chat, cext, counts, zero_sums ? 1 : 0);
     return cudaGetLastError();
 }
 

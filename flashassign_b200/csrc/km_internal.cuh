@@ -20,8 +20,9 @@ int32_t* fault_word();  // device address of the word on the current device
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Tile width of the assignment kernels along K; the half-norm array is padded
-// to a multiple of it with +inf so that padded columns never win.
+// Tile width of the tensor-core assignment along K; the centroids' norm-slice
+// array [B, padded_k(K), 16] is padded to a multiple of it with rows whose
+// score is -inf, so that padded columns never win.
 constexpr int kAssignTileK = 128;
 inline int64_t padded_k(int64_t K) { return ceil_div(K, kAssignTileK) * kAssignTileK; }
 
@@ -33,24 +34,23 @@ struct DeviceInfo {
 km_status device_info(DeviceInfo* out);
 
 // ---- launchers (all asynchronous on `st`) ----
-// Centroid preparation for the assignment: chat = fp16(C) (RNE) and
-// cnh[b][k] = 0.5 * ||chat_k||^2 for k < K, +inf for K <= k < padded_k(K).
-// For fp32 runs chat may be null (the fp32 kernel reads C directly) and cnh
-// holds 0.5 * ||C_k||^2.
+// Centroid preparation for the tensor-core assignment: chat = fp16(C) (RNE)
+// and cext[b][k][0..16) = fp16 pieces summing to -||chat_k||^2 / 2 for k < K,
+// (-inf, 0, ...) for K <= k < padded_k(K).
 cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
-                                  float* cnh, cudaStream_t st);
+                                  __half* cext, cudaStream_t st);
 
 // C_out[b][k] = sums / n_k where n_k > 0 (else unchanged), n_k taken from the
 // segment offsets [B, K+1] (and written to counts when non-null); when chat
-// or cnh is non-null, also prepares the next assignment's centroids from
+// or cext is non-null, also prepares the next assignment's centroids from
 // C_out; with zero_sums the sums are reset to 0 once consumed.
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
-                            int dtype, __half* chat, float* cnh, int32_t* counts, bool zero_sums, cudaStream_t st);
+                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, cudaStream_t st);
 
 // Tensor-core assignment (fp16, 64 <= d <= 128).  Returns cudaErrorNotSupported
 // for shapes it does not take.
 bool assign_tc_supported(int64_t d, int dtype);
-cudaError_t launch_assign_tc(const __half* X, const __half* chat, const float* cnh, int64_t B, int64_t N, int64_t K,
+cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
                              int64_t d, int32_t* labels, float* mindist, int sms, cudaStream_t st);
 
 // CUDA-core assignment for every supported shape (fp32 inputs, and fp16
