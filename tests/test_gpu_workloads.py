@@ -1,0 +1,74 @@
+"""Parity at the full workload sizes, in the launch configuration the benchmark uses.
+
+Lock-step protocol: at each iteration the oracle takes the GPU's centroids C_t; the GPU's labels are
+checked on sampled rows (the oracle's assignment is O(K d) per row), the argsort and counts bit-exactly
+over all points, and the update over all points.  A multi-iteration call is checked at its end.
+"""
+import numpy as np
+import pytest
+
+import synth
+from parity import check_centroids, check_labels, check_sort
+
+torch = pytest.importorskip("torch")
+import flashassign_b200 as km  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+def cuda(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def sample_rows(B, N, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = rng.choice(B * N, size=min(n, B * N), replace=False)
+    # always include the first and last rows of every batch (tile edges)
+    edges = np.concatenate([np.arange(B) * N, np.arange(B) * N + N - 1])
+    return np.unique(np.concatenate([rows, edges]))
+
+
+def lockstep(w, iters, nsample):
+    X = synth.points(w)
+    C = synth.init_centroids(w, X)
+    Xg = cuda(X)
+    near = 0
+    for t in range(iters):
+        lab, C_next, obj = km.lloyd(Xg, cuda(C), 1)
+        torch.cuda.synchronize()
+        lab, C_next = lab.cpu().numpy(), C_next.cpu().numpy()
+        rows = sample_rows(w.B, w.N, nsample, seed=t)
+        near += check_labels(X, C, lab, rows=rows)
+        sidx, counts, offs = km.sort_labels(cuda(lab), w.K)
+        check_sort(lab, w.K, sidx.cpu().numpy(), counts.cpu().numpy(), offs.cpu().numpy())
+        check_centroids(X, lab, C, C_next)
+        C = C_next
+    assert km.device_fault() == 0
+    return X, C, near
+
+
+def test_workload1_small_fp32_full_lockstep():
+    w = synth.WORKLOADS[1]
+    X, C, near = lockstep(w, w.iters, nsample=w.B * w.N)
+
+
+def test_workload2_metric_configuration():
+    w = synth.WORKLOADS[2]
+    X, C, near = lockstep(w, 3, nsample=4096)
+    # and a multi-iteration call, as the benchmark makes it: check its last assignment
+    Xg = cuda(X)
+    lab_a, C_a, _ = km.lloyd(Xg, cuda(C), 4)        # four more iterations ...
+    lab_b, C_b, _ = km.lloyd(Xg, cuda(C), 3)        # ... whose first three give the last one's input
+    torch.cuda.synchronize()
+    C3 = C_b.cpu().numpy()
+    check_labels(X, C3, lab_a.cpu().numpy(), rows=sample_rows(w.B, w.N, 4096, seed=99))
+
+
+def test_workload3_zipf_hot_clusters():
+    w = synth.WORKLOADS[3]
+    lockstep(w, 2, nsample=2048)
+
+
+def test_workload4_large_k():
+    w = synth.WORKLOADS[4]
+    lockstep(w, 2, nsample=384)
