@@ -27,6 +27,8 @@ SIGNATURES = {
     "km_status_string": (ctypes.c_char_p, [_INT]),
     "km_last_error": (ctypes.c_char_p, []),
     "km_device_fault": (_INT, [ctypes.POINTER(ctypes.c_int32), _P]),
+    "km_assign_noalloc": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "km_assign_noalloc_limit": (ctypes.c_size_t, []),
     "km_trace_enable": (None, [_INT]),
     "km_trace_read": (_INT, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _INT]),
 }

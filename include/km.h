@@ -33,6 +33,7 @@
 #ifndef KM_H
 #define KM_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -124,6 +125,29 @@ KM_API km_status km_update(const void* X, const int32_t* labels, int64_t B, int6
  */
 KM_API km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
                    int iters, int32_t* labels, float* C_out, float* objective, void* stream);
+
+/*
+ * km_assign without any device-memory allocation.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate --
+ * e.g. a framework that has reserved the device's memory for its own pool,
+ * or a latency-critical loop that must not enter the allocator, which can
+ * synchronise and take locks.  Same arguments, results and kernels as
+ * km_assign; the scratch (fp16 centroids and their norm slices) lives in one
+ * fixed array of km_assign_noalloc_limit() bytes (16 MiB) compiled into the
+ * library, which every GPU that loads the library holds until exit.
+ *   - Needs 2*B*K*d + 32*B*ceil(K/128)*128 bytes for fp16 inputs with
+ *     64 <= d <= 128 (none otherwise); larger problems return
+ *     KM_E_UNSUPPORTED with the sizes in km_last_error().
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call rewrites what it reads.  Calls whose work overlaps on the GPU
+ *     (e.g. on two streams without ordering) race on it: order them.
+ */
+KM_API km_status km_assign_noalloc(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
+                                   int dtype, int32_t* labels, float* mindist, void* stream);
+KM_API size_t km_assign_noalloc_limit(void);
 
 /* Rows per chunk used by km_lloyd for host-resident X (0 restores the default, 2^23). */
 KM_API void km_set_chunk_rows(int64_t rows);
