@@ -30,6 +30,23 @@ METRIC = "ms per Lloyd iter at B32·N65536·K1024·d128 fp16; assign/update % of
 UNIT = "ms/iter"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic of one launch on this workload (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu
+# captures summarised in profiles/assign_tc_kernel_b32_n65536_k1024_d128_f16.md and
+# profiles/update_kernel_b32_n65536_k1024_d128_f16.md, each valid only for the kernel source it was
+# taken on (sha1 of the .cu file); reported as null once that source changes.
+ASSIGN_TRAFFIC = {"sha1": "f678660a53efdcf194671074c5f5b680e53f02ed", "bytes": 546.345984e6 + 20.080384e6}
+UPDATE_TRAFFIC = {"sha1": "9f133d72b690f094d1ceba919954c8667c0bcb82", "bytes": 557.686784e6 + 17.115648e6}
+
+
+def traffic_for(src: str, rec: dict):
+    import hashlib
+    path = os.path.join(ROOT, "flashassign_b200", "csrc", src)
+    try:
+        h = hashlib.sha1(open(path, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return rec["bytes"] if rec["sha1"] == h else None
+
 
 def parse():
     p = argparse.ArgumentParser()
@@ -294,11 +311,13 @@ def run_ours(args, w):
         "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "global_problems": w.B * world,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (X is 512 MiB)"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": round(tflops / peak_tf, 4), "traffic": None, "kernel": "assign_tc_kernel",
+                     "frac": round(tflops / peak_tf, 4), "traffic": traffic_for("assign_tc.cu", ASSIGN_TRAFFIC),
+                     "kernel": "assign_tc_kernel",
                      "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)",
                      "ms_per_launch": round(t_assign, 4)},
         "roofline_update": {"bound": "hbm", "achieved": round(upd_gbs, 1), "peak": peak_bw, "unit": "GB/s",
                             "frac": round(upd_gbs / peak_bw, 4), "kernel": "update_kernel",
+                            "traffic": traffic_for("update.cu", UPDATE_TRAFFIC),
                             "ms_per_launch": round(t_update, 4), "peak_source": peak_src},
         "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4)},
         "phases_ms_per_iter": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
