@@ -28,16 +28,16 @@
 //   * Warp roles per CTA: warp 0 issues TMA loads (one thread: X tiles of the
 //     units into two buffers; another: centroid tiles plus their norm slices
 //     into an 8-stage ring), completing on the leader CTA's barriers; warp 1 allocates TMEM
-//     for the pair; in the leader CTA, warps 1 and 18 issue the MMAs
+//     for the pair; in the leader CTA, warps 1 and 10 issue the MMAs
 //     (alternate tiles: one thread issues at most ~1 MMA per 100 cycles) and
 //     commit them to both CTAs' barriers; warps 2..17 are the epilogue: TMEM lane = point
 //     row, four warps per row split each tile's 128 columns in 32-column
 //     slices; each reads its slice with one TMEM load and releases the
 //     accumulator before doing any arithmetic on it.
 //   * Epilogue: per 32-column group, the group maximum (3-input max) is
-//     compared with the running best; when it improves for any lane of the
-//     warp, the first column equal to the group maximum is found by an
-//     equality scan and kept with it.  The four column slices of a row are
+//     compared with the running best; only when it improves are the group's
+//     32 scores kept in registers, and the winning column is resolved once
+//     per unit from the kept group (first column equal to the maximum).  The two column slices of a row are
 //     joined in shared memory (larger score, then lower index).  mindist = ||x||^2 - 2 * best, ||x||^2 summed from the
 //     staged X tile.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
@@ -63,12 +63,12 @@ constexpr int kBoxBytes = 128 * 128;            // X: [128 rows x 64 fp16], 128-
 constexpr int kCBoxBytes = kHalfTile * 128;     // C: [64 centroids x 64 fp16], 128-byte swizzled
 constexpr int kExtBytes = 128 * 32;             // ones: [128 rows x 16 fp16], 32-byte swizzled
 constexpr int kCExtBytes = kHalfTile * 32;      // norm slice: [64 centroids x 16 fp16], 32-byte swizzled
-constexpr int kThreads = 608;                   // 19 warps: producers, MMA issuer A, 16 epilogue, MMA issuer B
+constexpr int kThreads = 352;                   // 11 warps: producers, MMA issuer A, 8 epilogue, MMA issuer B
 constexpr int kEpiWarp0 = 2;
-constexpr int kMmaWarpB = 18;                   // second issuer, on another SMSP than warp 1
-constexpr int kEpiWarps = 16;
+constexpr int kMmaWarpB = 10;                   // second issuer, on another SMSP than warp 1
+constexpr int kEpiWarps = 8;                    // at most 3 warps per SMSP: up to 168 registers each
 constexpr int kColParts = kEpiWarps / 4;        // warps per TMEM lane quarter, each with a column slice
-constexpr int kPartCols = kTileK / kColParts;   // 32 columns of each tile per epilogue warp
+constexpr int kPartCols = kTileK / kColParts;   // 64 columns of each tile per epilogue warp
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -207,17 +207,17 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
-// 32 consecutive fp32 columns of this thread's TMEM lane, waited on.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
+// 64 consecutive fp32 columns of this thread's TMEM lane, waited on.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+    uint32_t r[64];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
         : "r"(taddr)
         : "memory");
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(r[j]);
 }
 
 struct Params {
@@ -374,18 +374,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ------------------------------ epilogue (both CTAs) ------------------------------
         const int e = warp - kEpiWarp0;
         const int q = warp % 4;   // TMEM lane quarter this warp may access
-        const int h = e / 4;      // which 32-column slice of each 128-column tile
+        const int h = e / 4;      // which 64-column slice of each 128-column tile
         const int row = q * 32 + lane;
         const uint32_t acc_empty_leader0 = map_to_rank(bar_acc_empty, 0);
         uint32_t it_x = 0, it_a = 0;
         bool ok = true;
-        for (int64_t u = pair; u < P.units && ok; u += P.pairs, ++it_x) {
-            const int64_t b = u / P.units_per_batch;
-            const int64_t n = (u % P.units_per_batch) * kUnitRows + (int64_t)rank * kRows + row;
+        const int units = (int)P.units, pairs = (int)P.pairs;  // < 2^23: 32-bit counters
+        for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
             const uint32_t xb = it_x % kXBufs;
             float xnorm = 0.f;
             float best = -INFINITY;
-            int label = -1;
+            int gbest = -1;    // column of the first score of the group holding the running best
+            float kept[32];    // that group's 32 scores
+#pragma unroll
+            for (int j = 0; j < 32; ++j) kept[j] = -INFINITY;
             for (int kt = 0; kt < P.ktiles; ++kt, ++it_a) {
                 const uint32_t s = it_a % kAccSets;
                 if (!(ok = mbar_wait(bar_acc_full + 8 * s, (it_a / kAccSets) & 1, abort_flag, P.fault))) break;
@@ -394,7 +396,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // this warp's 64 columns of the tile, then hand the accumulator
                 // straight back so the MMA of tile t+2 is not held up by the math
                 float v[kPartCols];
-                tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + s * kTileK + h * kPartCols, v);
+                tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + s * kTileK + h * kPartCols, v);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
@@ -435,18 +437,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const float gmax = max3(max3(ga, w[30], w[31]), gb, gb);
                     const bool better = gmax > best;  // strict: an earlier group keeps ties
                     if (__any_sync(0xffffffffu, better)) {
-                        // first column of the group holding the maximum
-                        int j0 = 31;
 #pragma unroll
-                        for (int j = 31; j >= 0; --j) j0 = (w[j] == gmax) ? j : j0;
-                        if (better) {
-                            best = gmax;
-                            label = kt * kTileK + h * kPartCols + g * 32 + j0;
-                        }
+                        for (int j = 0; j < 32; ++j) kept[j] = better ? w[j] : kept[j];
+                    }
+                    if (better) {
+                        best = gmax;
+                        gbest = kt * kTileK + h * kPartCols + g * 32;
                     }
                 }
             }
             if (!ok) break;
+            // this slice's winner: the first column of the kept group holding the maximum
+            int j0 = 31;
+#pragma unroll
+            for (int j = 31; j >= 0; --j) j0 = (kept[j] == best) ? j : j0;
+            const int label = gbest < 0 ? -1 : gbest + j0;
             // join the column slices of each row (larger score, then lower
             // index) through a double-buffered shared slot with bounded handoffs
             const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
@@ -473,9 +478,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
+                const int upb = (int)P.units_per_batch;
+                const int b = u / upb;
+                const int n = (u - b * upb) * kUnitRows + (int)rank * kRows + row;
                 if (n < P.N) {
-                    P.labels[b * P.N + n] = fl;
-                    if (P.mindist) P.mindist[b * P.N + n] = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
+                    const int64_t o = (int64_t)b * P.N + n;
+                    P.labels[o] = fl;
+                    if (P.mindist) P.mindist[o] = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
                 }
             }
         }
