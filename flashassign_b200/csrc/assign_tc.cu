@@ -16,30 +16,31 @@
 //     pieces (exact to ~2^-33 relative), so one more K=16 MMA step adds the
 //     norm term in fp32 and the epilogue only tracks maxima.
 //   * CTA pairs (a cluster of 2) run tcgen05.mma.cta_group::2 with M=256,
-//     N=128, K=16: each CTA stages its own 128 point rows and its own half
-//     (64) of each 128-centroid tile, so each SM reads only half of the B
-//     operand.  Four 128-column accumulator sets fill the 512 TMEM columns:
-//     the MMAs may run three tiles ahead of the epilogue, which hides the
-//     completion -> epilogue -> release -> issue round trip (measured at
-//     more than one 256-column tile of MMA work, the reason for N=128).
+//     N=256, K=16: each CTA stages its own 128 point rows and its own half
+//     (128) of each 256-centroid tile, so every instruction runs at the full
+//     N=256 rate (128 cycles) while each SM reads only half of the B operand:
+//     about 64 B/cycle of operand reads plus ~31 B/cycle of TMA writes, within
+//     the shared-memory bandwidth (an N=128 tile would need ~125 B/cycle).
+//     Two 256-column accumulator sets fill the 512 TMEM columns.
 //   * Persistent grid of pairs; a work unit is 256 consecutive points of one
 //     batch; units are strided over the pairs so that pairs running at the
 //     same time share their batch's centroids in L2.
 //   * Warp roles per CTA: warp 0 issues TMA loads (one thread: X tiles of the
 //     units into two buffers; another: centroid tiles plus their norm slices
-//     into an 8-stage ring), completing on the leader CTA's barriers; warp 1 allocates TMEM
-//     for the pair; in the leader CTA, warps 1 and 10 issue the MMAs
-//     (alternate tiles: one thread issues at most ~1 MMA per 100 cycles) and
-//     commit them to both CTAs' barriers; warps 2..17 are the epilogue: TMEM lane = point
-//     row, four warps per row split each tile's 128 columns in 32-column
-//     slices; each reads its slice with one TMEM load and releases the
-//     accumulator before doing any arithmetic on it.
+//     into a 4-stage ring), completing on the leader CTA's barriers; warp 1
+//     allocates TMEM for the pair; in the leader CTA, warps 1 and 10 issue
+//     the MMAs (alternate tiles: one thread issues at most ~1 MMA per 100
+//     cycles) and commit them to both CTAs' barriers; warps 2..9 are the
+//     epilogue: TMEM lane = point row, two warps per row split each tile's
+//     256 columns in 128-column slices, read 64 columns at a time; the
+//     accumulator is released as soon as the last 64 are in registers.
 //   * Epilogue: per 32-column group, the group maximum (3-input max) is
 //     compared with the running best; only when it improves are the group's
 //     32 scores kept in registers, and the winning column is resolved once
-//     per unit from the kept group (first column equal to the maximum).  The two column slices of a row are
-//     joined in shared memory (larger score, then lower index).  mindist = ||x||^2 - 2 * best, ||x||^2 summed from the
-//     staged X tile.
+//     per unit from the kept group (first column equal to the maximum).  The
+//     two column slices of a row are joined in shared memory (larger score,
+//     then lower index).  mindist = ||x||^2 - 2 * best, ||x||^2 summed from
+//     the staged X tile.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records a fault code in the device fault word, stops issuing work, frees
 // its TMEM and returns.
@@ -52,13 +53,13 @@ namespace {
 
 constexpr int kRows = 128;                      // point rows per CTA per unit (TMEM lanes)
 constexpr int kUnitRows = 2 * kRows;            // points per unit (per CTA pair)
-constexpr int kTileK = kAssignTileK;            // centroids per K tile (MMA N) = 128
-constexpr int kHalfTile = kTileK / 2;           // centroids staged per CTA per tile (64)
+constexpr int kTileK = kAssignTileK;            // centroids per K tile (MMA N) = 256
+constexpr int kHalfTile = kTileK / 2;           // centroids staged per CTA per tile (128)
 constexpr int kBoxK = 64;                       // fp16 elements per 128-byte swizzle row
 constexpr int kMaxBoxes = 2;                    // d <= 128
-constexpr int kCStages = 8;
+constexpr int kCStages = 4;
 constexpr int kXBufs = 2;
-constexpr int kAccSets = 4;                     // 4 x 128 TMEM columns: the MMA may run 3 tiles ahead
+constexpr int kAccSets = 2;                     // 2 x 256 TMEM columns
 constexpr int kBoxBytes = 128 * 128;            // X: [128 rows x 64 fp16], 128-byte swizzled
 constexpr int kCBoxBytes = kHalfTile * 128;     // C: [64 centroids x 64 fp16], 128-byte swizzled
 constexpr int kExtBytes = 128 * 32;             // ones: [128 rows x 16 fp16], 32-byte swizzled
@@ -68,7 +69,7 @@ constexpr int kEpiWarp0 = 2;
 constexpr int kMmaWarpB = 10;                   // second issuer, on another SMSP than warp 1
 constexpr int kEpiWarps = 8;                    // at most 3 warps per SMSP: up to 168 registers each
 constexpr int kColParts = kEpiWarps / 4;        // warps per TMEM lane quarter, each with a column slice
-constexpr int kPartCols = kTileK / kColParts;   // 64 columns of each tile per epilogue warp
+constexpr int kPartCols = kTileK / kColParts;   // 128 columns of each tile per epilogue warp
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -76,7 +77,7 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kXOff = 0;
 constexpr int kXBytes = kXBufs * kMaxBoxes * kBoxBytes;             // 64 KB
 constexpr int kCOff = kXOff + kXBytes;
-constexpr int kCStageBytes = kMaxBoxes * kCBoxBytes + kCExtBytes;  // 18 KB: centroid boxes + norm slice
+constexpr int kCStageBytes = kMaxBoxes * kCBoxBytes + kCExtBytes;  // 36 KB: centroid boxes + norm slice
 constexpr int kCBytes = kCStages * kCStageBytes;                    // 144 KB
 constexpr int kAOnesOff = kCOff + kCBytes;                          // 4 KB of ones (the points' extra slice)
 constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 3 parts x 128 x (score, label)
@@ -374,7 +375,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ------------------------------ epilogue (both CTAs) ------------------------------
         const int e = warp - kEpiWarp0;
         const int q = warp % 4;   // TMEM lane quarter this warp may access
-        const int h = e / 4;      // which 64-column slice of each 128-column tile
+        const int h = e / 4;      // which 128-column slice of each 256-column tile
         const int row = q * 32 + lane;
         const uint32_t acc_empty_leader0 = map_to_rank(bar_acc_empty, 0);
         uint32_t it_x = 0, it_a = 0;
@@ -393,13 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!(ok = mbar_wait(bar_acc_full + 8 * s, (it_a / kAccSets) & 1, abort_flag, P.fault))) break;
                 __syncwarp();  // tcgen05.ld below is warp-collective
                 tc_fence_after();
-                // this warp's 64 columns of the tile, then hand the accumulator
-                // straight back so the MMA of tile t+2 is not held up by the math
-                float v[kPartCols];
-                tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + s * kTileK + h * kPartCols, v);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
+                const uint32_t tcol = tmem_base + ((uint32_t)(q * 32) << 16) + s * kTileK + h * kPartCols;
                 if (kt == 0) {
                     // The MMA has consumed this unit's X tile, so it is in place.
                     // ||x||^2 from it: the swizzle permutes 16-byte chunks within a
@@ -424,8 +419,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
                 }
+#pragma unroll 1
+                for (int sub = 0; sub < kPartCols / 64; ++sub) {
+                  // 64 columns at a time; the accumulator is handed back as soon as
+                  // its last columns are in registers, before their arithmetic
+                  float v[64];
+                  tmem_ld64(tcol + sub * 64, v);
+                  if (sub == kPartCols / 64 - 1) {
+                      tc_fence_before();
+                      __syncwarp();
+                      if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
+                  }
 #pragma unroll
-                for (int g = 0; g < kPartCols / 32; ++g) {
+                  for (int g = 0; g < 2; ++g) {
                     const float* w = v + 32 * g;
                     // two interleaved 3-input chains: few live temporaries
                     float ga = max3(w[0], w[1], w[2]), gb = max3(w[3], w[4], w[5]);
@@ -442,8 +448,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     if (better) {
                         best = gmax;
-                        gbest = kt * kTileK + h * kPartCols + g * 32;
+                        gbest = kt * kTileK + h * kPartCols + sub * 64 + g * 32;
                     }
+                  }
                 }
             }
             if (!ok) break;

@@ -23,7 +23,7 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Tile width of the tensor-core assignment along K; the centroids' norm-slice
 // array [B, padded_k(K), 16] is padded to a multiple of it with rows whose
 // score is -inf, so that padded columns never win.
-constexpr int kAssignTileK = 128;
+constexpr int kAssignTileK = 256;
 inline int64_t padded_k(int64_t K) { return ceil_div(K, kAssignTileK) * kAssignTileK; }
 
 struct DeviceInfo {
