@@ -282,8 +282,8 @@ km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, 
         return KM_E_INVALID;
     }
     KM_TRY(check_shape(B, N, K, d, dtype));
-    if (!aligned(X, 16) || !aligned(sums, 16) || !aligned(C_out, 4) || !aligned(labels, 4) || !aligned(counts, 4)) {
-        set_error("km_update: X and sums must be 16-byte aligned, the other arrays 4-byte aligned");
+    if (!aligned(X, 16) || !aligned(sums, 16) || !aligned(C_out, 16) || !aligned(labels, 4) || !aligned(counts, 4)) {
+        set_error("km_update: X, sums and C_out must be 16-byte aligned, labels and counts 4-byte aligned");
         return KM_E_UNSUPPORTED;
     }
     DeviceInfo dev;
@@ -301,12 +301,14 @@ km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, 
         KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * (size_t)(B * K * d), st), "zero sums"));
     }
     {
-        PhaseScope ph(st, KM_PHASE_SORT, sort_kernel_launches(N, K, false));
-        KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, offs, work, st), "label sort"));
+        PhaseScope ph(st, KM_PHASE_SORT, sort_kernel_launches(N, K, false, false));
+        KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
+                        "label sort"));
     }
     {
         PhaseScope ph(st, KM_PHASE_UPDATE, 1);
-        KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, st), "segmented update"));
+        KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, offs, st),
+                        "segmented update"));
     }
     PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
     return launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, nullptr, nullptr, counts, false, st),
@@ -371,7 +373,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         PhaseScope ph(st, KM_PHASE_OTHER, 0);
         KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * ckd, st), "zero sums"));
     }
-    const int sort_launches = sort_kernel_launches(N, K, false);
+    const int sort_launches = sort_kernel_launches(N, K, false, false);
     for (int t = 0; t < iters; ++t) {
         KM_TRY(run_assign(X, dtype, C_out, chat, cext, B, N, K, d, labels, mindist, dev, st));
         if (objective) {
@@ -380,11 +382,13 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         }
         {
             PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
-            KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, offs, work, st), "label sort"));
+            KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
+                            "label sort"));
         }
         {
             PhaseScope ph(st, KM_PHASE_UPDATE, 1);
-            KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, st), "segmented update"));
+            KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, offs, st),
+                            "segmented update"));
         }
         const bool prep_next = tc && t + 1 < iters;
         PhaseScope ph(st, KM_PHASE_FINALIZE, 1);

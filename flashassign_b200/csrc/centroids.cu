@@ -26,13 +26,14 @@ __device__ __forceinline__ double warp_sum(double v) {
 // nearest fp16 to what is left, clamped to the fp16 range).
 __device__ __forceinline__ void write_norm_slice(__half* out, double v) {
     double r = -v;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    int i = 0;
+    for (; i < 16 && r != 0.0; ++i) {  // typically 3-4 pieces leave nothing
         const double c = fmin(fmax(r, -65504.0), 65504.0);
         const __half p = __float2half_rn((float)c);
         out[i] = p;
         r -= (double)__half2float(p);
     }
+    for (; i < 16; ++i) out[i] = __float2half(0.f);
 }
 
 __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, int64_t Kp, int64_t d, int dtype,
@@ -75,21 +76,27 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
     const float fn = (float)n;
     const int64_t base = row * d;
     double acc = 0.0;
-    for (int64_t j = lane; j < d; j += 32) {
-        float v;
+    // four consecutive coordinates per lane (d is a multiple of 4)
+    for (int64_t j = 4 * lane; j < d; j += 128) {
+        float4 v;
         if (n > 0) {
-            v = sums[base + j] / fn;
-            C_out[base + j] = v;
-            if (zero_sums) sums[base + j] = 0.f;
+            const float4 sv = *reinterpret_cast<const float4*>(sums + base + j);
+            v = make_float4(sv.x / fn, sv.y / fn, sv.z / fn, sv.w / fn);
+            *reinterpret_cast<float4*>(C_out + base + j) = v;
+            if (zero_sums) *reinterpret_cast<float4*>(sums + base + j) = make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
-            v = C_out[base + j];
+            v = *reinterpret_cast<const float4*>(C_out + base + j);
         }
         if (dtype == KM_F16) {
-            const __half h = __float2half_rn(v);
-            if (chat) chat[base + j] = h;
-            v = __half2float(h);
+            const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+            if (chat) {
+                *reinterpret_cast<__half2*>(chat + base + j) = h01;
+                *reinterpret_cast<__half2*>(chat + base + j + 2) = h23;
+            }
+            const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+            v = make_float4(f01.x, f01.y, f23.x, f23.y);
         }
-        acc += (double)v * (double)v;
+        acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
     }
     if (cext) {
         acc = warp_sum(acc);

@@ -60,13 +60,18 @@ cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t
 
 // Stable LSD radix argsort of labels in [0, K).  Scratch: sort_scratch_bytes().
 size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K);
-int sort_kernel_launches(int64_t N, int64_t K, bool with_counts);
+int sort_kernel_launches(int64_t N, int64_t K, bool with_counts, bool bounds = true);
+// With bounds = false the segment offsets (and counts) are left to the caller
+// (the update kernel writes them while it walks the sorted labels).
 cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* a_sorted,
-                        int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st);
+                        int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st,
+                        bool bounds = true);
 
-// Segmented gather-reduce over the sorted order (sums must be zeroed first).
+// Segmented gather-reduce over the sorted order (sums must be zeroed first);
+// when offsets [B, K+1] is non-null it also writes the segment offsets.
 cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
-                               int64_t B, int64_t N, int64_t K, int64_t d, float* sums, cudaStream_t st);
+                               int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
+                               cudaStream_t st);
 
 // objective[b] = sum_i mindist[b][i] (fp32, one block per batch).
 cudaError_t launch_objective(const float* mindist, int64_t B, int64_t N, float* objective, cudaStream_t st);

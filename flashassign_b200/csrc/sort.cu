@@ -8,9 +8,11 @@
 // two 5-bit passes; K=65536: two 8-bit passes).  Each pass is
 //   1. a per-tile digit histogram (2048 keys per CTA),
 //   2. an exclusive scan over (digit, tile) per batch,
-//   3. a scatter in which each warp ranks its keys with __match_any_sync and
-//      the warps of a tile are combined by a per-digit scan, so equal digits
-//      keep their input order (stability).
+//   3. a scatter in which each warp ranks its keys with __match_any_sync, the
+//      warps of a tile are combined by a per-digit scan (equal digits keep
+//      their input order: stability), the tile is laid out digit by digit in
+//      shared memory, and each digit's run is written to consecutive global
+//      positions (coalesced stores).
 // The segment offsets and counts then follow from the sorted labels without
 // any atomics: position p starts label k exactly when a[p-1] < k <= a[p].
 #include "km_internal.cuh"
@@ -107,13 +109,17 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
                                                                  int32_t* __restrict__ vals_out, int64_t N, int shift,
                                                                  int bits, int64_t T,
                                                                  const int32_t* __restrict__ offs) {
-    __shared__ int wh[kWarps][256];
+    __shared__ int wh[kWarps][256];      // per-warp digit counts, then per-warp exclusive offsets
+    __shared__ int tstart[256];          // first tile-local position of each digit
+    __shared__ int s_key[kTile];         // the tile's keys in tile-sorted (stable) order
+    __shared__ int s_val[kTile];
     const int64_t b = blockIdx.y, tile = blockIdx.x;
     const int bins = 1 << bits, mask = bins - 1;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     for (int t = threadIdx.x; t < kWarps * 256; t += kThreads) (&wh[0][0])[t] = 0;
     __syncthreads();
 
+    // 1. rank each key among the equal digits before it (warp by warp, in input order)
     const uint32_t lt = (1u << lane) - 1u;
     const int64_t base = tile * kTile + (int64_t)w * (kItems * 32);
     int key[kItems], val[kItems], rank[kItems];
@@ -132,25 +138,52 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
         __syncwarp();
     }
     __syncthreads();
+    // 2. per digit: exclusive offsets across warps, and the digit's total in this tile
+    int total = 0;
     if (threadIdx.x < bins) {
-        int run = 0;
 #pragma unroll
         for (int ww = 0; ww < kWarps; ++ww) {
             const int t = wh[ww][threadIdx.x];
-            wh[ww][threadIdx.x] = run;
-            run += t;
+            wh[ww][threadIdx.x] = total;
+            total += t;
         }
     }
+    // 3. exclusive scan of the digit totals (bins <= 256 = kThreads): where each digit starts in the tile
+    {
+        __shared__ int warp_sum[kWarps];
+        int incl = total;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_sum[w] = incl;
+        __syncthreads();
+        int before = 0;
+        for (int ww = 0; ww < w; ++ww) before += warp_sum[ww];
+        if (threadIdx.x < bins) tstart[threadIdx.x] = before + incl - total;
+    }
     __syncthreads();
+    // 4. place the keys in tile-sorted order in shared memory
 #pragma unroll
     for (int s = 0; s < kItems; ++s) {
         const int64_t i = base + s * 32 + lane;
         if (i < N) {
             const int dig = (key[s] >> shift) & mask;
-            const int64_t pos = (int64_t)offs[(b * bins + dig) * T + tile] + wh[w][dig] + rank[s];
-            keys_out[b * N + pos] = key[s];
-            vals_out[b * N + pos] = val[s];
+            const int lp = tstart[dig] + wh[w][dig] + rank[s];
+            s_key[lp] = key[s];
+            s_val[lp] = val[s];
         }
+    }
+    __syncthreads();
+    // 5. write out: consecutive tile positions of one digit go to consecutive global positions
+    const int n_here = (int)min((int64_t)kTile, N - tile * kTile);
+    for (int lp = threadIdx.x; lp < n_here; lp += kThreads) {
+        const int k = s_key[lp];
+        const int dig = (k >> shift) & mask;
+        const int64_t pos = (int64_t)offs[(b * bins + dig) * T + tile] + (lp - tstart[dig]);
+        keys_out[b * N + pos] = k;
+        vals_out[b * N + pos] = s_val[lp];
     }
 }
 
@@ -174,8 +207,8 @@ __global__ void counts_kernel(const int32_t* __restrict__ offsets, int64_t B, in
 
 }  // namespace
 
-int sort_kernel_launches(int64_t N, int64_t K, bool with_counts) {
-    return 3 * make_plan(N, K).passes + 1 + (with_counts ? 1 : 0);
+int sort_kernel_launches(int64_t N, int64_t K, bool with_counts, bool bounds) {
+    return 3 * make_plan(N, K).passes + (bounds ? 1 + (with_counts ? 1 : 0) : 0);
 }
 
 size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K) {
@@ -188,7 +221,8 @@ size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K) {
 }
 
 cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* a_sorted,
-                        int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st) {
+                        int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st,
+                        bool bounds) {
     const Plan p = make_plan(N, K);
     int32_t* tmp_k = (int32_t*)scratch;
     int32_t* tmp_v = tmp_k + B * N;
@@ -211,8 +245,10 @@ cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, 
         in_k = out_k;
         in_v = out_v;
     }
-    seg_bounds_kernel<<<dim3((unsigned)ceil_div(N + 1, 256), (unsigned)B), 256, 0, st>>>(a_sorted, N, K, offsets);
-    if (counts) counts_kernel<<<(unsigned)ceil_div(B * K, 256), 256, 0, st>>>(offsets, B, K, counts);
+    if (bounds) {
+        seg_bounds_kernel<<<dim3((unsigned)ceil_div(N + 1, 256), (unsigned)B), 256, 0, st>>>(a_sorted, N, K, offsets);
+        if (counts) counts_kernel<<<(unsigned)ceil_div(B * K, 256), 256, 0, st>>>(offsets, B, K, counts);
+    }
     return cudaGetLastError();
 }
 

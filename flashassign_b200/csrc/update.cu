@@ -7,8 +7,9 @@
 // The page's count of O((K + ceil(N / B_N)) d) atomic additions is met
 // exactly: at most two intervals per CTA are added atomically; every other
 // interval is a whole cluster owned by this CTA and is written with a plain
-// store.  Cluster counts come from the sort's segment offsets (exact
-// integers), so no counter atomics are needed at all.
+// store.  Cluster counts come from the segment offsets of the sorted labels
+// (exact integers), which this kernel also writes while it walks them, so no
+// counter atomics and no separate pass are needed.
 //
 // Layout of a CTA (16-byte chunks of a row per thread):
 //   tpr = d * sizeof(T) / 16 threads cover one row; G = 256 / tpr row-lanes;
@@ -57,7 +58,8 @@ struct Chunk<float> {
 template <typename T>
 __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, const int32_t* __restrict__ a_sorted,
                                                      const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
-                                                     int64_t d, int tpr, int G, float* __restrict__ sums) {
+                                                     int64_t d, int tpr, int G, float* __restrict__ sums,
+                                                     int32_t* __restrict__ offsets) {
     constexpr int E = Chunk<T>::kElems;
     extern __shared__ __align__(16) unsigned char smem[];
     const int BN = G * kRowsPerLane;
@@ -78,6 +80,21 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         s_idx[t] = sorted_idx[b * N + p0 + t];
     }
     __syncthreads();
+    if (offsets) {
+        // Segment offsets of the sorted labels: position p starts every label k
+        // with a[p-1] < k <= a[p] (labels clamped so nothing is written out of
+        // bounds); the last run also closes labels above a[N-1] at N.
+        int32_t* ob = offsets + b * (K + 1);
+        for (int t = threadIdx.x; t <= n; t += blockDim.x) {
+            const int64_t p = p0 + t;
+            if (t == n && p != N) break;
+            int64_t prev = t > 0 ? s_lab[t - 1] : (p0 > 0 ? ab[p0 - 1] : -1);
+            int64_t cur = p == N ? K : s_lab[t];
+            prev = min(max(prev, (int64_t)-1), K);
+            cur = min(max(cur, (int64_t)-1), K);
+            for (int64_t k = prev + 1; k <= cur; ++k) ob[k] = (int32_t)p;
+        }
+    }
 
     const int g = threadIdx.x / tpr, c = threadIdx.x % tpr;
     const int r0 = g * kRowsPerLane, r1 = min(r0 + kRowsPerLane, n);
@@ -176,7 +193,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
 
 template <typename T>
 cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sorted_idx, int64_t B, int64_t N,
-                     int64_t K, int64_t d, float* sums, cudaStream_t st) {
+                     int64_t K, int64_t d, float* sums, int32_t* offsets, cudaStream_t st) {
     const int tpr = (int)(d * (int64_t)sizeof(T) / 16);
     const int G = 256 / tpr;
     const int BN = G * kRowsPerLane;
@@ -186,16 +203,18 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
         if (e != cudaSuccess) return e;
     }
     const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B);
-    update_kernel<T><<<grid, G * tpr, smem, st>>>((const T*)X, a_sorted, sorted_idx, N, K, d, tpr, G, sums);
+    update_kernel<T><<<grid, G * tpr, smem, st>>>((const T*)X, a_sorted, sorted_idx, N, K, d, tpr, G, sums,
+                                                  offsets);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
-                               int64_t B, int64_t N, int64_t K, int64_t d, float* sums, cudaStream_t st) {
-    if (dtype == KM_F16) return launch_t<__half>(X, a_sorted, sorted_idx, B, N, K, d, sums, st);
-    return launch_t<float>(X, a_sorted, sorted_idx, B, N, K, d, sums, st);
+                               int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
+                               cudaStream_t st) {
+    if (dtype == KM_F16) return launch_t<__half>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, st);
+    return launch_t<float>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, st);
 }
 
 }  // namespace km

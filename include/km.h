@@ -24,8 +24,9 @@
  *     Every call is asynchronous on it: results are ready once the stream is
  *     synchronised.  Argument errors return before any work is enqueued.
  *   - Supported: B >= 1, N >= 1, K >= 1, B*N < 2^31, K < 2^24, 1 <= d <= 512,
- *     d * sizeof(dtype) a multiple of 16 bytes, X and C 16-byte aligned,
- *     every other array 4-byte aligned, a device of compute capability 10.0.
+ *     d * sizeof(dtype) a multiple of 16 bytes, X and the [B, K, d] arrays
+ *     (C, C_init, C_out, sums) 16-byte aligned, every other array 4-byte
+ *     aligned, a device of compute capability 10.0.
  *     Anything else returns KM_E_UNSUPPORTED (KM_E_INVALID for null pointers
  *     and non-positive sizes).  There is no CPU fallback.
  *   - Inputs must be finite; non-finite values are outside the contract.

@@ -63,6 +63,11 @@ def test_assign_rejects_bad_arguments_before_touching_the_device(args, expect):
     assert km.lib().km_last_error()
 
 
+def test_update_rejects_misaligned_centroids_before_touching_the_device():
+    rc = km.lib().km_update(FAKE, FAKE, 1, 64, 4, 16, km.KM_F32, FAKE, FAKE, ctypes.c_void_p(0x10004), None)
+    assert rc == 2 and b"16-byte" in km.lib().km_last_error()
+
+
 def test_update_and_sort_and_lloyd_reject_nulls():
     L = km.lib()
     assert L.km_update(None, FAKE, 1, 10, 2, 16, 0, FAKE, FAKE, FAKE, None) == 1
