@@ -150,13 +150,15 @@ km_status launched(cudaError_t e, const char* what) {
 
 // The assignment for one iteration, given prepared centroids.
 km_status run_assign(const void* X, int dtype, const float* C, const __half* chat, const __half* cext, int64_t B,
-                     int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, const DeviceInfo& dev,
-                     cudaStream_t st) {
+                     int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
+                     const DeviceInfo& dev, cudaStream_t st) {
     PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
     if (dtype == KM_F16 && assign_tc_supported(d, dtype))
-        return launched(launch_assign_tc((const __half*)X, chat, cext, B, N, K, d, labels, mindist, dev.sms, st),
-                        "assign (tensor cores)");
-    return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, st), "assign (CUDA cores)");
+        return launched(
+            launch_assign_tc((const __half*)X, chat, cext, B, N, K, d, labels, mindist, obj_acc, dev.sms, st),
+            "assign (tensor cores)");
+    return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st),
+                    "assign (CUDA cores)");
 }
 
 bool uses_tc(int dtype, int64_t d) { return dtype == KM_F16 && assign_tc_supported(d, dtype); }
@@ -247,7 +249,7 @@ km_status km_assign(const void* X, const float* C, int64_t B, int64_t N, int64_t
         PhaseScope ph(st, KM_PHASE_PREP, 1);
         KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, chat, cext, st), "centroid preparation"));
     }
-    return run_assign(X, dtype, C, chat, cext, B, N, K, d, labels, mindist, dev, st);
+    return run_assign(X, dtype, C, chat, cext, B, N, K, d, labels, mindist, nullptr, dev, st);
 }
 
 km_status km_sort_labels(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* sorted_idx,
@@ -311,8 +313,9 @@ km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, 
                         "segmented update"));
     }
     PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
-    return launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, nullptr, nullptr, counts, false, st),
-                    "centroid finalize");
+    return launched(
+        launch_finalize(sums, offs, B, K, d, C_out, dtype, nullptr, nullptr, counts, false, nullptr, nullptr, st),
+        "centroid finalize");
 }
 
 km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
@@ -351,14 +354,15 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     Scratch scratch(st);
     const bool tc = uses_tc(dtype, d);
     __half *chat = nullptr, *cext = nullptr;
-    float *mindist = nullptr, *sums = nullptr;
+    float* sums = nullptr;
+    double* obj_acc = nullptr;
     int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
     unsigned char* work = nullptr;
     if (tc) {
         KM_TRY(scratch.get(&chat, ckd, "rounded centroids"));
         KM_TRY(scratch.get(&cext, (size_t)(B * padded_k(K) * 16), "centroid norm slices"));
     }
-    KM_TRY(scratch.get(&mindist, (size_t)(B * N), "minimum distances"));
+    if (objective) KM_TRY(scratch.get(&obj_acc, (size_t)B, "objective accumulator"));
     KM_TRY(scratch.get(&sums, ckd, "cluster sums"));
     KM_TRY(scratch.get(&offs, (size_t)(B * (K + 1)), "segment offsets"));
     KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
@@ -372,14 +376,11 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     {
         PhaseScope ph(st, KM_PHASE_OTHER, 0);
         KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * ckd, st), "zero sums"));
+        if (obj_acc) KM_TRY(launched(cudaMemsetAsync(obj_acc, 0, sizeof(double) * B, st), "zero objective"));
     }
     const int sort_launches = sort_kernel_launches(N, K, false, false);
     for (int t = 0; t < iters; ++t) {
-        KM_TRY(run_assign(X, dtype, C_out, chat, cext, B, N, K, d, labels, mindist, dev, st));
-        if (objective) {
-            PhaseScope ph(st, KM_PHASE_OTHER, 1);
-            KM_TRY(launched(launch_objective(mindist, B, N, objective + (size_t)t * B, st), "objective"));
-        }
+        KM_TRY(run_assign(X, dtype, C_out, chat, cext, B, N, K, d, labels, nullptr, obj_acc, dev, st));
         {
             PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
             KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
@@ -394,7 +395,8 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
         // the finalize zeroes the consumed sums, so the next update starts from 0
         KM_TRY(launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
-                                        prep_next ? cext : nullptr, nullptr, true, st),
+                                        prep_next ? cext : nullptr, nullptr, true, obj_acc,
+                                        objective ? objective + (size_t)t * B : nullptr, st),
                         "centroid finalize"));
     }
     return KM_OK;

@@ -28,7 +28,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restrict__ X, const float* __restrict__ C,
                                                                int64_t N, int64_t K, int64_t d,
                                                                int32_t* __restrict__ labels,
-                                                               float* __restrict__ mindist) {
+                                                               float* __restrict__ mindist,
+                                                               double* __restrict__ obj_acc) {
     __shared__ float xs[kThreads][kTileD + 1];
     __shared__ float cs[kTileK][kTileD + 1];
     const int64_t b = blockIdx.y;
@@ -82,17 +83,23 @@ __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restri
         labels[b * N + i] = arg;
         if (mindist) mindist[b * N + i] = best;
     }
+    if (obj_acc) {  // the objective: one atomic per warp
+        double part = i < N ? (double)best : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if ((threadIdx.x & 31) == 0) atomicAdd(obj_acc + b, part);
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
-                               int32_t* labels, float* mindist, cudaStream_t st) {
+                               int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st) {
     dim3 grid((unsigned)ceil_div(N, kThreads), (unsigned)B);
     if (dtype == KM_F16)
-        assign_simt_kernel<__half><<<grid, kThreads, 0, st>>>((const __half*)X, C, N, K, d, labels, mindist);
+        assign_simt_kernel<__half><<<grid, kThreads, 0, st>>>((const __half*)X, C, N, K, d, labels, mindist, obj_acc);
     else
-        assign_simt_kernel<float><<<grid, kThreads, 0, st>>>((const float*)X, C, N, K, d, labels, mindist);
+        assign_simt_kernel<float><<<grid, kThreads, 0, st>>>((const float*)X, C, N, K, d, labels, mindist, obj_acc);
     return cudaGetLastError();
 }
 

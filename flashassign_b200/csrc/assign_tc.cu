@@ -227,6 +227,7 @@ struct Params {
     int ktiles, ksteps, boxes;
     int32_t* labels;
     float* mindist;
+    double* obj_acc;  // [B] running sum of minimum distances, nullable
     int32_t* fault;
 };
 
@@ -488,10 +489,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int upb = (int)P.units_per_batch;
                 const int b = u / upb;
                 const int n = (u - b * upb) * kUnitRows + (int)rank * kRows + row;
+                const float md = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
                 if (n < P.N) {
                     const int64_t o = (int64_t)b * P.N + n;
                     P.labels[o] = fl;
-                    if (P.mindist) P.mindist[o] = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
+                    if (P.mindist) P.mindist[o] = md;
+                }
+                if (P.obj_acc) {  // the objective: this warp's 32 rows, one atomic per warp
+                    double part = n < P.N ? (double)md : 0.0;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                    if (lane == 0) atomicAdd(P.obj_acc + b, part);
                 }
             }
         }
@@ -546,7 +554,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t B, int64_t rows, int64_t
 bool assign_tc_supported(int64_t d, int dtype) { return dtype == KM_F16 && d >= 64 && d <= 128 && d % 8 == 0; }
 
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
-                             int64_t d, int32_t* labels, float* mindist, int sms, cudaStream_t st) {
+                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st) {
     if (!assign_tc_supported(d, KM_F16)) return cudaErrorNotSupported;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -564,6 +572,7 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* 
     P.boxes = (int)ceil_div(d, kBoxK);
     P.labels = labels;
     P.mindist = mindist;
+    P.obj_acc = obj_acc;
     P.fault = fault_word();
     // co-resident CTA pairs (a GPC with an odd number of free SMs cannot host a whole pair)
     static int pair_cache[64] = {0};

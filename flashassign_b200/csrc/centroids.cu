@@ -5,7 +5,8 @@
 //    ||c||^2 - 2 x.c, papernotes.org "Flash-KMeans" page, 关键设计 1);
 //  * finalisation of the update: c_k = s_k / n_k, an empty cluster keeping its
 //    previous centroid (the flowchart's C_new on the same page, 整体框架);
-//  * the per-batch objective sum of the minimum distances.
+//  * the per-batch objective: the assignment accumulates the sum of minimum
+//    distances, the finalisation hands it out and resets the accumulator.
 // All three are tiny next to the assignment and the gather; one warp per
 // centroid row keeps them coalesced.
 #include "km_internal.cuh"
@@ -66,9 +67,14 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
 // sums are reset to 0, ready for the next iteration's boundary atomics.
 __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t B, int64_t K,
                                 int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype, __half* __restrict__ chat,
-                                __half* __restrict__ cext, int32_t* __restrict__ counts, int zero_sums) {
+                                __half* __restrict__ cext, int32_t* __restrict__ counts, int zero_sums,
+                                double* __restrict__ obj_acc, float* __restrict__ obj_out) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
+    if (obj_out && row < B && lane == 0) {  // this iteration's objective, and a fresh accumulator
+        obj_out[row] = (float)obj_acc[row];
+        obj_acc[row] = 0.0;
+    }
     if (row >= B * K) return;
     const int64_t b = row / K, k = row % K;
     const int32_t n = offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
@@ -78,9 +84,11 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
     double acc = 0.0;
     // four consecutive coordinates per lane (d is a multiple of 4)
     for (int64_t j = 4 * lane; j < d; j += 128) {
+        // the sums are read whatever the count (zero for an empty cluster), so the
+        // load does not wait for the offsets
+        const float4 sv = *reinterpret_cast<const float4*>(sums + base + j);
         float4 v;
         if (n > 0) {
-            const float4 sv = *reinterpret_cast<const float4*>(sums + base + j);
             v = make_float4(sv.x / fn, sv.y / fn, sv.z / fn, sv.w / fn);
             *reinterpret_cast<float4*>(C_out + base + j) = v;
             if (zero_sums) *reinterpret_cast<float4*>(sums + base + j) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -104,35 +112,6 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
     }
 }
 
-__global__ void objective_kernel(const float* __restrict__ mindist, int64_t N, float* __restrict__ objective) {
-    const int64_t b = blockIdx.x;
-    const float* m = mindist + b * N;
-    double acc = 0.0;
-    // 16-byte loads where the batch row is aligned (N % 4 == 0), with four
-    // independent partial sums to keep several loads in flight
-    if ((N & 3) == 0) {
-        const float4* m4 = reinterpret_cast<const float4*>(m);
-        const int64_t n4 = N / 4;
-        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-        for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
-            const float4 v = __ldg(m4 + i);
-            a0 += v.x; a1 += v.y; a2 += v.z; a3 += v.w;
-        }
-        acc = (a0 + a1) + (a2 + a3);
-    } else {
-        for (int64_t i = threadIdx.x; i < N; i += blockDim.x) acc += (double)m[i];
-    }
-    acc = warp_sum(acc);
-    __shared__ double part[32];
-    if ((threadIdx.x & 31) == 0) part[threadIdx.x / 32] = acc;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        double v = threadIdx.x < blockDim.x / 32 ? part[threadIdx.x] : 0.0;
-        v = warp_sum(v);
-        if (threadIdx.x == 0) objective[b] = (float)v;
-    }
-}
-
 }  // namespace
 
 cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
@@ -145,16 +124,13 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
 }
 
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
-                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, cudaStream_t st) {
+                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, double* obj_acc,
+                            float* obj_out, cudaStream_t st) {
     const int warps = 8;
     finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(
-        sums, offsets, B, K, padded_k(K), d, C_out, dtype, chat, cext, counts, zero_sums ? 1 : 0);
+        sums, offsets, B, K, padded_k(K), d, C_out, dtype, chat, cext, counts, zero_sums ? 1 : 0, obj_acc, obj_out);
     return cudaGetLastError();
 }
 
-cudaError_t launch_objective(const float* mindist, int64_t B, int64_t N, float* objective, cudaStream_t st) {
-    objective_kernel<<<(unsigned)B, 1024, 0, st>>>(mindist, N, objective);
-    return cudaGetLastError();
-}
 
 }  // namespace km

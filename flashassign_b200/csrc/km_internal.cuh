@@ -44,19 +44,22 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
 // segment offsets [B, K+1] (and written to counts when non-null); when chat
 // or cext is non-null, also prepares the next assignment's centroids from
 // C_out; with zero_sums the sums are reset to 0 once consumed.
+// When obj_out is non-null, obj_out[b] = obj_acc[b] (as fp32) and obj_acc[b] = 0.
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
-                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, cudaStream_t st);
+                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, double* obj_acc,
+                            float* obj_out, cudaStream_t st);
 
 // Tensor-core assignment (fp16, 64 <= d <= 128).  Returns cudaErrorNotSupported
 // for shapes it does not take.
 bool assign_tc_supported(int64_t d, int dtype);
+// obj_acc (nullable, [B] double) accumulates the sum of minimum distances.
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
-                             int64_t d, int32_t* labels, float* mindist, int sms, cudaStream_t st);
+                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st);
 
 // CUDA-core assignment for every supported shape (fp32 inputs, and fp16
 // shapes outside the tensor-core kernel's range): direct-difference distances.
 cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
-                               int32_t* labels, float* mindist, cudaStream_t st);
+                               int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st);
 
 // Stable LSD radix argsort of labels in [0, K).  Scratch: sort_scratch_bytes().
 size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K);
@@ -73,7 +76,5 @@ cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted
                                int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
                                cudaStream_t st);
 
-// objective[b] = sum_i mindist[b][i] (fp32, one block per batch).
-cudaError_t launch_objective(const float* mindist, int64_t B, int64_t N, float* objective, cudaStream_t st);
 
 }  // namespace km

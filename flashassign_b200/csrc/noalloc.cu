@@ -86,7 +86,7 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
     cudaStream_t stm = (cudaStream_t)stream;
     const bool tc = dtype == KM_F16 && assign_tc_supported(d, dtype);
     if (!tc) {  // the CUDA-core kernel reads C directly and needs no scratch
-        cudaError_t e = launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, stm);
+        cudaError_t e = launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, nullptr, stm);
         return e == cudaSuccess ? KM_OK : cuda_error(e, "km_assign_noalloc: assign (CUDA cores)");
     }
     const size_t chat_bytes = round_up(sizeof(__half) * (size_t)(B * K * d), 256);
@@ -104,6 +104,7 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
     // every element of both scratch regions that the assignment reads is written here first
     cudaError_t e = launch_prep_centroids(C, B, K, d, dtype, chat, cext, stm);
     if (e != cudaSuccess) return cuda_error(e, "km_assign_noalloc: centroid preparation");
-    e = launch_assign_tc(static_cast<const __half*>(X), chat, cext, B, N, K, d, labels, mindist, dev.sms, stm);
+    e = launch_assign_tc(static_cast<const __half*>(X), chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms,
+                         stm);
     return e == cudaSuccess ? KM_OK : cuda_error(e, "km_assign_noalloc: assign (tensor cores)");
 }

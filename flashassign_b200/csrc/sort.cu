@@ -7,7 +7,8 @@
 // digits of at most 8 bits: ceil(log2 K) bits in ceil(bits/8) passes (K=1024:
 // two 5-bit passes; K=65536: two 8-bit passes).  Each pass is
 //   1. a per-tile digit histogram (2048 keys per CTA),
-//   2. an exclusive scan over (digit, tile) per batch,
+//   2. an exclusive scan over (digit, tile) per batch (done by each scatter
+//      CTA itself when the histogram is small),
 //   3. a scatter in which each warp ranks its keys with __match_any_sync, the
 //      warps of a tile are combined by a per-digit scan (equal digits keep
 //      their input order: stability), the tile is laid out digit by digit in
@@ -47,6 +48,10 @@ Plan make_plan(int64_t N, int64_t K) {
     p.tiles = ceil_div(N, kTile);
     return p;
 }
+
+// A histogram of at most this many (digit, tile) entries per batch is summed
+// by each scatter CTA itself instead of a separate scan pass.
+bool small_hist(int bins, int64_t tiles) { return (int64_t)bins * tiles <= 8192; }
 
 __global__ void __launch_bounds__(kThreads) radix_hist_kernel(const int32_t* __restrict__ keys, int64_t N, int shift,
                                                               int bits, int64_t T, int32_t* __restrict__ hist) {
@@ -108,8 +113,10 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
                                                                  int32_t* __restrict__ keys_out,
                                                                  int32_t* __restrict__ vals_out, int64_t N, int shift,
                                                                  int bits, int64_t T,
-                                                                 const int32_t* __restrict__ offs) {
+                                                                 const int32_t* __restrict__ offs,
+                                                                 const int32_t* __restrict__ hist) {
     __shared__ int wh[kWarps][256];      // per-warp digit counts, then per-warp exclusive offsets
+    __shared__ int gstart[256];          // global first position of each digit of this tile (hist path)
     __shared__ int tstart[256];          // first tile-local position of each digit
     __shared__ int s_key[kTile];         // the tile's keys in tile-sorted (stable) order
     __shared__ int s_val[kTile];
@@ -176,12 +183,41 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
         }
     }
     __syncthreads();
-    // 5. write out: consecutive tile positions of one digit go to consecutive global positions
+    // 5. global start of each digit of this tile.  With a small histogram the
+    //    CTA sums it itself (all earlier digits of the batch plus this digit's
+    //    earlier tiles); otherwise the scanned offsets are read.
+    if (hist) {
+        __shared__ int wsum[kWarps];
+        int tot = 0, mine = 0;
+        if (threadIdx.x < bins) {
+            const int32_t* hd = hist + (b * bins + threadIdx.x) * T;
+            for (int64_t t2 = 0; t2 < T; ++t2) {
+                const int c = hd[t2];
+                tot += c;
+                if (t2 < tile) mine += c;
+            }
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[w] = incl;
+        __syncthreads();
+        int before = 0;
+        for (int ww = 0; ww < w; ++ww) before += wsum[ww];
+        if (threadIdx.x < bins) gstart[threadIdx.x] = before + incl - tot + mine;
+    } else if (threadIdx.x < bins) {
+        gstart[threadIdx.x] = offs[(b * bins + threadIdx.x) * T + tile];
+    }
+    __syncthreads();
+    // 6. write out: consecutive tile positions of one digit go to consecutive global positions
     const int n_here = (int)min((int64_t)kTile, N - tile * kTile);
     for (int lp = threadIdx.x; lp < n_here; lp += kThreads) {
         const int k = s_key[lp];
         const int dig = (k >> shift) & mask;
-        const int64_t pos = (int64_t)offs[(b * bins + dig) * T + tile] + (lp - tstart[dig]);
+        const int64_t pos = (int64_t)gstart[dig] + (lp - tstart[dig]);
         keys_out[b * N + pos] = k;
         vals_out[b * N + pos] = s_val[lp];
     }
@@ -208,7 +244,10 @@ __global__ void counts_kernel(const int32_t* __restrict__ offsets, int64_t B, in
 }  // namespace
 
 int sort_kernel_launches(int64_t N, int64_t K, bool with_counts, bool bounds) {
-    return 3 * make_plan(N, K).passes + (bounds ? 1 + (with_counts ? 1 : 0) : 0);
+    const Plan p = make_plan(N, K);
+    int n = 0;
+    for (int i = 0; i < p.passes; ++i) n += small_hist(1 << p.bits[i], p.tiles) ? 2 : 3;
+    return n + (bounds ? 1 + (with_counts ? 1 : 0) : 0);
 }
 
 size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K) {
@@ -239,9 +278,14 @@ cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, 
         int32_t* out_v = to_final ? sorted_idx : tmp_v;
         const int bins = 1 << p.bits[i];
         radix_hist_kernel<<<grid, kThreads, 0, st>>>(in_k, N, p.shift[i], p.bits[i], p.tiles, hist);
-        exclusive_scan_kernel<<<(unsigned)B, 1024, 0, st>>>(hist, (int64_t)bins * p.tiles);
-        radix_scatter_kernel<<<grid, kThreads, 0, st>>>(in_k, in_v, out_k, out_v, N, p.shift[i], p.bits[i], p.tiles,
-                                                        hist);
+        if (small_hist(bins, p.tiles)) {
+            radix_scatter_kernel<<<grid, kThreads, 0, st>>>(in_k, in_v, out_k, out_v, N, p.shift[i], p.bits[i],
+                                                            p.tiles, nullptr, hist);
+        } else {
+            exclusive_scan_kernel<<<(unsigned)B, 1024, 0, st>>>(hist, (int64_t)bins * p.tiles);
+            radix_scatter_kernel<<<grid, kThreads, 0, st>>>(in_k, in_v, out_k, out_v, N, p.shift[i], p.bits[i],
+                                                            p.tiles, hist, nullptr);
+        }
         in_k = out_k;
         in_v = out_v;
     }
