@@ -5,11 +5,13 @@
 #include "km_internal.cuh"
 
 #include <atomic>
+#include <chrono>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <thread>
 #include <vector>
 
 namespace km {
@@ -162,6 +164,167 @@ km_status run_assign(const void* X, int dtype, const float* C, const __half* cha
 }
 
 bool uses_tc(int dtype, int64_t d) { return dtype == KM_F16 && assign_tc_supported(d, dtype); }
+
+std::atomic<int64_t> g_chunk_rows{0};
+constexpr int64_t kDefaultChunkRows = int64_t(1) << 23;
+constexpr int kSlots = 2;
+
+// Host-side wait for a stream, polled against a deadline (KM_HOST_TIMEOUT_S,
+// default 3600 s) so that a caller never blocks forever.
+km_status wait_stream(cudaStream_t st, const char* what) {
+    double limit_s = 3600.0;
+    if (const char* e = std::getenv("KM_HOST_TIMEOUT_S")) limit_s = std::atof(e) > 0 ? std::atof(e) : limit_s;
+    const auto t0 = std::chrono::steady_clock::now();
+    while (true) {
+        cudaError_t e = cudaStreamQuery(st);
+        if (e == cudaSuccess) return KM_OK;
+        if (e != cudaErrorNotReady) return cuda_error(e, what);
+        if (std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count() > limit_s) {
+            set_error("%s: still running after %.0f s", what, limit_s);
+            return KM_E_TIMEOUT;
+        }
+        std::this_thread::sleep_for(std::chrono::microseconds(200));
+    }
+}
+
+// Makes `st` wait for everything enqueued on `side` (on every exit path), so
+// that stream-ordered frees on `st` never overtake a copy still in flight.
+struct JoinGuard {
+    cudaStream_t st, side;
+    ~JoinGuard() {
+        cudaEvent_t ev = nullptr;
+        if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess) {
+            cudaEventRecord(ev, side);
+            cudaStreamWaitEvent(st, ev, 0);
+            cudaEventDestroy(ev);
+        } else {
+            cudaGetLastError();
+            cudaStreamSynchronize(side);
+        }
+    }
+};
+
+// RAII holder for the pipeline's side stream and events.
+struct PipelineRes {
+    cudaStream_t copy = nullptr;
+    cudaEvent_t ready[kSlots] = {nullptr, nullptr}, freed[kSlots] = {nullptr, nullptr};
+    ~PipelineRes() {
+        for (int i = 0; i < kSlots; ++i) {
+            if (ready[i]) cudaEventDestroy(ready[i]);
+            if (freed[i]) cudaEventDestroy(freed[i]);
+        }
+        if (copy) cudaStreamDestroy(copy);
+    }
+};
+
+// km_lloyd with X in pinned host memory: every iteration streams X through
+// kSlots device slots of R rows (papernotes.org "Flash-KMeans" page, 关键设计 3:
+// chunked, multi-stream H2D overlapped with the assignment and update).  A
+// side stream copies chunk r+1 while the caller's stream assigns, sorts and
+// accumulates chunk r; slots are recycled through events.  Sums and counts
+// accumulate over the chunks of an iteration; the centroids are finalised
+// once per iteration.  The call waits for the work (bounded) before returning.
+km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, int dtype, int iters,
+                     int32_t* labels, bool labels_on_host, float* C_out, float* objective, const DeviceInfo& dev,
+                     cudaStream_t st) {
+    const int64_t s = dtype == KM_F16 ? 2 : 4;
+    int64_t R = g_chunk_rows.load();
+    if (R <= 0) R = kDefaultChunkRows;
+    if (R > N) R = N;
+    const bool tc = uses_tc(dtype, d);
+    const int64_t Kp = padded_k(K);
+    PipelineRes res;
+    cudaError_t e = cudaStreamCreateWithFlags(&res.copy, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_error(e, "cudaStreamCreateWithFlags");
+    for (int i = 0; i < kSlots; ++i) {
+        if ((e = cudaEventCreateWithFlags(&res.ready[i], cudaEventDisableTiming)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&res.freed[i], cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_error(e, "cudaEventCreate");
+    }
+    km_status status = KM_OK;
+    {
+        Scratch scratch(st);
+        JoinGuard join{st, res.copy};  // destroyed before `scratch`: frees wait for the copies
+        unsigned char* slot[kSlots] = {nullptr, nullptr};
+        __half *chat = nullptr, *cext = nullptr;
+        float* sums = nullptr;
+        double* obj_acc = nullptr;
+        int32_t *lab = nullptr, *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr, *counts = nullptr;
+        unsigned char* work = nullptr;
+        for (int i = 0; i < kSlots && status == KM_OK; ++i) status = scratch.get(&slot[i], (size_t)(R * d * s), "X slot");
+        if (status == KM_OK && tc) status = scratch.get(&chat, (size_t)(B * K * d), "rounded centroids");
+        if (status == KM_OK && tc) status = scratch.get(&cext, (size_t)(B * Kp * 16), "centroid norm slices");
+        if (status == KM_OK) status = scratch.get(&sums, (size_t)(B * K * d), "cluster sums");
+        if (status == KM_OK) status = scratch.get(&counts, (size_t)(B * K), "cluster counts");
+        if (status == KM_OK && objective) status = scratch.get(&obj_acc, (size_t)B, "objective accumulator");
+        if (status == KM_OK) status = scratch.get(&lab, (size_t)R, "chunk labels");
+        if (status == KM_OK) status = scratch.get(&a_sorted, (size_t)R, "sorted labels");
+        if (status == KM_OK) status = scratch.get(&sidx, (size_t)R, "sorted indices");
+        if (status == KM_OK) status = scratch.get(&offs, (size_t)(K + 1), "segment offsets");
+        if (status == KM_OK) status = scratch.get(&work, sort_scratch_bytes(1, R, K), "radix sort buffers");
+        if (status != KM_OK) return status;
+
+        if (tc) {
+            PhaseScope ph(st, KM_PHASE_PREP, 1);
+            KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, chat, cext, st), "centroid preparation"));
+        }
+        {
+            PhaseScope ph(st, KM_PHASE_OTHER, 0);
+            KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * (size_t)(B * K * d), st), "zero sums"));
+            if (obj_acc) KM_TRY(launched(cudaMemsetAsync(obj_acc, 0, sizeof(double) * B, st), "zero objective"));
+        }
+        const int sort_launches = sort_kernel_launches(R, K, false, false);
+        int64_t g = 0;  // global chunk counter: slot = g % kSlots
+        for (int t = 0; t < iters; ++t) {
+            KM_TRY(launched(cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)(B * K), st), "zero counts"));
+            for (int64_t b = 0; b < B; ++b) {
+                for (int64_t r0 = 0; r0 < N; r0 += R, ++g) {
+                    const int64_t rows = (N - r0) < R ? (N - r0) : R;
+                    const int si = (int)(g % kSlots);
+                    // copy stream: reuse the slot only once the compute stream released it
+                    if (g >= kSlots) KM_TRY(launched(cudaStreamWaitEvent(res.copy, res.freed[si], 0), "wait slot"));
+                    KM_TRY(launched(cudaMemcpyAsync(slot[si], static_cast<const unsigned char*>(X) + (b * N + r0) * d * s,
+                                                    (size_t)(rows * d * s), cudaMemcpyHostToDevice, res.copy),
+                                    "copy X chunk"));
+                    KM_TRY(launched(cudaEventRecord(res.ready[si], res.copy), "record chunk ready"));
+                    // compute stream
+                    KM_TRY(launched(cudaStreamWaitEvent(st, res.ready[si], 0), "wait chunk"));
+                    KM_TRY(run_assign(slot[si], dtype, C_out + b * K * d, tc ? chat + b * K * d : nullptr,
+                                      tc ? cext + b * Kp * 16 : nullptr, 1, rows, K, d, lab, nullptr,
+                                      obj_acc ? obj_acc + b : nullptr, dev, st));
+                    {
+                        PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
+                        KM_TRY(launched(launch_sort(lab, 1, rows, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
+                                        "label sort"));
+                    }
+                    {
+                        PhaseScope ph(st, KM_PHASE_UPDATE, 2);
+                        KM_TRY(launched(launch_update_sums(slot[si], dtype, a_sorted, sidx, 1, rows, K, d,
+                                                           sums + b * K * d, offs, st, true),
+                                        "segmented update"));
+                        KM_TRY(launched(launch_add_counts(offs, 1, K, counts + b * K, st), "chunk counts"));
+                    }
+                    if (t == iters - 1) {
+                        PhaseScope ph(st, KM_PHASE_OTHER, 0);
+                        KM_TRY(launched(cudaMemcpyAsync(labels + b * N + r0, lab, sizeof(int32_t) * (size_t)rows,
+                                                        labels_on_host ? cudaMemcpyDeviceToHost
+                                                                       : cudaMemcpyDeviceToDevice,
+                                                        st),
+                                        "copy labels"));
+                    }
+                    KM_TRY(launched(cudaEventRecord(res.freed[si], st), "record slot free"));
+                }
+            }
+            const bool prep_next = tc && t + 1 < iters;
+            PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
+            KM_TRY(launched(launch_finalize(sums, nullptr, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
+                                            prep_next ? cext : nullptr, nullptr, true, obj_acc,
+                                            objective ? objective + (size_t)t * B : nullptr, st, counts),
+                            "centroid finalize"));
+        }
+    }  // scratch released on the stream
+    return wait_stream(st, "km_lloyd (host-resident X)");
+}
 
 }  // namespace
 
@@ -340,9 +503,20 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     cudaPointerAttributes pa;
     cudaError_t e = cudaPointerGetAttributes(&pa, X);
     if (e != cudaSuccess) return cuda_error(e, "cudaPointerGetAttributes(X)");
-    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged) {
-        set_error("km_lloyd: X must be device memory (host-resident X is not available in this build)");
+    const bool host_x = pa.type == cudaMemoryTypeHost;
+    if (!host_x && pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged) {
+        set_error("km_lloyd: X must be device memory or pinned host memory (cudaHostAlloc / cudaHostRegister)");
         return KM_E_UNSUPPORTED;
+    }
+    bool labels_on_host = false;
+    if (host_x) {
+        cudaPointerAttributes pl;
+        if ((e = cudaPointerGetAttributes(&pl, labels)) != cudaSuccess) return cuda_error(e, "cudaPointerGetAttributes");
+        labels_on_host = pl.type == cudaMemoryTypeHost;
+        if (!labels_on_host && pl.type != cudaMemoryTypeDevice && pl.type != cudaMemoryTypeManaged) {
+            set_error("km_lloyd: with host-resident X, labels must be pinned host or device memory");
+            return KM_E_UNSUPPORTED;
+        }
     }
     cudaStream_t st = (cudaStream_t)stream;
     const size_t ckd = (size_t)(B * K * d);
@@ -350,6 +524,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         KM_TRY(launched(cudaMemcpyAsync(C_out, C_init, sizeof(float) * ckd, cudaMemcpyDeviceToDevice, st),
                         "copy C_init"));
     if (iters == 0) return KM_OK;
+    if (host_x) return lloyd_host(X, B, N, K, d, dtype, iters, labels, labels_on_host, C_out, objective, dev, st);
 
     Scratch scratch(st);
     const bool tc = uses_tc(dtype, d);
@@ -402,7 +577,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     return KM_OK;
 }
 
-void km_set_chunk_rows(int64_t rows) { (void)rows; }
+void km_set_chunk_rows(int64_t rows) { g_chunk_rows.store(rows > 0 ? rows : 0); }
 
 void km_trace_enable(int on) { g_trace_on.store(on != 0); }
 

@@ -68,7 +68,8 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
 __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t B, int64_t K,
                                 int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype, __half* __restrict__ chat,
                                 __half* __restrict__ cext, int32_t* __restrict__ counts, int zero_sums,
-                                double* __restrict__ obj_acc, float* __restrict__ obj_out) {
+                                double* __restrict__ obj_acc, float* __restrict__ obj_out,
+                                const int32_t* __restrict__ counts_in) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (obj_out && row < B && lane == 0) {  // this iteration's objective, and a fresh accumulator
@@ -77,7 +78,7 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
     }
     if (row >= B * K) return;
     const int64_t b = row / K, k = row % K;
-    const int32_t n = offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
+    const int32_t n = counts_in ? counts_in[row] : offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
     if (counts && lane == 0) counts[row] = n;
     const float fn = (float)n;
     const int64_t base = row * d;
@@ -112,7 +113,20 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
     }
 }
 
+__global__ void add_counts_kernel(const int32_t* __restrict__ offsets, int64_t B, int64_t K,
+                                  int32_t* __restrict__ counts) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= B * K) return;
+    const int64_t b = t / K, k = t % K;
+    counts[t] += offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
+}
+
 }  // namespace
+
+cudaError_t launch_add_counts(const int32_t* offsets, int64_t B, int64_t K, int32_t* counts, cudaStream_t st) {
+    add_counts_kernel<<<(unsigned)ceil_div(B * K, 256), 256, 0, st>>>(offsets, B, K, counts);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
                                   __half* cext, cudaStream_t st) {
@@ -125,10 +139,12 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
 
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
                             int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, double* obj_acc,
-                            float* obj_out, cudaStream_t st) {
+                            float* obj_out, cudaStream_t st, const int32_t* counts_in) {
     const int warps = 8;
-    finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(
-        sums, offsets, B, K, padded_k(K), d, C_out, dtype, chat, cext, counts, zero_sums ? 1 : 0, obj_acc, obj_out);
+    finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(sums, offsets, B, K, padded_k(K), d,
+                                                                            C_out, dtype, chat, cext, counts,
+                                                                            zero_sums ? 1 : 0, obj_acc, obj_out,
+                                                                            counts_in);
     return cudaGetLastError();
 }
 

@@ -45,9 +45,10 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
 // or cext is non-null, also prepares the next assignment's centroids from
 // C_out; with zero_sums the sums are reset to 0 once consumed.
 // When obj_out is non-null, obj_out[b] = obj_acc[b] (as fp32) and obj_acc[b] = 0.
+// n_k is taken from counts_in when it is non-null, else from the offsets.
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
                             int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, double* obj_acc,
-                            float* obj_out, cudaStream_t st);
+                            float* obj_out, cudaStream_t st, const int32_t* counts_in = nullptr);
 
 // Tensor-core assignment (fp16, 64 <= d <= 128).  Returns cudaErrorNotSupported
 // for shapes it does not take.
@@ -72,9 +73,13 @@ cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, 
 
 // Segmented gather-reduce over the sorted order (sums must be zeroed first);
 // when offsets [B, K+1] is non-null it also writes the segment offsets.
+// With accumulate, the sums are added to (points streamed in chunks).
 cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
                                int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
-                               cudaStream_t st);
+                               cudaStream_t st, bool accumulate = false);
+
+// counts[b][k] += offsets[b][k+1] - offsets[b][k] (chunked accumulation of cluster sizes).
+cudaError_t launch_add_counts(const int32_t* offsets, int64_t B, int64_t K, int32_t* counts, cudaStream_t st);
 
 
 }  // namespace km

@@ -21,6 +21,9 @@
 //   in position order joins equal labels across row-lanes and decides, from
 //   the labels just outside the CTA's run, whether each joined interval is the
 //   whole cluster (plain store) or a part of it (fp32 vector atomic add).
+// In accumulate mode (points streamed in chunks, sums carried across
+// launches) the plain stores become read-add-writes: within one launch each
+// such cluster still has exactly one writer.
 #include "km_internal.cuh"
 
 namespace km {
@@ -59,7 +62,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, const int32_t* __restrict__ a_sorted,
                                                      const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
                                                      int64_t d, int tpr, int G, float* __restrict__ sums,
-                                                     int32_t* __restrict__ offsets) {
+                                                     int32_t* __restrict__ offsets, int accumulate) {
     constexpr int E = Chunk<T>::kElems;
     extern __shared__ __align__(16) unsigned char smem[];
     const int BN = G * kRowsPerLane;
@@ -124,9 +127,15 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
                         for (int e = 0; e < E; ++e) head_vec[(size_t)g * d + c * E + e] = acc[e];
                     } else if (cur >= 0 && cur < K) {  // a whole cluster inside this walk
 #pragma unroll
-                        for (int e = 0; e < E; e += 4)
-                            *reinterpret_cast<float4*>(sums_b + (int64_t)cur * d + e) =
-                                make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                        for (int e = 0; e < E; e += 4) {
+                            float4* dst = reinterpret_cast<float4*>(sums_b + (int64_t)cur * d + e);
+                            float4 o = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+                            if (accumulate) {  // this CTA is the only writer of the cluster in this launch
+                                const float4 prev = *dst;
+                                o.x += prev.x; o.y += prev.y; o.z += prev.z; o.w += prev.w;
+                            }
+                            *dst = o;
+                        }
                     }
                     ++piece;
 #pragma unroll
@@ -167,6 +176,9 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         float* dst = sums + (b * K + lab) * d + j4;
         if (shared_left || shared_right) {
             atomicAdd(reinterpret_cast<float4*>(dst), v);
+        } else if (accumulate) {
+            const float4 prev = *reinterpret_cast<const float4*>(dst);
+            *reinterpret_cast<float4*>(dst) = make_float4(prev.x + v.x, prev.y + v.y, prev.z + v.z, prev.w + v.w);
         } else {
             *reinterpret_cast<float4*>(dst) = v;
         }
@@ -193,7 +205,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
 
 template <typename T>
 cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sorted_idx, int64_t B, int64_t N,
-                     int64_t K, int64_t d, float* sums, int32_t* offsets, cudaStream_t st) {
+                     int64_t K, int64_t d, float* sums, int32_t* offsets, bool accumulate, cudaStream_t st) {
     const int tpr = (int)(d * (int64_t)sizeof(T) / 16);
     const int G = 256 / tpr;
     const int BN = G * kRowsPerLane;
@@ -204,7 +216,7 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
     }
     const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B);
     update_kernel<T><<<grid, G * tpr, smem, st>>>((const T*)X, a_sorted, sorted_idx, N, K, d, tpr, G, sums,
-                                                  offsets);
+                                                  offsets, accumulate ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -212,9 +224,9 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
 
 cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
                                int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
-                               cudaStream_t st) {
-    if (dtype == KM_F16) return launch_t<__half>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, st);
-    return launch_t<float>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, st);
+                               cudaStream_t st, bool accumulate) {
+    if (dtype == KM_F16) return launch_t<__half>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, accumulate, st);
+    return launch_t<float>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, accumulate, st);
 }
 
 }  // namespace km
