@@ -72,3 +72,43 @@ def test_workload3_zipf_hot_clusters():
 def test_workload4_large_k():
     w = synth.WORKLOADS[4]
     lockstep(w, 2, nsample=384)
+
+
+def test_workload5_host_resident_fp32_chunked():
+    """2^27 x 128 fp32 points (64 GiB) in pinned host memory, streamed in 2^23-row chunks."""
+    import time
+    import oracle
+    w = synth.WORKLOADS[5]
+    Xh = torch.empty((w.B, w.N, w.d), dtype=torch.float32).pin_memory()
+    X = Xh.numpy()
+    synth.points(w, out=X)
+    C = synth.init_centroids(w, X)
+    lab_h = torch.empty((w.B, w.N), dtype=torch.int32).pin_memory()
+    km.lib().km_set_chunk_rows(w.chunk_rows)
+    try:
+        for t in range(2):
+            t0 = time.perf_counter()
+            lab_h, C_next, obj = km.lloyd(Xh, torch.from_numpy(C).cuda(), 1, labels=lab_h)
+            torch.cuda.synchronize()
+            print(f"workload 5 iteration {t}: {time.perf_counter() - t0:.2f} s")
+            lab = lab_h.numpy()
+            C_next = C_next.cpu().numpy()
+            check_labels(X, C, lab, rows=sample_rows(w.B, w.N, 8192, seed=50 + t))
+            # argsort and counts over every point
+            sidx, counts, offs = km.sort_labels(torch.from_numpy(lab).cuda(), w.K)
+            check_sort(lab, w.K, sidx.cpu().numpy(), counts.cpu().numpy(), offs.cpu().numpy())
+            # update: the oracle's means of a sample of clusters, from their member rows
+            rng = np.random.default_rng(60 + t)
+            ks = np.sort(rng.choice(w.K, 48, replace=False))
+            members = np.isin(lab[0], ks)
+            Xs = np.ascontiguousarray(X[0][members])[None]
+            remap = np.full(w.K, -1, dtype=np.int32)
+            remap[ks] = np.arange(len(ks), dtype=np.int32)
+            C_sub, _, _ = oracle.update(Xs, remap[lab[0][members]][None], C[:, ks])
+            err = np.abs(C_next[0, ks].astype(np.float64) - C_sub[0]).max(axis=1)
+            lim = 1e-4 * np.maximum(np.abs(C_sub[0]).max(axis=1), 1e-6)
+            assert (err <= lim).all(), (err / lim).max()
+            C = C_next
+    finally:
+        km.lib().km_set_chunk_rows(0)
+    assert km.device_fault() == 0
