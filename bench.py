@@ -34,18 +34,23 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captures summarised in profiles/assign_tc_kernel_b32_n65536_k1024_d128_f16.md and
 # profiles/update_kernel_b32_n65536_k1024_d128_f16.md, each valid only for the kernel source it was
 # taken on (sha1 of the .cu file); reported as null once that source changes.
-ASSIGN_TRAFFIC = {"sha1": "f678660a53efdcf194671074c5f5b680e53f02ed", "bytes": 546.345984e6 + 20.080384e6}
-UPDATE_TRAFFIC = {"sha1": "9f133d72b690f094d1ceba919954c8667c0bcb82", "bytes": 557.686784e6 + 17.115648e6}
+ASSIGN_TRAFFIC = {"sha1": ["0a203d68193b824e70e267411cda0959ae9919af", "f0924f98116dbe93ff46af367ce72068d83b6d27"],
+                  "bytes": 546.434816e6 + 12.584192e6}
+UPDATE_TRAFFIC = {"sha1": ["c9054cceeb01068c671f1d62d9236f6ddc985079", "f0924f98116dbe93ff46af367ce72068d83b6d27"],
+                  "bytes": 557.689088e6 + 16.940288e6}
 
 
 def traffic_for(src: str, rec: dict):
+    """The recorded traffic while the kernel's source and the shared internal header are unchanged."""
     import hashlib
-    path = os.path.join(ROOT, "flashassign_b200", "csrc", src)
-    try:
-        h = hashlib.sha1(open(path, "rb").read()).hexdigest()
-    except OSError:
-        return None
-    return rec["bytes"] if rec["sha1"] == h else None
+    hashes = []
+    for name in (src, "km_internal.cuh"):
+        try:
+            with open(os.path.join(ROOT, "flashassign_b200", "csrc", name), "rb") as f:
+                hashes.append(hashlib.sha1(f.read()).hexdigest())
+        except OSError:
+            return None
+    return rec["bytes"] if hashes == rec["sha1"] else None
 
 
 def parse():
@@ -143,6 +148,32 @@ def cpu_oracle_ms_per_iter(w, X, C, rows: int):
     return dt * scale * 1e3, dt, oracle.threads()
 
 
+def cpu_oracle_baseline(w, X, C, target_s: float = 12.0):
+    """The oracle's assign + update on a bounded sample of about `target_s` seconds: whole batches when
+    one batch fits in the budget (the whole workload when all do), else leading rows of batch 0.
+    Returns (ms per full iteration, seconds measured, threads, description of the sample)."""
+    import numpy as np
+    import oracle
+    probe = min(2048, w.N)
+    _, dt_probe, _ = cpu_oracle_ms_per_iter(w, X, C, probe)
+    fit = target_s * probe / max(dt_probe, 1e-9)
+    if fit >= w.N:
+        nb = int(min(w.B, fit // w.N))
+        sample_X, sample_C, rows = X[:nb], C[:nb], nb * w.N
+        what = (f"the whole iteration ({nb} of {w.B} problems)" if nb == w.B else
+                f"{nb} of the {w.B} problems, extrapolated x{w.B / nb:g}")
+    else:
+        rows = max(probe, int(fit))
+        sample_X, sample_C = np.ascontiguousarray(X[:1, :rows]), C[:1]
+        what = f"{rows} of the {w.B * w.N} points (batch 0), extrapolated x{w.B * w.N / rows:.1f}"
+    t0 = time.perf_counter()
+    lab, _, _ = oracle.assign(sample_X, sample_C)
+    oracle.update(sample_X, lab, sample_C)
+    dt = time.perf_counter() - t0
+    ms = dt * 1e3 * (w.B * w.N) / rows
+    return ms, dt, oracle.threads(), f"oracle assign+update (K={w.K}, d={w.d}) on {what}: {dt:.2f} s measured"
+
+
 def run_reference(args, w):
     """The oracle arm: plain C++ CPU Lloyd on bounded samples of the same workload."""
     import numpy as np
@@ -150,7 +181,7 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    rows = 4096
+    rows = min(16384, w.N)
     wx = w.with_(B=1)
     X = synth.points(wx, 0, rows)  # batch 0, first rows: same distribution as the full workload
     rng = np.random.default_rng(0)
@@ -223,9 +254,8 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     assert km.device_fault() == 0
 
-    # timed: K iterations, one call, device-resident inputs (X = 512 MiB > L2)
-    km.trace_read()
-    km.trace_enable(True)
+    # timed: K iterations, one call, device-resident inputs (X = 512 MiB > L2); kernels
+    # chained with programmatic dependent launch
     barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -234,29 +264,42 @@ def run_ours(args, w):
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    km.trace_enable(False)
-    phases = km.trace_read()
     total_ms = allmax(ev0.elapsed_time(ev1))
     ms_iter = total_ms / args.steps
+
+    # the same K iterations again with the library's per-phase CUDA events on the launching
+    # stream (this turns the launch overlap off, so each kernel is timed alone)
+    km.trace_read()
+    km.trace_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    ev2, ev3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev2.record(stream)
+    km.lloyd(X, C, args.steps, labels=labels, C_out=C_out)
+    ev3.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    km.trace_enable(False)
+    phases = km.trace_read()
+    traced_ms_iter = allmax(ev2.elapsed_time(ev3)) / args.steps
     C.copy_(C_out)
     fault = km.device_fault()
 
-    # end to end: host buffers, copies inside the timed region
+    # end to end: host buffers, copies inside the timed region.  X stays in pinned host memory
+    # and km_lloyd streams it through the GPU in chunks, its copies overlapped with the
+    # kernels; the labels come back into pinned host memory inside the call.
     e2e = None
     if not args.no_e2e:
         Xp = torch.from_numpy(X_host).pin_memory()
         Cp = torch.from_numpy(C_init).pin_memory()
         lab_h = torch.empty((w.B, w.N), dtype=torch.int32).pin_memory()
         C_h = torch.empty_like(Cp).pin_memory()
-        Xd = torch.empty_like(X)
         Cd = torch.empty_like(C)
         steps_e = max(1, args.e2e_steps)
 
         def e2e_step():
-            Xd.copy_(Xp, non_blocking=True)
             Cd.copy_(Cp, non_blocking=True)
-            km.lloyd(Xd, Cd, 1, labels=labels, C_out=C_out)
-            lab_h.copy_(labels, non_blocking=True)
+            km.lloyd(Xp, Cd, 1, labels=lab_h, C_out=C_out)
             C_h.copy_(C_out, non_blocking=True)
 
         e2e_step()
@@ -273,7 +316,8 @@ def run_ours(args, w):
         e2e = {"value": round(e_ms, 4), "unit": UNIT, "steps": steps_e,
                "h2d_bytes_per_step": int(Xp.numel() * Xp.element_size() + Cp.numel() * 4),
                "d2h_bytes_per_step": int(lab_h.numel() * 4 + C_h.numel() * 4),
-               "path": "pinned host X and C copied in, km_lloyd(iters=1), labels and C copied out"}
+               "path": "km_lloyd(iters=1) on X in pinned host memory (chunked copies overlapped with the "
+                       "kernels, labels written back to pinned host memory); C copied in and out"}
     clocks = sampler.stop()
 
     if rank != 0:
@@ -298,11 +342,8 @@ def run_ours(args, w):
 
     cpu = None
     if not args.no_cpu and world == 1:
-        rows = 65536
-        ms_cpu, dt, cores = cpu_oracle_ms_per_iter(w, X_host, C_init, rows)
-        cpu = {"value": round(ms_cpu, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"oracle assign+update of batch 0 ({rows} points, K={w.K}, d={w.d}) took {dt:.2f} s; "
-                         f"extrapolated x{w.B} to the full {w.B}-problem iteration"}
+        ms_cpu, dt, cores, what = cpu_oracle_baseline(w, X_host, C_init)
+        cpu = {"value": round(ms_cpu, 1), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": what}
 
     out = {
         "metric": METRIC, "value": round(ms_iter, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -321,6 +362,7 @@ def run_ours(args, w):
                             "ms_per_launch": round(t_update, 4), "peak_source": peak_src},
         "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4)},
         "phases_ms_per_iter": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
+        "traced_ms_per_iter": round(traced_ms_iter, 4),
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,

@@ -340,6 +340,8 @@ km_status cuda_error(cudaError_t e, const char* what) {
     return e == cudaErrorMemoryAllocation ? KM_E_NOMEM : KM_E_CUDA;
 }
 
+bool pdl_enabled() { return !g_trace_on.load(std::memory_order_relaxed); }
+
 int32_t* fault_word() {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fault) != cudaSuccess) return nullptr;

@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restri
                                                                int32_t* __restrict__ labels,
                                                                float* __restrict__ mindist,
                                                                double* __restrict__ obj_acc) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ float xs[kThreads][kTileD + 1];
     __shared__ float cs[kTileK][kTileD + 1];
     const int64_t b = blockIdx.y;
@@ -97,10 +99,10 @@ cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t
                                int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st) {
     dim3 grid((unsigned)ceil_div(N, kThreads), (unsigned)B);
     if (dtype == KM_F16)
-        assign_simt_kernel<__half><<<grid, kThreads, 0, st>>>((const __half*)X, C, N, K, d, labels, mindist, obj_acc);
-    else
-        assign_simt_kernel<float><<<grid, kThreads, 0, st>>>((const float*)X, C, N, K, d, labels, mindist, obj_acc);
-    return cudaGetLastError();
+        return launch_kernel(assign_simt_kernel<__half>, grid, kThreads, 0, st, (const __half*)X, C, N, K, d, labels,
+                             mindist, obj_acc);
+    return launch_kernel(assign_simt_kernel<float>, grid, kThreads, 0, st, (const float*)X, C, N, K, d, labels, mindist,
+                         obj_acc);
 }
 
 }  // namespace km

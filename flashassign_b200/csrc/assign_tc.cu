@@ -291,6 +291,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // everything above overlaps the previous kernel's tail; the centroid tiles
+    // and the objective accumulator are written by it
+    pdl_trigger();
+    pdl_wait();
 
     const int boxes = P.boxes;
     const uint32_t x_bytes_pair = (uint32_t)(2 * boxes * kBoxBytes);
@@ -593,8 +597,7 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* 
         if (dev >= 0 && dev < 64) pair_cache[dev] = max_pairs;
     }
     P.pairs = P.units < max_pairs ? P.units : max_pairs;
-    assign_tc_kernel<<<(unsigned)(2 * P.pairs), kThreads, kSmemBytes, st>>>(mx, mc, me, P);
-    return cudaGetLastError();
+    return launch_kernel(assign_tc_kernel, dim3((unsigned)(2 * P.pairs)), dim3(kThreads), kSmemBytes, st, mx, mc, me, P);
 }
 
 }  // namespace km

@@ -39,6 +39,8 @@ __device__ __forceinline__ void write_norm_slice(__half* out, double v) {
 
 __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, int64_t Kp, int64_t d, int dtype,
                             __half* __restrict__ chat, __half* __restrict__ cext) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (row >= B * Kp) return;
@@ -70,6 +72,8 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
                                 __half* __restrict__ cext, int32_t* __restrict__ counts, int zero_sums,
                                 double* __restrict__ obj_acc, float* __restrict__ obj_out,
                                 const int32_t* __restrict__ counts_in) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
     if (obj_out && row < B && lane == 0) {  // this iteration's objective, and a fresh accumulator
@@ -115,6 +119,8 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
 
 __global__ void add_counts_kernel(const int32_t* __restrict__ offsets, int64_t B, int64_t K,
                                   int32_t* __restrict__ counts) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= B * K) return;
     const int64_t b = t / K, k = t % K;
@@ -124,8 +130,8 @@ __global__ void add_counts_kernel(const int32_t* __restrict__ offsets, int64_t B
 }  // namespace
 
 cudaError_t launch_add_counts(const int32_t* offsets, int64_t B, int64_t K, int32_t* counts, cudaStream_t st) {
-    add_counts_kernel<<<(unsigned)ceil_div(B * K, 256), 256, 0, st>>>(offsets, B, K, counts);
-    return cudaGetLastError();
+    return launch_kernel(add_counts_kernel, dim3((unsigned)ceil_div(B * K, 256)), dim3(256), 0, st, offsets, B, K,
+                         counts);
 }
 
 cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
@@ -133,18 +139,17 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
     const int64_t Kp = padded_k(K);
     const int64_t rows = B * Kp;
     const int warps = 8;
-    prep_kernel<<<(unsigned)ceil_div(rows, warps), warps * 32, 0, st>>>(C, B, K, Kp, d, dtype, chat, cext);
-    return cudaGetLastError();
+    return launch_kernel(prep_kernel, dim3((unsigned)ceil_div(rows, warps)), dim3(warps * 32), 0, st, C, B, K, Kp, d,
+                         dtype, chat, cext);
 }
 
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
                             int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, double* obj_acc,
                             float* obj_out, cudaStream_t st, const int32_t* counts_in) {
     const int warps = 8;
-    finalize_kernel<<<(unsigned)ceil_div(B * K, warps), warps * 32, 0, st>>>(sums, offsets, B, K, padded_k(K), d,
-                                                                            C_out, dtype, chat, cext, counts,
-                                                                            zero_sums ? 1 : 0, obj_acc, obj_out,
-                                                                            counts_in);
+    return launch_kernel(finalize_kernel, dim3((unsigned)ceil_div(B * K, warps)), dim3(warps * 32), 0, st, sums,
+                         offsets, B, K, padded_k(K), d, C_out, dtype, chat, cext, counts, zero_sums ? 1 : 0, obj_acc,
+                         obj_out, counts_in);
     return cudaGetLastError();
 }
 

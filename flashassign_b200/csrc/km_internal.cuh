@@ -26,6 +26,38 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 constexpr int kAssignTileK = 256;
 inline int64_t padded_k(int64_t K) { return ceil_div(K, kAssignTileK) * kAssignTileK; }
 
+// ---- programmatic dependent launch ----
+// Kernels on the iteration's path are launched with programmatic stream
+// serialisation: a kernel may start (prologue, resource allocation) while
+// its predecessor in the stream is still draining, and waits for it with
+// pdl_wait() before reading anything the predecessor wrote.  Every kernel
+// calls pdl_wait() in every thread before its first dependent access and
+// before it exits, so a grid never completes ahead of its predecessor and
+// the chain stays ordered transitively.  Without the launch attribute both
+// instructions are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Whether launches carry the attribute: off while per-phase event tracing is
+// on, so that traced kernel times are not overlapped with their neighbours.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct DeviceInfo {
     int device = -1;
     int sms = 0;

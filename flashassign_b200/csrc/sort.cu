@@ -55,6 +55,8 @@ bool small_hist(int bins, int64_t tiles) { return (int64_t)bins * tiles <= 8192;
 
 __global__ void __launch_bounds__(kThreads) radix_hist_kernel(const int32_t* __restrict__ keys, int64_t N, int shift,
                                                               int bits, int64_t T, int32_t* __restrict__ hist) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int s[256];
     const int64_t b = blockIdx.y, tile = blockIdx.x;
     const int bins = 1 << bits, mask = bins - 1;
@@ -72,6 +74,8 @@ __global__ void __launch_bounds__(kThreads) radix_hist_kernel(const int32_t* __r
 
 // In-place exclusive scan of `len` ints per batch (one 1024-thread block per batch).
 __global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t* __restrict__ data, int64_t len) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int warp_tot[32];
     __shared__ int carry_s;
     int32_t* p = data + (int64_t)blockIdx.x * len;
@@ -115,6 +119,8 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
                                                                  int bits, int64_t T,
                                                                  const int32_t* __restrict__ offs,
                                                                  const int32_t* __restrict__ hist) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ int wh[kWarps][256];      // per-warp digit counts, then per-warp exclusive offsets
     __shared__ int gstart[256];          // global first position of each digit of this tile (hist path)
     __shared__ int tstart[256];          // first tile-local position of each digit
@@ -225,6 +231,8 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
 
 // offsets[b][k] = first sorted position holding a label >= k (offsets[b][K] = N).
 __global__ void seg_bounds_kernel(const int32_t* __restrict__ a, int64_t N, int64_t K, int32_t* __restrict__ offsets) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t b = blockIdx.y;
     const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (p > N) return;
@@ -235,6 +243,8 @@ __global__ void seg_bounds_kernel(const int32_t* __restrict__ a, int64_t N, int6
 }
 
 __global__ void counts_kernel(const int32_t* __restrict__ offsets, int64_t B, int64_t K, int32_t* __restrict__ counts) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= B * K) return;
     const int64_t b = t / K, k = t % K;
@@ -277,23 +287,31 @@ cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, 
         int32_t* out_k = to_final ? a_sorted : tmp_k;
         int32_t* out_v = to_final ? sorted_idx : tmp_v;
         const int bins = 1 << p.bits[i];
-        radix_hist_kernel<<<grid, kThreads, 0, st>>>(in_k, N, p.shift[i], p.bits[i], p.tiles, hist);
+        cudaError_t e = launch_kernel(radix_hist_kernel, grid, dim3(kThreads), 0, st, in_k, N, p.shift[i], p.bits[i],
+                                      p.tiles, hist);
+        if (e != cudaSuccess) return e;
         if (small_hist(bins, p.tiles)) {
-            radix_scatter_kernel<<<grid, kThreads, 0, st>>>(in_k, in_v, out_k, out_v, N, p.shift[i], p.bits[i],
-                                                            p.tiles, nullptr, hist);
+            e = launch_kernel(radix_scatter_kernel, grid, dim3(kThreads), 0, st, in_k, in_v, out_k, out_v, N,
+                              p.shift[i], p.bits[i], p.tiles, (const int32_t*)nullptr, (const int32_t*)hist);
         } else {
-            exclusive_scan_kernel<<<(unsigned)B, 1024, 0, st>>>(hist, (int64_t)bins * p.tiles);
-            radix_scatter_kernel<<<grid, kThreads, 0, st>>>(in_k, in_v, out_k, out_v, N, p.shift[i], p.bits[i],
-                                                            p.tiles, hist, nullptr);
+            e = launch_kernel(exclusive_scan_kernel, dim3((unsigned)B), dim3(1024), 0, st, hist,
+                              (int64_t)bins * p.tiles);
+            if (e != cudaSuccess) return e;
+            e = launch_kernel(radix_scatter_kernel, grid, dim3(kThreads), 0, st, in_k, in_v, out_k, out_v, N,
+                              p.shift[i], p.bits[i], p.tiles, (const int32_t*)hist, (const int32_t*)nullptr);
         }
+        if (e != cudaSuccess) return e;
         in_k = out_k;
         in_v = out_v;
     }
     if (bounds) {
-        seg_bounds_kernel<<<dim3((unsigned)ceil_div(N + 1, 256), (unsigned)B), 256, 0, st>>>(a_sorted, N, K, offsets);
-        if (counts) counts_kernel<<<(unsigned)ceil_div(B * K, 256), 256, 0, st>>>(offsets, B, K, counts);
+        cudaError_t e = launch_kernel(seg_bounds_kernel, dim3((unsigned)ceil_div(N + 1, 256), (unsigned)B), dim3(256),
+                                      0, st, (const int32_t*)a_sorted, N, K, offsets);
+        if (e != cudaSuccess || !counts) return e;
+        return launch_kernel(counts_kernel, dim3((unsigned)ceil_div(B * K, 256)), dim3(256), 0, st,
+                             (const int32_t*)offsets, B, K, counts);
     }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 }  // namespace km

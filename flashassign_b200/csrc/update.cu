@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
                                                      const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
                                                      int64_t d, int tpr, int G, float* __restrict__ sums,
                                                      int32_t* __restrict__ offsets, int accumulate) {
+    pdl_trigger();
+    pdl_wait();
     constexpr int E = Chunk<T>::kElems;
     extern __shared__ __align__(16) unsigned char smem[];
     const int BN = G * kRowsPerLane;
@@ -215,9 +217,8 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
         if (e != cudaSuccess) return e;
     }
     const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B);
-    update_kernel<T><<<grid, G * tpr, smem, st>>>((const T*)X, a_sorted, sorted_idx, N, K, d, tpr, G, sums,
-                                                  offsets, accumulate ? 1 : 0);
-    return cudaGetLastError();
+    return launch_kernel(update_kernel<T>, grid, dim3(G * tpr), smem, st, (const T*)X, a_sorted, sorted_idx, N, K, d,
+                         tpr, G, sums, offsets, accumulate ? 1 : 0);
 }
 
 }  // namespace
