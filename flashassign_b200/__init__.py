@@ -27,6 +27,7 @@ SIGNATURES = {
     "km_status_string": (ctypes.c_char_p, [_INT]),
     "km_last_error": (ctypes.c_char_p, []),
     "km_device_fault": (_INT, [ctypes.POINTER(ctypes.c_int32), _P]),
+    "km_assign_rescans": (_INT, [ctypes.POINTER(ctypes.c_int64), _P]),
     "km_assign_noalloc": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
     "km_assign_noalloc_limit": (ctypes.c_size_t, []),
     "km_trace_enable": (None, [_INT]),
@@ -167,6 +168,13 @@ def device_fault(stream=None) -> int:
     code = ctypes.c_int32(0)
     check("km_device_fault", lib().km_device_fault(ctypes.byref(code), _stream(stream)))
     return int(code.value)
+
+
+def assign_rescans(stream=None) -> int:
+    """Read and clear the count of fp32 points handed to the exact re-scan (see include/km.h)."""
+    n = ctypes.c_int64(0)
+    check("km_assign_rescans", lib().km_assign_rescans(ctypes.byref(n), _stream(stream)))
+    return int(n.value)
 
 
 def trace_enable(on: bool = True) -> None:

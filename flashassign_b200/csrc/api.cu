@@ -4,6 +4,7 @@
 // (papernotes.org "Flash-KMeans" page, 方法详解: 整体框架 and 关键设计 1-3).
 #include "km_internal.cuh"
 
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <cstdarg>
@@ -19,6 +20,7 @@ namespace km {
 namespace {
 thread_local char g_err[512] = "";
 __device__ int32_t g_fault;  // device fault word (see km_device_fault)
+__device__ unsigned long long g_rescans;  // points handed to the exact re-scan (see km_assign_rescans)
 
 bool inject(const char* what) {
     const char* f = std::getenv("KM_FAULT");
@@ -150,20 +152,86 @@ km_status launched(cudaError_t e, const char* what) {
         if (_s != KM_OK) return _s;        \
     } while (0)
 
-// The assignment for one iteration, given prepared centroids.
-km_status run_assign(const void* X, int dtype, const float* C, const __half* chat, const __half* cext, int64_t B,
-                     int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
-                     const DeviceInfo& dev, cudaStream_t st) {
+bool uses_tc(int dtype, int64_t d) {
+    return dtype == KM_F16 ? assign_tc_supported(d, dtype) : assign_tf32_supported(d);
+}
+
+// Scratch of a tensor-core assignment: the prepared centroids and, for fp32,
+// the per-batch list of points left to the exact re-scan.
+struct TcScratch {
+    PreparedC prep;
+    int32_t* flag_count = nullptr;  // [B]
+    int32_t* flag_rows = nullptr;   // [B, list_rows / B]
+    // batch b alone (the chunk pipeline assigns one batch at a time; its list
+    // and counter serve every chunk in turn)
+    TcScratch batch(int64_t b, int64_t K, int64_t d, int dtype) const {
+        TcScratch t = *this;
+        const int64_t Kp = padded_k(K);
+        if (dtype == KM_F16) {
+            t.prep.chat = static_cast<__half*>(prep.chat) + b * K * d;
+            t.prep.cext = static_cast<__half*>(prep.cext) + b * Kp * 16;
+        } else {
+            t.prep.chat = static_cast<float*>(prep.chat) + b * K * 2 * d;
+            t.prep.cext = static_cast<float*>(prep.cext) + b * Kp * 8;
+            t.prep.cmax = prep.cmax + b;
+        }
+        return t;
+    }
+};
+
+// Takes the tensor-core scratch for B batches of K centroids from `s`, with
+// room for list_rows listed points (fp32), and zeroes the norm bound.
+km_status alloc_tc(Scratch& s, int dtype, int64_t B, int64_t K, int64_t d, int64_t list_rows, cudaStream_t st,
+                   TcScratch* out) {
+    const int64_t Kp = padded_k(K);
+    if (dtype == KM_F16) {
+        __half *chat = nullptr, *cext = nullptr;
+        KM_TRY(s.get(&chat, (size_t)(B * K * d), "rounded centroids"));
+        KM_TRY(s.get(&cext, (size_t)(B * Kp * 16), "centroid norm slices"));
+        out->prep.chat = chat;
+        out->prep.cext = cext;
+        return KM_OK;
+    }
+    float *chat = nullptr, *cext = nullptr;
+    KM_TRY(s.get(&chat, (size_t)(B * K * 2 * d), "centroid heads and tails"));
+    KM_TRY(s.get(&cext, (size_t)(B * Kp * 8), "centroid norm pieces"));
+    KM_TRY(s.get(&out->prep.cmax, (size_t)B, "centroid norm bound"));
+    KM_TRY(s.get(&out->flag_count, (size_t)B, "re-scan counters"));
+    KM_TRY(s.get(&out->flag_rows, (size_t)list_rows, "re-scan lists"));
+    out->prep.chat = chat;
+    out->prep.cext = cext;
+    return launched(cudaMemsetAsync(out->prep.cmax, 0, sizeof(float) * (size_t)B, st), "zero norm bound");
+}
+
+// The assignment for one iteration, given prepared centroids (tc == nullptr:
+// the CUDA-core kernel).  fp32 on tensor cores is two launches: the tf32
+// kernel, then the exact re-scan of the points it listed.
+km_status run_assign(const void* X, int dtype, const float* C, const TcScratch* tc, int64_t B, int64_t N, int64_t K,
+                     int64_t d, int32_t* labels, float* mindist, double* obj_acc, const DeviceInfo& dev,
+                     cudaStream_t st) {
+    if (tc && dtype == KM_F16) {
+        PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
+        return launched(launch_assign_tc((const __half*)X, static_cast<const __half*>(tc->prep.chat),
+                                         static_cast<const __half*>(tc->prep.cext), B, N, K, d, labels, mindist,
+                                         obj_acc, dev.sms, st),
+                        "assign (tensor cores)");
+    }
+    if (tc) {
+        PhaseScope ph(st, KM_PHASE_ASSIGN, 2);
+        KM_TRY(launched(cudaMemsetAsync(tc->flag_count, 0, sizeof(int32_t) * (size_t)B, st), "zero re-scan counters"));
+        KM_TRY(launched(launch_assign_tf32((const float*)X, static_cast<const float*>(tc->prep.chat),
+                                           static_cast<const float*>(tc->prep.cext), tc->prep.cmax, B, N, K, d,
+                                           labels, mindist, obj_acc, tc->flag_count, tc->flag_rows, dev.sms, st),
+                        "assign (tf32 tensor cores)"));
+        const int blocks = (int)std::max<int64_t>(1, 4 * (int64_t)dev.sms / B);
+        return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st, tc->flag_rows,
+                                           tc->flag_count, blocks),
+                        "assign (exact re-scan of listed points)");
+    }
     PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
-    if (dtype == KM_F16 && assign_tc_supported(d, dtype))
-        return launched(
-            launch_assign_tc((const __half*)X, chat, cext, B, N, K, d, labels, mindist, obj_acc, dev.sms, st),
-            "assign (tensor cores)");
     return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st),
                     "assign (CUDA cores)");
 }
-
-bool uses_tc(int dtype, int64_t d) { return dtype == KM_F16 && assign_tc_supported(d, dtype); }
 
 std::atomic<int64_t> g_chunk_rows{0};
 constexpr int64_t kDefaultChunkRows = int64_t(1) << 23;
@@ -246,14 +314,13 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
         Scratch scratch(st);
         JoinGuard join{st, res.copy};  // destroyed before `scratch`: frees wait for the copies
         unsigned char* slot[kSlots] = {nullptr, nullptr};
-        __half *chat = nullptr, *cext = nullptr;
+        TcScratch tcs;
         float* sums = nullptr;
         double* obj_acc = nullptr;
         int32_t *lab = nullptr, *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr, *counts = nullptr;
         unsigned char* work = nullptr;
         for (int i = 0; i < kSlots && status == KM_OK; ++i) status = scratch.get(&slot[i], (size_t)(R * d * s), "X slot");
-        if (status == KM_OK && tc) status = scratch.get(&chat, (size_t)(B * K * d), "rounded centroids");
-        if (status == KM_OK && tc) status = scratch.get(&cext, (size_t)(B * Kp * 16), "centroid norm slices");
+        if (status == KM_OK && tc) status = alloc_tc(scratch, dtype, B, K, d, R, st, &tcs);
         if (status == KM_OK) status = scratch.get(&sums, (size_t)(B * K * d), "cluster sums");
         if (status == KM_OK) status = scratch.get(&counts, (size_t)(B * K), "cluster counts");
         if (status == KM_OK && objective) status = scratch.get(&obj_acc, (size_t)B, "objective accumulator");
@@ -266,7 +333,7 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
 
         if (tc) {
             PhaseScope ph(st, KM_PHASE_PREP, 1);
-            KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, chat, cext, st), "centroid preparation"));
+            KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
         }
         {
             PhaseScope ph(st, KM_PHASE_OTHER, 0);
@@ -289,9 +356,9 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
                     KM_TRY(launched(cudaEventRecord(res.ready[si], res.copy), "record chunk ready"));
                     // compute stream
                     KM_TRY(launched(cudaStreamWaitEvent(st, res.ready[si], 0), "wait chunk"));
-                    KM_TRY(run_assign(slot[si], dtype, C_out + b * K * d, tc ? chat + b * K * d : nullptr,
-                                      tc ? cext + b * Kp * 16 : nullptr, 1, rows, K, d, lab, nullptr,
-                                      obj_acc ? obj_acc + b : nullptr, dev, st));
+                    const TcScratch tcb = tc ? tcs.batch(b, K, d, dtype) : TcScratch();
+                    KM_TRY(run_assign(slot[si], dtype, C_out + b * K * d, tc ? &tcb : nullptr, 1, rows, K, d, lab,
+                                      nullptr, obj_acc ? obj_acc + b : nullptr, dev, st));
                     {
                         PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
                         KM_TRY(launched(launch_sort(lab, 1, rows, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
@@ -317,8 +384,8 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
             }
             const bool prep_next = tc && t + 1 < iters;
             PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
-            KM_TRY(launched(launch_finalize(sums, nullptr, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
-                                            prep_next ? cext : nullptr, nullptr, true, obj_acc,
+            KM_TRY(launched(launch_finalize(sums, nullptr, B, K, d, C_out, dtype, prep_next ? tcs.prep : PreparedC(),
+                                            nullptr, true, obj_acc,
                                             objective ? objective + (size_t)t * B : nullptr, st, counts),
                             "centroid finalize"));
         }
@@ -346,6 +413,12 @@ int32_t* fault_word() {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fault) != cudaSuccess) return nullptr;
     return static_cast<int32_t*>(p);
+}
+
+unsigned long long* rescan_word() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_rescans) != cudaSuccess) return nullptr;
+    return static_cast<unsigned long long*>(p);
 }
 
 km_status device_info(DeviceInfo* out) {
@@ -407,14 +480,14 @@ km_status km_assign(const void* X, const float* C, int64_t B, int64_t N, int64_t
     KM_TRY(check_device(&dev));
     cudaStream_t st = (cudaStream_t)stream;
     Scratch scratch(st);
-    __half *chat = nullptr, *cext = nullptr;
-    if (uses_tc(dtype, d)) {
-        KM_TRY(scratch.get(&chat, (size_t)(B * K * d), "rounded centroids"));
-        KM_TRY(scratch.get(&cext, (size_t)(B * padded_k(K) * 16), "centroid norm slices"));
+    const bool tc = uses_tc(dtype, d);
+    TcScratch tcs;
+    if (tc) {
+        KM_TRY(alloc_tc(scratch, dtype, B, K, d, B * N, st, &tcs));
         PhaseScope ph(st, KM_PHASE_PREP, 1);
-        KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, chat, cext, st), "centroid preparation"));
+        KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
     }
-    return run_assign(X, dtype, C, chat, cext, B, N, K, d, labels, mindist, nullptr, dev, st);
+    return run_assign(X, dtype, C, tc ? &tcs : nullptr, B, N, K, d, labels, mindist, nullptr, dev, st);
 }
 
 km_status km_sort_labels(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* sorted_idx,
@@ -479,7 +552,7 @@ km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, 
     }
     PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
     return launched(
-        launch_finalize(sums, offs, B, K, d, C_out, dtype, nullptr, nullptr, counts, false, nullptr, nullptr, st),
+        launch_finalize(sums, offs, B, K, d, C_out, dtype, PreparedC(), counts, false, nullptr, nullptr, st),
         "centroid finalize");
 }
 
@@ -530,15 +603,12 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
 
     Scratch scratch(st);
     const bool tc = uses_tc(dtype, d);
-    __half *chat = nullptr, *cext = nullptr;
+    TcScratch tcs;
     float* sums = nullptr;
     double* obj_acc = nullptr;
     int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
     unsigned char* work = nullptr;
-    if (tc) {
-        KM_TRY(scratch.get(&chat, ckd, "rounded centroids"));
-        KM_TRY(scratch.get(&cext, (size_t)(B * padded_k(K) * 16), "centroid norm slices"));
-    }
+    if (tc) KM_TRY(alloc_tc(scratch, dtype, B, K, d, B * N, st, &tcs));
     if (objective) KM_TRY(scratch.get(&obj_acc, (size_t)B, "objective accumulator"));
     KM_TRY(scratch.get(&sums, ckd, "cluster sums"));
     KM_TRY(scratch.get(&offs, (size_t)(B * (K + 1)), "segment offsets"));
@@ -548,7 +618,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
 
     if (tc) {
         PhaseScope ph(st, KM_PHASE_PREP, 1);
-        KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, chat, cext, st), "centroid preparation"));
+        KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
     }
     {
         PhaseScope ph(st, KM_PHASE_OTHER, 0);
@@ -557,7 +627,7 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     }
     const int sort_launches = sort_kernel_launches(N, K, false, false);
     for (int t = 0; t < iters; ++t) {
-        KM_TRY(run_assign(X, dtype, C_out, chat, cext, B, N, K, d, labels, nullptr, obj_acc, dev, st));
+        KM_TRY(run_assign(X, dtype, C_out, tc ? &tcs : nullptr, B, N, K, d, labels, nullptr, obj_acc, dev, st));
         {
             PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
             KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
@@ -571,8 +641,8 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
         const bool prep_next = tc && t + 1 < iters;
         PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
         // the finalize zeroes the consumed sums, so the next update starts from 0
-        KM_TRY(launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, prep_next ? chat : nullptr,
-                                        prep_next ? cext : nullptr, nullptr, true, obj_acc,
+        KM_TRY(launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, prep_next ? tcs.prep : PreparedC(),
+                                        nullptr, true, obj_acc,
                                         objective ? objective + (size_t)t * B : nullptr, st),
                         "centroid finalize"));
     }
@@ -625,6 +695,22 @@ km_status km_device_fault(int32_t* code, void* stream) {
     if ((e = cudaMemcpyFromSymbol(&v, g_fault, sizeof(v))) != cudaSuccess) return cuda_error(e, "read fault word");
     if ((e = cudaMemcpyToSymbol(g_fault, &zero, sizeof(zero))) != cudaSuccess) return cuda_error(e, "clear fault word");
     *code = v;
+    return KM_OK;
+}
+
+km_status km_assign_rescans(int64_t* count, void* stream) {
+    g_err[0] = 0;
+    if (!count) {
+        set_error("km_assign_rescans: count must be non-null");
+        return KM_E_INVALID;
+    }
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_error(e, "cudaStreamSynchronize");
+    unsigned long long v = 0, zero = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_rescans, sizeof(v))) != cudaSuccess) return cuda_error(e, "read re-scan count");
+    if ((e = cudaMemcpyToSymbol(g_rescans, &zero, sizeof(zero))) != cudaSuccess)
+        return cuda_error(e, "clear re-scan count");
+    *count = (int64_t)v;
     return KM_OK;
 }
 

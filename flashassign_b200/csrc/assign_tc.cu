@@ -44,11 +44,10 @@
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records a fault code in the device fault word, stops issuing work, frees
 // its TMEM and returns.
-#include "km_internal.cuh"
-
-#include <cuda.h>
+#include "tc_ptx.cuh"
 
 namespace km {
+using namespace ptx;
 namespace {
 
 constexpr int kRows = 128;                      // point rows per CTA per unit (TMEM lanes)
@@ -61,9 +60,9 @@ constexpr int kCStages = 4;
 constexpr int kXBufs = 2;
 constexpr int kAccSets = 2;                     // 2 x 256 TMEM columns
 constexpr int kBoxBytes = 128 * 128;            // X: [128 rows x 64 fp16], 128-byte swizzled
-constexpr int kCBoxBytes = kHalfTile * 128;     // C: [64 centroids x 64 fp16], 128-byte swizzled
+constexpr int kCBoxBytes = kHalfTile * 128;     // C: [128 centroids x 64 fp16], 128-byte swizzled
 constexpr int kExtBytes = 128 * 32;             // ones: [128 rows x 16 fp16], 32-byte swizzled
-constexpr int kCExtBytes = kHalfTile * 32;      // norm slice: [64 centroids x 16 fp16], 32-byte swizzled
+constexpr int kCExtBytes = kHalfTile * 32;      // norm slice: [128 centroids x 16 fp16], 32-byte swizzled
 constexpr int kThreads = 352;                   // 11 warps: producers, MMA issuer A, 8 epilogue, MMA issuer B
 constexpr int kEpiWarp0 = 2;
 constexpr int kMmaWarpB = 10;                   // second issuer, on another SMSP than warp 1
@@ -71,7 +70,6 @@ constexpr int kEpiWarps = 8;                    // at most 3 warps per SMSP: up 
 constexpr int kColParts = kEpiWarps / 4;        // warps per TMEM lane quarter, each with a column slice
 constexpr int kPartCols = kTileK / kColParts;   // 128 columns of each tile per epilogue warp
 constexpr uint32_t kTmemCols = 512;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kXOff = 0;
@@ -80,7 +78,7 @@ constexpr int kCOff = kXOff + kXBytes;
 constexpr int kCStageBytes = kMaxBoxes * kCBoxBytes + kCExtBytes;  // 36 KB: centroid boxes + norm slice
 constexpr int kCBytes = kCStages * kCStageBytes;                    // 144 KB
 constexpr int kAOnesOff = kCOff + kCBytes;                          // 4 KB of ones (the points' extra slice)
-constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 3 parts x 128 x (score, label)
+constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 1 part x 128 rows x (score, label)
 constexpr int kMergeBytes = 2 * (kColParts - 1) * kRows * 8;
 constexpr int kBarOff = kMergeOff + kMergeBytes;
 constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 4;  // + merge handoff (2 slots x full/empty)
@@ -88,94 +86,6 @@ constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;      // + tmem sl
 static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA exceeded");
 static_assert(kCStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 
-// ---- PTX wrappers -------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint32_t cta_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// The same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// Arrive on a barrier given by its shared::cluster address (own or peer CTA).
-// Used to hand an accumulator back: the TMEM reads are already ordered by
-// tcgen05.wait::ld and tcgen05.fence::before_thread_sync, and nothing this
-// thread wrote needs to be seen by the MMA thread, so no cluster-scope
-// release (which would wait for this thread's outstanding global stores).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait: false when the CTA is aborting or the limit expired (which
-// starts the abort and records the fault).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* fault) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicExch(fault, FAULT_PIPELINE_TIMEOUT);
-            return false;
-        }
-    }
-}
-// TMA tile load into this CTA's shared memory, completing on a barrier that
-// may live in either CTA of the pair (cluster address).
-__device__ __forceinline__ void tma_load_pair(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                              uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-        "%4}], [%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
-        : "memory");
-}
-// UMMA shared-memory descriptors, K-major operands, descriptor version 1.
-//  128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
-//  32-byte swizzle:  rows of 32 bytes (one K=16 fp16 slice), 8-row groups 256 bytes apart.
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-__device__ __forceinline__ uint64_t umma_desc_sw32(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
-}
 // Instruction descriptor, kind::f16: D fp32, A and B fp16, both K-major, N=256, M=256.
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kTileK >> 3) << 17) |
                             ((uint32_t)(kUnitRows >> 4) << 24);
@@ -187,38 +97,6 @@ __device__ __forceinline__ void umma_pair_f16(uint32_t tmem_d, uint64_t adesc, u
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
         : "memory");
-}
-// Arrive on the barrier at this offset in both CTAs of the pair once every
-// MMA issued so far has completed.
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-    const uint16_t both = 0x3;
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-        "h"(both)
-        : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ float max3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-// 64 consecutive fp32 columns of this thread's TMEM lane, waited on.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
-    uint32_t r[64];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int j = 0; j < 64; ++j) v[j] = __uint_as_float(r[j]);
 }
 
 struct Params {
@@ -523,36 +401,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---- host side ------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// [B, rows, cols] fp16 with boxes of [1, box_rows, box_cols], zero fill outside.
-bool make_map(CUtensorMap* m, const void* base, int64_t B, int64_t rows, int64_t cols, int box_cols, int box_rows,
-              CUtensorMapSwizzle swz) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)B};
-    cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(rows * cols * 2)};
-    cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool assign_tc_supported(int64_t d, int dtype) { return dtype == KM_F16 && d >= 64 && d <= 128 && d % 8 == 0; }
@@ -561,9 +409,9 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* 
                              int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st) {
     if (!assign_tc_supported(d, KM_F16)) return cudaErrorNotSupported;
     CUtensorMap mx, mc, me;
-    if (!make_map(&mx, X, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mc, chat, B, K, d, kBoxK, kHalfTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&me, cext, B, padded_k(K), 16, 16, kHalfTile, CU_TENSOR_MAP_SWIZZLE_32B))
+    if (!make_map(&mx, X, 2, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mc, chat, 2, B, K, d, kBoxK, kHalfTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&me, cext, 2, B, padded_k(K), 16, 16, kHalfTile, CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -1,8 +1,9 @@
 // Centroid-side kernels of the Lloyd iteration:
 //  * preparation for the assignment: round the fp32 centroids to the dtype of
-//    X and write -||c||^2/2 as a 16-wide fp16 slice that the tensor cores
-//    add to x.c (the ||c||^2 term of the expansion ||x - c||^2 = ||x||^2 +
-//    ||c||^2 - 2 x.c, papernotes.org "Flash-KMeans" page, 关键设计 1);
+//    X (fp16), or split them into tf32 heads and tails (fp32), and write
+//    -||c||^2/2 as a slice of pieces that the tensor cores add to x.c (the
+//    ||c||^2 term of the expansion ||x - c||^2 = ||x||^2 + ||c||^2 - 2 x.c,
+//    papernotes.org "Flash-KMeans" page, 关键设计 1);
 //  * finalisation of the update: c_k = s_k / n_k, an empty cluster keeping its
 //    previous centroid (the flowchart's C_new on the same page, 整体框架);
 //  * the per-batch objective: the assignment accumulates the sum of minimum
@@ -22,8 +23,8 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
-// The centroid's norm slice for the tensor-core assignment: 16 fp16 values
-// whose sum is -v to within ~2^-33 relative (greedy pieces, each the
+// The centroid's norm slice for the fp16 tensor-core assignment: 16 fp16
+// values whose sum is -v to within ~2^-33 relative (greedy pieces, each the
 // nearest fp16 to what is left, clamped to the fp16 range).
 __device__ __forceinline__ void write_norm_slice(__half* out, double v) {
     double r = -v;
@@ -37,8 +38,40 @@ __device__ __forceinline__ void write_norm_slice(__half* out, double v) {
     for (; i < 16; ++i) out[i] = __float2half(0.f);
 }
 
+// tf32 head of an fp32 value: its low 13 mantissa bits cleared (exact in tf32).
+__device__ __forceinline__ float tf32_head(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
+
+// The same for the fp32 (tf32) assignment: 8 tf32-exact fp32 pieces whose sum
+// is -v (each piece takes ~10 more bits of what is left).
+__device__ __forceinline__ void write_norm_pieces_tf32(float* out, double v) {
+    double r = -v;
+    int i = 0;
+    for (; i < 8 && r != 0.0; ++i) {
+        const float p = tf32_head((float)r);
+        out[i] = p;
+        r -= (double)p;
+    }
+    for (; i < 8; ++i) out[i] = 0.f;
+}
+
+// Everything the assignment needs of one centroid row, from the warp's sum of
+// squares `acc` (lane 0 writes): the norm slice, and for fp32 the running
+// bound of max_k ||c_k||^2 (non-negative floats order like their bit patterns).
+__device__ __forceinline__ void write_row_norm(const PreparedC& p, int dtype, int64_t b, int64_t slice_row,
+                                               double acc) {
+    if (dtype == KM_F16) {
+        write_norm_slice(static_cast<__half*>(p.cext) + slice_row * 16, 0.5 * acc);
+    } else {
+        write_norm_pieces_tf32(static_cast<float*>(p.cext) + slice_row * 8, 0.5 * acc);
+        atomicMax(reinterpret_cast<int*>(p.cmax + b), __float_as_int((float)(acc * (1.0 + 1e-6))));
+    }
+}
+
+// One warp per centroid row of [B, Kp]: fp16 rounds C (chat) and writes the
+// fp16 norm slice; fp32 writes each row's tf32 heads and tails (chat = [B, K, 2d])
+// and the tf32 norm pieces.  Padding rows K <= k < Kp get a -inf score.
 __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, int64_t Kp, int64_t d, int dtype,
-                            __half* __restrict__ chat, __half* __restrict__ cext) {
+                            PreparedC p) {
     pdl_trigger();
     pdl_wait();
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
@@ -46,7 +79,13 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
     if (row >= B * Kp) return;
     const int64_t b = row / Kp, k = row % Kp;
     if (k >= K) {  // padding centroid: score -inf, never the maximum
-        if (lane < 16) cext[row * 16 + lane] = lane == 0 ? __ushort_as_half((unsigned short)0xFC00) : __float2half(0.f);
+        if (dtype == KM_F16) {
+            if (lane < 16)
+                static_cast<__half*>(p.cext)[row * 16 + lane] =
+                    lane == 0 ? __ushort_as_half((unsigned short)0xFC00) : __float2half(0.f);
+        } else if (lane < 8) {
+            static_cast<float*>(p.cext)[row * 8 + lane] = lane == 0 ? -INFINITY : 0.f;
+        }
         return;
     }
     const int64_t base = (b * K + k) * d;
@@ -55,23 +94,29 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
         float v = C[base + j];
         if (dtype == KM_F16) {
             const __half h = __float2half_rn(v);
-            if (chat) chat[base + j] = h;
+            if (p.chat) static_cast<__half*>(p.chat)[base + j] = h;
             v = __half2float(h);
+        } else {
+            float* row2 = static_cast<float*>(p.chat) + 2 * base;
+            const float hv = tf32_head(v);
+            row2[j] = hv;
+            row2[d + j] = v - hv;
         }
         acc += (double)v * (double)v;
     }
     acc = warp_sum(acc);
-    if (lane == 0) write_norm_slice(cext + row * 16, 0.5 * acc);
+    if (lane == 0) write_row_norm(p, dtype, b, row, acc);
 }
 
 // n_k comes from the sort's segment offsets (offsets[k+1] - offsets[k]); it is
 // also written to counts when that is non-null.  With zero_sums the consumed
-// sums are reset to 0, ready for the next iteration's boundary atomics.
+// sums are reset to 0, ready for the next iteration's boundary atomics.  When
+// `next` holds buffers, the new centroids are prepared for the next
+// assignment as prep_kernel does.
 __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t B, int64_t K,
-                                int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype, __half* __restrict__ chat,
-                                __half* __restrict__ cext, int32_t* __restrict__ counts, int zero_sums,
-                                double* __restrict__ obj_acc, float* __restrict__ obj_out,
-                                const int32_t* __restrict__ counts_in) {
+                                int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype, PreparedC next,
+                                int32_t* __restrict__ counts, int zero_sums, double* __restrict__ obj_acc,
+                                float* __restrict__ obj_out, const int32_t* __restrict__ counts_in) {
     pdl_trigger();
     pdl_wait();
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
@@ -100,20 +145,25 @@ __global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restr
         } else {
             v = *reinterpret_cast<const float4*>(C_out + base + j);
         }
+        if (!next.cext) continue;
         if (dtype == KM_F16) {
             const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
-            if (chat) {
-                *reinterpret_cast<__half2*>(chat + base + j) = h01;
-                *reinterpret_cast<__half2*>(chat + base + j + 2) = h23;
-            }
+            __half* chat = static_cast<__half*>(next.chat);
+            *reinterpret_cast<__half2*>(chat + base + j) = h01;
+            *reinterpret_cast<__half2*>(chat + base + j + 2) = h23;
             const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
             v = make_float4(f01.x, f01.y, f23.x, f23.y);
+        } else {
+            float* row2 = static_cast<float*>(next.chat) + 2 * base;
+            const float4 hv = make_float4(tf32_head(v.x), tf32_head(v.y), tf32_head(v.z), tf32_head(v.w));
+            *reinterpret_cast<float4*>(row2 + j) = hv;
+            *reinterpret_cast<float4*>(row2 + d + j) = make_float4(v.x - hv.x, v.y - hv.y, v.z - hv.z, v.w - hv.w);
         }
         acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
     }
-    if (cext) {
+    if (next.cext) {
         acc = warp_sum(acc);
-        if (lane == 0) write_norm_slice(cext + (b * Kp + k) * 16, 0.5 * acc);
+        if (lane == 0) write_row_norm(next, dtype, b, b * Kp + k, acc);
     }
 }
 
@@ -134,24 +184,22 @@ cudaError_t launch_add_counts(const int32_t* offsets, int64_t B, int64_t K, int3
                          counts);
 }
 
-cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
-                                  __half* cext, cudaStream_t st) {
+cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, PreparedC p,
+                                  cudaStream_t st) {
     const int64_t Kp = padded_k(K);
     const int64_t rows = B * Kp;
     const int warps = 8;
     return launch_kernel(prep_kernel, dim3((unsigned)ceil_div(rows, warps)), dim3(warps * 32), 0, st, C, B, K, Kp, d,
-                         dtype, chat, cext);
+                         dtype, p);
 }
 
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
-                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, double* obj_acc,
+                            int dtype, PreparedC next, int32_t* counts, bool zero_sums, double* obj_acc,
                             float* obj_out, cudaStream_t st, const int32_t* counts_in) {
     const int warps = 8;
     return launch_kernel(finalize_kernel, dim3((unsigned)ceil_div(B * K, warps)), dim3(warps * 32), 0, st, sums,
-                         offsets, B, K, padded_k(K), d, C_out, dtype, chat, cext, counts, zero_sums ? 1 : 0, obj_acc,
+                         offsets, B, K, padded_k(K), d, C_out, dtype, next, counts, zero_sums ? 1 : 0, obj_acc,
                          obj_out, counts_in);
-    return cudaGetLastError();
 }
-
 
 }  // namespace km

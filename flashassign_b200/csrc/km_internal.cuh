@@ -17,6 +17,9 @@ km_status cuda_error(cudaError_t e, const char* what);
 // Device fault word: kernels write a non-zero code when a bounded wait expires.
 enum : int32_t { FAULT_NONE = 0, FAULT_PIPELINE_TIMEOUT = 1 };
 int32_t* fault_word();  // device address of the word on the current device
+// Running count of points the fp32 tensor-core assignment left to the exact
+// re-scan (device address on the current device).
+unsigned long long* rescan_word();
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -66,20 +69,30 @@ struct DeviceInfo {
 km_status device_info(DeviceInfo* out);
 
 // ---- launchers (all asynchronous on `st`) ----
-// Centroid preparation for the tensor-core assignment: chat = fp16(C) (RNE)
-// and cext[b][k][0..16) = fp16 pieces summing to -||chat_k||^2 / 2 for k < K,
-// (-inf, 0, ...) for K <= k < padded_k(K).
-cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, __half* chat,
-                                  __half* cext, cudaStream_t st);
+// Centroids prepared for a tensor-core assignment (buffers owned by the caller):
+//  fp16 X: chat = [B, K, d] fp16, C rounded RNE; cext = [B, Kp, 16] fp16 pieces
+//          summing to -||chat_k||^2 / 2;
+//  fp32 X: chat = [B, K, 2d] fp32, each row the tf32 heads of c (low 13 mantissa
+//          bits cleared) then the tails c - head; cext = [B, Kp, 8] tf32-exact
+//          fp32 pieces summing to -||c_k||^2 / 2; cmax = [B] running upper bound
+//          of max_k ||c_k||^2 (atomic max; zero it before the first preparation).
+// Rows K <= k < Kp = padded_k(K) of cext give the score -inf.
+struct PreparedC {
+    void* chat = nullptr;
+    void* cext = nullptr;
+    float* cmax = nullptr;
+};
+cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t d, int dtype, PreparedC p,
+                                  cudaStream_t st);
 
 // C_out[b][k] = sums / n_k where n_k > 0 (else unchanged), n_k taken from the
-// segment offsets [B, K+1] (and written to counts when non-null); when chat
-// or cext is non-null, also prepares the next assignment's centroids from
-// C_out; with zero_sums the sums are reset to 0 once consumed.
+// segment offsets [B, K+1] (and written to counts when non-null); when `next`
+// holds buffers, also prepares the next assignment's centroids from C_out;
+// with zero_sums the sums are reset to 0 once consumed.
 // When obj_out is non-null, obj_out[b] = obj_acc[b] (as fp32) and obj_acc[b] = 0.
 // n_k is taken from counts_in when it is non-null, else from the offsets.
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
-                            int dtype, __half* chat, __half* cext, int32_t* counts, bool zero_sums, double* obj_acc,
+                            int dtype, PreparedC next, int32_t* counts, bool zero_sums, double* obj_acc,
                             float* obj_out, cudaStream_t st, const int32_t* counts_in = nullptr);
 
 // Tensor-core assignment (fp16, 64 <= d <= 128).  Returns cudaErrorNotSupported
@@ -89,10 +102,23 @@ bool assign_tc_supported(int64_t d, int dtype);
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
                              int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st);
 
-// CUDA-core assignment for every supported shape (fp32 inputs, and fp16
-// shapes outside the tensor-core kernel's range): direct-difference distances.
+// Tensor-core assignment of fp32 points (tf32 head/tail split, 32 <= d <= 128,
+// d % 32 == 0).  Points whose best two scores lie within the split's error
+// bound are not resolved: they are appended to flag_rows[b * N + ...]
+// (flag_count [B] must be zero on entry) for launch_assign_simt's list mode,
+// and left out of obj_acc.
+bool assign_tf32_supported(int64_t d);
+cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float* cext, const float* cmax, int64_t B,
+                               int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
+                               int32_t* flag_count, int32_t* flag_rows, int sms, cudaStream_t st);
+
+// CUDA-core assignment for every supported shape: direct-difference
+// distances.  With `list`, only the list_count[b] points list[b * N + r] of
+// each batch are assigned, by at most max_blocks blocks per batch.
 cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
-                               int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st);
+                               int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st,
+                               const int32_t* list = nullptr, const int32_t* list_count = nullptr,
+                               int max_blocks = 0);
 
 // Stable LSD radix argsort of labels in [0, K).  Scratch: sort_scratch_bytes().
 size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K);

@@ -102,7 +102,10 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
     __half* chat = static_cast<__half*>(base);
     __half* cext = reinterpret_cast<__half*>(static_cast<unsigned char*>(base) + chat_bytes);
     // every element of both scratch regions that the assignment reads is written here first
-    cudaError_t e = launch_prep_centroids(C, B, K, d, dtype, chat, cext, stm);
+    PreparedC prep;
+    prep.chat = chat;
+    prep.cext = cext;
+    cudaError_t e = launch_prep_centroids(C, B, K, d, dtype, prep, stm);
     if (e != cudaSuccess) return cuda_error(e, "km_assign_noalloc: centroid preparation");
     e = launch_assign_tc(static_cast<const __half*>(X), chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms,
                          stm);

@@ -65,8 +65,14 @@ typedef enum {
  *     mindist[b][i] = that minimum squared distance (clamped at 0).
  * The distance is expanded as ||x||^2 + ||c||^2 - 2 x.c; the N x K distance
  * matrix is never written to memory.  The centroids are first rounded
- * (round-to-nearest-even) to `dtype`, and x.c is accumulated in fp32 on the
- * tensor cores (fp16) or in fp32 on the CUDA cores (fp32 inputs).
+ * (round-to-nearest-even) to `dtype`, and x.c is accumulated in fp32:
+ *   - fp16, 64 <= d <= 128: on the tensor cores;
+ *   - fp32, d in {32, 64, 96, 128}: on the tensor cores from tf32 head/tail
+ *     splits of both operands (three products); a point whose best two scores
+ *     lie within the split's error bound is re-scanned exactly on the CUDA
+ *     cores, so every label is the exact argmin up to fp32 rounding (see
+ *     km_assign_rescans);
+ *   - other shapes: direct differences sum_j (x_j - c_j)^2 on the CUDA cores.
  *   X       [B, N, d] dtype, device.     C [B, K, d] fp32, device.
  *   labels  [B, N] int32, device, written.
  *   mindist [B, N] fp32, device, written; may be NULL.
@@ -186,6 +192,16 @@ KM_API const char* km_last_error(void);
  * Returns KM_OK with *code = 0 when no fault was recorded.
  */
 KM_API km_status km_device_fault(int32_t* code, void* stream);
+
+/*
+ * Reads and clears the number of points, on the current device, that the
+ * fp32 tensor-core assignment could not resolve within its error bound and
+ * handed to the exact CUDA-core re-scan since the last call (near ties,
+ * duplicate centroids, data far from the origin).  Not a result of the
+ * method -- an observability counter for its numerics; 0 on fp16 and
+ * CUDA-core paths.  Synchronises `stream`.
+ */
+KM_API km_status km_assign_rescans(int64_t* count, void* stream);
 
 #ifdef __cplusplus
 }

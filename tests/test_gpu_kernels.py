@@ -43,9 +43,16 @@ ASSIGN_SHAPES = [
     (2, 600, 200, 96, "f16"),
     (2, 500, 100, 16, "f16"),    # below the tensor-core range: CUDA-core kernel
     (2, 300, 50, 256, "f16"),    # above it
-    (1, 4096, 8, 16, "f32"),
-    (2, 1000, 300, 128, "f32"),
+    (1, 4096, 8, 16, "f32"),     # fp32 below the tf32 tensor-core range (d % 32 != 0): CUDA cores
     (2, 129, 33, 4, "f32"),
+    (1, 1, 1, 32, "f32"),        # fp32 on tf32 tensor cores: d in {32, 64, 96, 128}
+    (1, 129, 127, 128, "f32"),
+    (2, 257, 255, 32, "f32"),
+    (3, 255, 129, 64, "f32"),
+    (2, 777, 257, 96, "f32"),
+    (2, 1000, 300, 128, "f32"),
+    (2, 1000, 513, 128, "f32"),
+    (1, 300, 50, 160, "f32"),    # above it
 ]
 
 
@@ -59,11 +66,11 @@ def test_assign_matches_oracle(B, N, K, d, dt):
     check_labels(X, C, lab, md)
 
 
-@pytest.mark.parametrize("dt", ["f16", "f32"])
-def test_assign_ties_go_to_the_lowest_index(dt):
+@pytest.mark.parametrize("dt,d", [("f16", 128), ("f32", 16), ("f32", 128)])
+def test_assign_ties_go_to_the_lowest_index(dt, d):
     # integer coordinates and duplicate centroids give exact ties in every precision
     rng = np.random.default_rng(11)
-    B, N, K, d = 2, 700, 260, 128 if dt == "f16" else 16
+    B, N, K = 2, 700, 260
     npdt = np.float16 if dt == "f16" else np.float32
     X = rng.integers(-2, 3, (B, N, d)).astype(npdt)
     base = rng.integers(-2, 3, (B, 40, d)).astype(np.float32)
@@ -72,6 +79,38 @@ def test_assign_ties_go_to_the_lowest_index(dt):
     ref, d1, d2 = oracle.assign(X, C)
     assert np.array_equal(lab, ref)
     assert np.array_equal(md, d1.astype(np.float32))
+
+
+def test_fp32_tensor_cores_resolve_clear_points_and_list_the_rest():
+    # well-separated mixture: almost every point is resolved by the tf32 tensor cores
+    w = synth.small(B=2, N=4000, d=128, K=300, dtype="f32", ncomp=150, sigma=0.3, seed=77)
+    X = synth.points(w)
+    C = synth.init_centroids(w, X)
+    km.assign_rescans()
+    lab, md = run_assign(X, C)
+    listed = km.assign_rescans()
+    check_labels(X, C, lab, md)
+    assert listed < 0.05 * w.B * w.N, f"{listed} of {w.B * w.N} points needed the exact re-scan"
+    # identical centroids: every score ties, every point goes to the re-scan and to centroid 0
+    C_same = np.repeat(C[:, :1], 300, axis=1)
+    lab, md = run_assign(X, C_same)
+    assert km.assign_rescans() == w.B * w.N
+    assert (lab == 0).all()
+    check_labels(X, C_same, lab, md)
+
+
+def test_fp32_tensor_cores_exact_where_the_gap_is_clear_far_from_the_origin():
+    # points and centroids offset from the origin: ||x||^2 and ||c||^2 dwarf the distances, so the
+    # expansion cancels; labels must still be exact wherever the relative top-2 gap is >= 1e-5
+    rng = np.random.default_rng(78)
+    B, N, K, d = 2, 3000, 200, 64
+    centres = rng.standard_normal((B, 40, d)) + 4.0
+    X = (centres[:, rng.integers(0, 40, N)] + 0.05 * rng.standard_normal((B, N, d))).astype(np.float32)
+    C = X[:, rng.choice(N, K, replace=False)].copy()
+    km.assign_rescans()
+    lab, md = run_assign(X, C)
+    km.assign_rescans()
+    check_labels(X, C, lab, md)
 
 
 def test_assign_single_centroid_and_far_centroids():
@@ -140,7 +179,8 @@ def test_update_matches_oracle(B, N, K, d, dt, case):
     check_centroids(X, lab, C_prev, C_out.cpu().numpy(), counts.cpu().numpy(), sums.cpu().numpy())
 
 
-@pytest.mark.parametrize("B,N,K,d,dt", [(2, 3000, 50, 128, "f16"), (1, 4096, 8, 16, "f32"), (2, 1000, 300, 64, "f16")])
+@pytest.mark.parametrize("B,N,K,d,dt", [(2, 3000, 50, 128, "f16"), (1, 4096, 8, 16, "f32"), (2, 1000, 300, 64, "f16"),
+                                        (2, 3000, 50, 128, "f32"), (1, 2000, 257, 32, "f32")])
 def test_lloyd_lockstep_with_oracle(B, N, K, d, dt):
     """Each iteration: the oracle takes the GPU's centroids and checks that iteration's labels and update."""
     w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=5 + K)
