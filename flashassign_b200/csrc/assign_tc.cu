@@ -32,12 +32,12 @@
 //     the MMAs (alternate tiles: one thread issues at most ~1 MMA per 100
 //     cycles) and commit them to both CTAs' barriers; warps 2..9 are the
 //     epilogue: TMEM lane = point row, two warps per row split each tile's
-//     256 columns in 128-column slices, read 64 columns at a time; the
-//     accumulator is released as soon as the last 64 are in registers.
+//     256 columns in 128-column slices, read in one 128-column TMEM load; the
+//     accumulator is released as soon as they are in registers.
 //   * Epilogue: per 32-column group, the group maximum (3-input max) is
-//     compared with the running best; only when it improves are the group's
-//     32 scores kept in registers, and the winning column is resolved once
-//     per unit from the kept group (first column equal to the maximum).  The
+//     compared with the running best; only when it improves (in any lane of
+//     the warp) is the group scanned for its first column equal to the
+//     maximum, which becomes the running label.  The
 //     two column slices of a row are joined in shared memory (larger score,
 //     then lower index).  mindist = ||x||^2 - 2 * best, ||x||^2 summed from
 //     the staged X tile.
@@ -268,10 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t xb = it_x % kXBufs;
             float xnorm = 0.f;
             float best = -INFINITY;
-            int gbest = -1;    // column of the first score of the group holding the running best
-            float kept[32];    // that group's 32 scores
-#pragma unroll
-            for (int j = 0; j < 32; ++j) kept[j] = -INFINITY;
+            int label = -1;    // column of the running best
             for (int kt = 0; kt < P.ktiles; ++kt, ++it_a) {
                 const uint32_t s = it_a % kAccSets;
                 if (!(ok = mbar_wait(bar_acc_full + 8 * s, (it_a / kAccSets) & 1, abort_flag, P.fault))) break;
@@ -302,19 +299,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
                 }
-#pragma unroll 1
-                for (int sub = 0; sub < kPartCols / 64; ++sub) {
-                  // 64 columns at a time; the accumulator is handed back as soon as
-                  // its last columns are in registers, before their arithmetic
-                  float v[64];
-                  tmem_ld64(tcol + sub * 64, v);
-                  if (sub == kPartCols / 64 - 1) {
-                      tc_fence_before();
-                      __syncwarp();
-                      if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
-                  }
+                // this warp's 128 columns in one load; the accumulator is handed
+                // back as soon as they are in registers, before their arithmetic
+                float v[kPartCols];
+                tmem_ld128(tcol, v);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
 #pragma unroll
-                  for (int g = 0; g < 2; ++g) {
+                for (int g = 0; g < kPartCols / 32; ++g) {
                     const float* w = v + 32 * g;
                     // two interleaved 3-input chains: few live temporaries
                     float ga = max3(w[0], w[1], w[2]), gb = max3(w[3], w[4], w[5]);
@@ -326,22 +319,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const float gmax = max3(max3(ga, w[30], w[31]), gb, gb);
                     const bool better = gmax > best;  // strict: an earlier group keeps ties
                     if (__any_sync(0xffffffffu, better)) {
+                        // the first column of the group holding its maximum
+                        int j0 = 31;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) kept[j] = better ? w[j] : kept[j];
+                        for (int j = 31; j >= 0; --j) j0 = (w[j] == gmax) ? j : j0;
+                        if (better) {
+                            best = gmax;
+                            label = kt * kTileK + h * kPartCols + g * 32 + j0;
+                        }
                     }
-                    if (better) {
-                        best = gmax;
-                        gbest = kt * kTileK + h * kPartCols + sub * 64 + g * 32;
-                    }
-                  }
                 }
             }
             if (!ok) break;
-            // this slice's winner: the first column of the kept group holding the maximum
-            int j0 = 31;
-#pragma unroll
-            for (int j = 31; j >= 0; --j) j0 = (kept[j] == best) ? j : j0;
-            const int label = gbest < 0 ? -1 : gbest + j0;
             // join the column slices of each row (larger score, then lower
             // index) through a double-buffered shared slot with bounded handoffs
             const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;

@@ -9,11 +9,11 @@
 //   1. a per-tile digit histogram (2048 keys per CTA),
 //   2. an exclusive scan over (digit, tile) per batch (done by each scatter
 //      CTA itself when the histogram is small),
-//   3. a scatter in which each warp ranks its keys with __match_any_sync, the
-//      warps of a tile are combined by a per-digit scan (equal digits keep
-//      their input order: stability), the tile is laid out digit by digit in
-//      shared memory, and each digit's run is written to consecutive global
-//      positions (coalesced stores).
+//   3. a scatter in which each warp ranks its keys by ballots over the digit
+//      bits (which lanes hold an equal digit), the warps of a tile are
+//      combined by a per-digit scan (equal digits keep their input order:
+//      stability), the tile is laid out digit by digit in shared memory, and
+//      each digit's run is written to consecutive global positions.
 // The segment offsets and counts then follow from the sorted labels without
 // any atomics: position p starts label k exactly when a[p-1] < k <= a[p].
 #include "km_internal.cuh"
@@ -142,8 +142,22 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
         const bool valid = i < N;
         key[s] = valid ? keys_in[b * N + i] : 0;
         val[s] = valid ? (vals_in ? vals_in[b * N + i] : (int)i) : 0;
-        const int dig = valid ? ((key[s] >> shift) & mask) : 256;  // 256: never a real digit
-        const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+    }
+#pragma unroll
+    for (int s = 0; s < kItems; ++s) {
+        const int64_t i = base + s * 32 + lane;
+        const bool valid = i < N;
+        const int dig = (key[s] >> shift) & mask;
+        // the lanes holding the same digit: one ballot per digit bit
+        uint32_t peers = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+        for (int bit = 0; bit < 8; ++bit) {
+            if (bit < bits) {
+                const bool on = (dig >> bit) & 1;
+                const uint32_t bal = __ballot_sync(0xffffffffu, on);
+                peers &= on ? bal : ~bal;
+            }
+        }
         const int cnt = valid ? wh[w][dig] : 0;
         rank[s] = cnt + __popc(peers & lt);
         __syncwarp();
@@ -193,16 +207,29 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
     //    CTA sums it itself (all earlier digits of the batch plus this digit's
     //    earlier tiles); otherwise the scanned offsets are read.
     if (hist) {
+        // each warp sums digits w, w + 8, ...: its lanes load a digit's tiles
+        // side by side (all loads of a warp independent), a warp reduction
+        // gives the digit's total and its count in the tiles before this one
         __shared__ int wsum[kWarps];
-        int tot = 0, mine = 0;
-        if (threadIdx.x < bins) {
-            const int32_t* hd = hist + (b * bins + threadIdx.x) * T;
-            for (int64_t t2 = 0; t2 < T; ++t2) {
+        __shared__ int d_tot[256], d_mine[256];
+        for (int d0 = w; d0 < bins; d0 += kWarps) {
+            const int32_t* hd = hist + (b * bins + d0) * T;
+            int tot_l = 0, mine_l = 0;
+            for (int64_t t2 = lane; t2 < T; t2 += 32) {
                 const int c = hd[t2];
-                tot += c;
-                if (t2 < tile) mine += c;
+                tot_l += c;
+                mine_l += t2 < tile ? c : 0;
+            }
+            tot_l = __reduce_add_sync(0xffffffffu, tot_l);
+            mine_l = __reduce_add_sync(0xffffffffu, mine_l);
+            if (lane == 0) {
+                d_tot[d0] = tot_l;
+                d_mine[d0] = mine_l;
             }
         }
+        __syncthreads();
+        const int tot = threadIdx.x < bins ? d_tot[threadIdx.x] : 0;
+        const int mine = threadIdx.x < bins ? d_mine[threadIdx.x] : 0;
         int incl = tot;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

@@ -122,7 +122,8 @@ def test_assign_single_centroid_and_far_centroids():
     check_labels(X, C, lab, md)
 
 
-@pytest.mark.parametrize("case", ["random", "all_equal", "k1", "sorted", "skewed", "big_k", "ragged"])
+@pytest.mark.parametrize("case", ["random", "all_equal", "k1", "sorted", "skewed", "big_k", "ragged",
+                                  "one_pass_max", "one_pass_tiles", "one_pass_tail", "k4096", "long_small_k"])
 def test_sort_is_bit_exact(case):
     rng = np.random.default_rng(13)
     B, N, K = 3, 5000, 1024
@@ -140,9 +141,24 @@ def test_sort_is_bit_exact(case):
     elif case == "big_k":
         K = 65536
         lab = rng.integers(0, K, (B, N))
-    else:
+    elif case == "ragged":
         B, N, K = 2, 2049, 3000  # one key past a 2048-key tile; 12-bit keys
         lab = rng.integers(0, K, (B, N))
+    elif case == "one_pass_max":
+        B, N, K = 2, 9000, 2048  # the largest single-pass label range
+        lab = rng.integers(0, K, (B, N))
+    elif case == "one_pass_tiles":
+        B, N, K = 2, 70000, 2000  # 18 tiles of 4096 keys, the last one ragged
+        lab = rng.integers(0, K, (B, N))
+    elif case == "long_small_k":
+        B, N, K = 1, 300000, 1000  # more tiles than the single pass takes: two 5-bit radix passes
+        lab = rng.integers(0, K, (B, N))
+    elif case == "one_pass_tail":
+        B, N, K = 3, 4097, 5  # one key past a 4096-key tile, a few labels
+        lab = rng.integers(0, K, (B, N))
+    else:
+        B, N, K = 2, 20000, 4096  # two 6-bit passes
+        lab = np.minimum(rng.zipf(1.1, (B, N)) - 1, K - 1)
     lab = lab.astype(np.int32)
     sidx, counts, offsets = km.sort_labels(cuda(lab), K)
     torch.cuda.synchronize()
