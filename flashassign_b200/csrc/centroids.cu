@@ -8,8 +8,8 @@
 //    previous centroid (the flowchart's C_new on the same page, 整体框架);
 //  * the per-batch objective: the assignment accumulates the sum of minimum
 //    distances, the finalisation hands it out and resets the accumulator.
-// All three are tiny next to the assignment and the gather; one warp per
-// centroid row keeps them coalesced.
+// All three are tiny next to the assignment and the gather; the preparation
+// takes one warp per centroid row, the finalisation eight lanes per row.
 #include "km_internal.cuh"
 
 #include <cmath>
@@ -25,17 +25,24 @@ __device__ __forceinline__ double warp_sum(double v) {
 
 // The centroid's norm slice for the fp16 tensor-core assignment: 16 fp16
 // values whose sum is -v to within ~2^-33 relative (greedy pieces, each the
-// nearest fp16 to what is left, clamped to the fp16 range).
+// nearest fp16 to what is left, clamped to the fp16 range), stored as two
+// 16-byte vectors.
 __device__ __forceinline__ void write_norm_slice(__half* out, double v) {
     double r = -v;
-    int i = 0;
-    for (; i < 16 && r != 0.0; ++i) {  // typically 3-4 pieces leave nothing
-        const double c = fmin(fmax(r, -65504.0), 65504.0);
-        const __half p = __float2half_rn((float)c);
-        out[i] = p;
-        r -= (double)__half2float(p);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        __half p[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // once r is 0 every further piece is 0
+            const double c = fmin(fmax(r, -65504.0), 65504.0);
+            p[h] = __float2half_rn((float)c);
+            r -= (double)__half2float(p[h]);
+        }
+        w[i] = (uint32_t)__half_as_ushort(p[0]) | ((uint32_t)__half_as_ushort(p[1]) << 16);
     }
-    for (; i < 16; ++i) out[i] = __float2half(0.f);
+    reinterpret_cast<uint4*>(out)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(out)[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
 // tf32 head of an fp32 value: its low 13 mantissa bits cleared (exact in tf32).
@@ -45,13 +52,14 @@ __device__ __forceinline__ float tf32_head(float v) { return __uint_as_float(__f
 // is -v (each piece takes ~10 more bits of what is left).
 __device__ __forceinline__ void write_norm_pieces_tf32(float* out, double v) {
     double r = -v;
-    int i = 0;
-    for (; i < 8 && r != 0.0; ++i) {
-        const float p = tf32_head((float)r);
-        out[i] = p;
-        r -= (double)p;
+    float p[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        p[i] = tf32_head((float)r);
+        r -= (double)p[i];
     }
-    for (; i < 8; ++i) out[i] = 0.f;
+    reinterpret_cast<float4*>(out)[0] = make_float4(p[0], p[1], p[2], p[3]);
+    reinterpret_cast<float4*>(out)[1] = make_float4(p[4], p[5], p[6], p[7]);
 }
 
 // Everything the assignment needs of one centroid row, from the warp's sum of
@@ -108,62 +116,71 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
     if (lane == 0) write_row_norm(p, dtype, b, row, acc);
 }
 
+// Lanes per centroid row in the finalisation: each lane takes every eighth
+// 4-wide chunk of the row, a warp finalises four rows at once.
+constexpr int kFinLanes = 8;
+constexpr int kFinThreads = 256;
+
 // n_k comes from the sort's segment offsets (offsets[k+1] - offsets[k]); it is
 // also written to counts when that is non-null.  With zero_sums the consumed
 // sums are reset to 0, ready for the next iteration's boundary atomics.  When
 // `next` holds buffers, the new centroids are prepared for the next
-// assignment as prep_kernel does.
-__global__ void finalize_kernel(float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t B, int64_t K,
-                                int64_t Kp, int64_t d, float* __restrict__ C_out, int dtype, PreparedC next,
-                                int32_t* __restrict__ counts, int zero_sums, double* __restrict__ obj_acc,
-                                float* __restrict__ obj_out, const int32_t* __restrict__ counts_in) {
+// assignment as prep_kernel does.  Grid: (rows of a batch / 32, B).
+__global__ void __launch_bounds__(kFinThreads) finalize_kernel(
+    float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t K, int64_t Kp, int64_t d,
+    float* __restrict__ C_out, int dtype, PreparedC next, int32_t* __restrict__ counts, int zero_sums,
+    double* __restrict__ obj_acc, float* __restrict__ obj_out, const int32_t* __restrict__ counts_in) {
     pdl_trigger();
     pdl_wait();
-    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-    const int lane = threadIdx.x & 31;
-    if (obj_out && row < B && lane == 0) {  // this iteration's objective, and a fresh accumulator
-        obj_out[row] = (float)obj_acc[row];
-        obj_acc[row] = 0.0;
+    const int64_t b = blockIdx.y;
+    const int sub = threadIdx.x % kFinLanes;
+    const int64_t k = ((int64_t)blockIdx.x * kFinThreads + threadIdx.x) / kFinLanes;
+    if (obj_out && blockIdx.x == 0 && threadIdx.x == 0) {  // this iteration's objective, and a fresh accumulator
+        obj_out[b] = (float)obj_acc[b];
+        obj_acc[b] = 0.0;
     }
-    if (row >= B * K) return;
-    const int64_t b = row / K, k = row % K;
-    const int32_t n = counts_in ? counts_in[row] : offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
-    if (counts && lane == 0) counts[row] = n;
-    const float fn = (float)n;
+    const bool valid = k < K;  // the warp's shuffles below need every lane, valid or not
+    const int64_t row = b * K + k;
+    int32_t n = 0;
+    if (valid) n = counts_in ? counts_in[row] : offsets[b * (K + 1) + k + 1] - offsets[b * (K + 1) + k];
+    if (valid && counts && sub == 0) counts[row] = n;
+    const float inv = n > 0 ? 1.0f / (float)n : 0.f;  // the mean as s * (1/n): within 1 ulp of s / n
     const int64_t base = row * d;
     double acc = 0.0;
-    // four consecutive coordinates per lane (d is a multiple of 4)
-    for (int64_t j = 4 * lane; j < d; j += 128) {
-        // the sums are read whatever the count (zero for an empty cluster), so the
-        // load does not wait for the offsets
-        const float4 sv = *reinterpret_cast<const float4*>(sums + base + j);
-        float4 v;
-        if (n > 0) {
-            v = make_float4(sv.x / fn, sv.y / fn, sv.z / fn, sv.w / fn);
-            *reinterpret_cast<float4*>(C_out + base + j) = v;
-            if (zero_sums) *reinterpret_cast<float4*>(sums + base + j) = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-            v = *reinterpret_cast<const float4*>(C_out + base + j);
+    if (valid) {
+        for (int64_t j = 4 * sub; j < d; j += 4 * kFinLanes) {
+            // the sums are read whatever the count (zero for an empty cluster), so the
+            // load does not wait for the offsets
+            const float4 sv = *reinterpret_cast<const float4*>(sums + base + j);
+            float4 v;
+            if (n > 0) {
+                v = make_float4(sv.x * inv, sv.y * inv, sv.z * inv, sv.w * inv);
+                *reinterpret_cast<float4*>(C_out + base + j) = v;
+                if (zero_sums) *reinterpret_cast<float4*>(sums + base + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                v = *reinterpret_cast<const float4*>(C_out + base + j);
+            }
+            if (!next.cext) continue;
+            if (dtype == KM_F16) {
+                const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+                __half* chat = static_cast<__half*>(next.chat);
+                *reinterpret_cast<__half2*>(chat + base + j) = h01;
+                *reinterpret_cast<__half2*>(chat + base + j + 2) = h23;
+                const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+                v = make_float4(f01.x, f01.y, f23.x, f23.y);
+            } else {
+                float* row2 = static_cast<float*>(next.chat) + 2 * base;
+                const float4 hv = make_float4(tf32_head(v.x), tf32_head(v.y), tf32_head(v.z), tf32_head(v.w));
+                *reinterpret_cast<float4*>(row2 + j) = hv;
+                *reinterpret_cast<float4*>(row2 + d + j) = make_float4(v.x - hv.x, v.y - hv.y, v.z - hv.z, v.w - hv.w);
+            }
+            acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
         }
-        if (!next.cext) continue;
-        if (dtype == KM_F16) {
-            const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
-            __half* chat = static_cast<__half*>(next.chat);
-            *reinterpret_cast<__half2*>(chat + base + j) = h01;
-            *reinterpret_cast<__half2*>(chat + base + j + 2) = h23;
-            const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-            v = make_float4(f01.x, f01.y, f23.x, f23.y);
-        } else {
-            float* row2 = static_cast<float*>(next.chat) + 2 * base;
-            const float4 hv = make_float4(tf32_head(v.x), tf32_head(v.y), tf32_head(v.z), tf32_head(v.w));
-            *reinterpret_cast<float4*>(row2 + j) = hv;
-            *reinterpret_cast<float4*>(row2 + d + j) = make_float4(v.x - hv.x, v.y - hv.y, v.z - hv.z, v.w - hv.w);
-        }
-        acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
     }
     if (next.cext) {
-        acc = warp_sum(acc);
-        if (lane == 0) write_row_norm(next, dtype, b, b * Kp + k, acc);
+#pragma unroll
+        for (int o = kFinLanes / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (valid && sub == 0) write_row_norm(next, dtype, b, b * Kp + k, acc);
     }
 }
 
@@ -196,10 +213,9 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
                             int dtype, PreparedC next, int32_t* counts, bool zero_sums, double* obj_acc,
                             float* obj_out, cudaStream_t st, const int32_t* counts_in) {
-    const int warps = 8;
-    return launch_kernel(finalize_kernel, dim3((unsigned)ceil_div(B * K, warps)), dim3(warps * 32), 0, st, sums,
-                         offsets, B, K, padded_k(K), d, C_out, dtype, next, counts, zero_sums ? 1 : 0, obj_acc,
-                         obj_out, counts_in);
+    const dim3 grid((unsigned)ceil_div(K * kFinLanes, kFinThreads), (unsigned)B);
+    return launch_kernel(finalize_kernel, grid, dim3(kFinThreads), 0, st, sums, offsets, K, padded_k(K), d, C_out, dtype,
+                         next, counts, zero_sums ? 1 : 0, obj_acc, obj_out, counts_in);
 }
 
 }  // namespace km
