@@ -34,23 +34,26 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captures summarised in profiles/assign_tc_kernel_b32_n65536_k1024_d128_f16.md and
 # profiles/update_kernel_b32_n65536_k1024_d128_f16.md, each valid only for the kernel source it was
 # taken on (sha1 of the .cu file); reported as null once that source changes.
-ASSIGN_TRAFFIC = {"sha1": ["0a203d68193b824e70e267411cda0959ae9919af", "f0924f98116dbe93ff46af367ce72068d83b6d27"],
-                  "bytes": 546.434816e6 + 12.584192e6}
-UPDATE_TRAFFIC = {"sha1": ["c9054cceeb01068c671f1d62d9236f6ddc985079", "f0924f98116dbe93ff46af367ce72068d83b6d27"],
+ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "3015919e48a9e44baf28be864699cba7d20ad824",
+                            "tc_ptx.cuh": "ee9645b484e88174263ad58b26408994fd536d40",
+                            "km_internal.cuh": "475c6be450de2a4cc966941be94fbf1e05e59b0b"},
+                  "bytes": 546.350592e6 + 10.823680e6}
+UPDATE_TRAFFIC = {"files": {"update.cu": "c9054cceeb01068c671f1d62d9236f6ddc985079",
+                            "km_internal.cuh": "f0924f98116dbe93ff46af367ce72068d83b6d27"},
                   "bytes": 557.689088e6 + 16.940288e6}
 
 
-def traffic_for(src: str, rec: dict):
-    """The recorded traffic while the kernel's source and the shared internal header are unchanged."""
+def traffic_for(rec: dict):
+    """The recorded traffic while every source file the kernel is built from is unchanged."""
     import hashlib
-    hashes = []
-    for name in (src, "km_internal.cuh"):
+    for name, want in rec["files"].items():
         try:
             with open(os.path.join(ROOT, "flashassign_b200", "csrc", name), "rb") as f:
-                hashes.append(hashlib.sha1(f.read()).hexdigest())
+                if hashlib.sha1(f.read()).hexdigest() != want:
+                    return None
         except OSError:
             return None
-    return rec["bytes"] if hashes == rec["sha1"] else None
+    return rec["bytes"]
 
 
 def parse():
@@ -352,13 +355,13 @@ def run_ours(args, w):
         "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "global_problems": w.B * world,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (X is 512 MiB)"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": round(tflops / peak_tf, 4), "traffic": traffic_for("assign_tc.cu", ASSIGN_TRAFFIC),
+                     "frac": round(tflops / peak_tf, 4), "traffic": traffic_for(ASSIGN_TRAFFIC),
                      "kernel": "assign_tc_kernel",
                      "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)",
                      "ms_per_launch": round(t_assign, 4)},
         "roofline_update": {"bound": "hbm", "achieved": round(upd_gbs, 1), "peak": peak_bw, "unit": "GB/s",
                             "frac": round(upd_gbs / peak_bw, 4), "kernel": "update_kernel",
-                            "traffic": traffic_for("update.cu", UPDATE_TRAFFIC),
+                            "traffic": traffic_for(UPDATE_TRAFFIC),
                             "ms_per_launch": round(t_update, 4), "peak_source": peak_src},
         "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4)},
         "phases_ms_per_iter": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
