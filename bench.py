@@ -66,6 +66,7 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-ablations", action="store_true", help="skip the dense-assign and scatter-update baselines")
     return p.parse_args()
 
 
@@ -207,6 +208,45 @@ def run_reference(args, w):
     return 0
 
 
+def run_ablations(w, X, C, labels, stream, calls: int = 3):
+    """The method's assignment and update against the two baselines it replaces, on the same inputs:
+    the dense-distance assignment (the N x K score matrix written to HBM and read back) and the
+    scatter-atomic update (one atomic per point coordinate).  Milliseconds per call, CUDA events."""
+    import torch
+    import flashassign_b200 as km
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(calls):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / calls
+
+    lab = torch.empty_like(labels)
+    md = torch.empty((w.B, w.N), dtype=torch.float32, device="cuda")
+    fused = timed(lambda: km.assign(X, C, labels=lab, mindist=md))
+    dense = timed(lambda: km.assign_dense(X, C, labels=lab, mindist=md))
+    sort_inverse = timed(lambda: km.update(X, lab, C))
+    scatter = timed(lambda: km.update_scatter(X, lab, C))
+    kp = -(-w.K // 256) * 256
+    bn_rows = (256 * 16) // (w.d * 2) * 16  # sorted positions per update CTA (fp16 rows)
+    ctas = -(-w.N // bn_rows) * w.B
+    assert km.device_fault() == 0
+    return {
+        "assign_fused_ms": round(fused, 4), "assign_dense_ms": round(dense, 4),
+        "dense_matrix_bytes_written_and_read": 2 * 4 * w.B * w.N * kp,
+        "update_sort_inverse_ms": round(sort_inverse, 4), "update_scatter_ms": round(scatter, 4),
+        "scatter_atomics": w.B * w.N * (w.d + 1),
+        "sort_inverse_vector_atomics_bound": 2 * ctas * (w.d * 2 // 16),
+        "note": "km_assign (prep + fused kernel) vs km_assign_dense (prep + scores to HBM + argmin pass); "
+                "km_update (sort + segmented update + finalize) vs km_update_scatter (atomics + finalize)",
+    }
+
+
 def run_ours(args, w):
     import numpy as np
     import torch
@@ -321,6 +361,9 @@ def run_ours(args, w):
                "d2h_bytes_per_step": int(lab_h.numel() * 4 + C_h.numel() * 4),
                "path": "km_lloyd(iters=1) on X in pinned host memory (chunked copies overlapped with the "
                        "kernels, labels written back to pinned host memory); C copied in and out"}
+    ablations = None
+    if not args.no_ablations and w.dtype == "f16":
+        ablations = run_ablations(w, X, C, labels, stream)
     clocks = sampler.stop()
 
     if rank != 0:
@@ -370,6 +413,7 @@ def run_ours(args, w):
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "ablations": ablations,
         "device_fault": fault,
     }
     print(json.dumps(out), flush=True)

@@ -29,6 +29,8 @@ SIGNATURES = {
     "km_device_fault": (_INT, [ctypes.POINTER(ctypes.c_int32), _P]),
     "km_assign_rescans": (_INT, [ctypes.POINTER(ctypes.c_int64), _P]),
     "km_assign_noalloc": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "km_assign_dense": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "km_update_scatter": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P, _P]),
     "km_assign_noalloc_limit": (ctypes.c_size_t, []),
     "km_trace_enable": (None, [_INT]),
     "km_trace_read": (_INT, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _INT]),
@@ -114,6 +116,36 @@ def assign(X, C, labels=None, mindist=None, stream=None):
     check("km_assign", lib().km_assign(_ptr(X), _ptr(C), B, N, K, d, _dtype_code(X), _ptr(labels), _ptr(mindist),
                                        _stream(stream)))
     return labels, mindist
+
+
+def assign_dense(X, C, labels=None, mindist=None, stream=None):
+    """Baseline: the assignment with the N x K score matrix materialised in HBM (same results as assign)."""
+    torch = _torch()
+    B, N, d = X.shape
+    K = C.shape[1]
+    _require(C, (B, K, d), torch.float32, "C")
+    if labels is None:
+        labels = torch.empty((B, N), dtype=torch.int32, device=X.device)
+    if mindist is None:
+        mindist = torch.empty((B, N), dtype=torch.float32, device=X.device)
+    check("km_assign_dense", lib().km_assign_dense(_ptr(X), _ptr(C), B, N, K, d, _dtype_code(X), _ptr(labels),
+                                                   _ptr(mindist), _stream(stream)))
+    return labels, mindist
+
+
+def update_scatter(X, labels, C_prev, stream=None):
+    """Baseline: the update with one atomic per point coordinate (same results as update)."""
+    torch = _torch()
+    B, N, d = X.shape
+    K = C_prev.shape[1]
+    _require(labels, (B, N), torch.int32, "labels")
+    _require(C_prev, (B, K, d), torch.float32, "C_prev")
+    C_out = C_prev.clone()
+    sums = torch.empty((B, K, d), dtype=torch.float32, device=X.device)
+    counts = torch.empty((B, K), dtype=torch.int32, device=X.device)
+    check("km_update_scatter", lib().km_update_scatter(_ptr(X), _ptr(labels), B, N, K, d, _dtype_code(X),
+                                                       _ptr(sums), _ptr(counts), _ptr(C_out), _stream(stream)))
+    return C_out, sums, counts
 
 
 def sort_labels(labels, K: int, stream=None):

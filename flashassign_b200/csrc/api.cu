@@ -556,6 +556,73 @@ km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, 
         "centroid finalize");
 }
 
+km_status km_assign_dense(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                          int32_t* labels, float* mindist, void* stream) {
+    g_err[0] = 0;
+    if (!X || !C || !labels) {
+        set_error("km_assign_dense: X, C and labels must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (dtype != KM_F16 || !assign_tc_supported(d, dtype)) {
+        set_error("km_assign_dense: fp16 points with 64 <= d <= 128 only (the tensor-core kernel's range)");
+        return KM_E_UNSUPPORTED;
+    }
+    if (!aligned(X, 16) || !aligned(C, 16) || !aligned(labels, 4) || (mindist && !aligned(mindist, 4))) {
+        set_error("km_assign_dense: X and C must be 16-byte aligned, labels and mindist 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    Scratch scratch(st);
+    TcScratch tcs;
+    float *dense = nullptr, *xnorm = nullptr;
+    KM_TRY(alloc_tc(scratch, dtype, B, K, d, 0, st, &tcs));
+    KM_TRY(scratch.get(&dense, (size_t)(B * N * padded_k(K)), "dense score matrix"));
+    KM_TRY(scratch.get(&xnorm, (size_t)(B * N), "point norms"));
+    {
+        PhaseScope ph(st, KM_PHASE_PREP, 1);
+        KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
+    }
+    PhaseScope ph(st, KM_PHASE_ASSIGN, 2);
+    KM_TRY(launched(launch_assign_tc_dense((const __half*)X, static_cast<const __half*>(tcs.prep.chat),
+                                           static_cast<const __half*>(tcs.prep.cext), B, N, K, d, dense, xnorm,
+                                           dev.sms, st),
+                    "dense scores (tensor cores)"));
+    return launched(launch_dense_argmin(dense, xnorm, B, N, K, labels, mindist, st), "argmin over the dense scores");
+}
+
+km_status km_update_scatter(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d,
+                            int dtype, float* sums, int32_t* counts, float* C_out, void* stream) {
+    g_err[0] = 0;
+    if (!X || !labels || !sums || !counts || !C_out) {
+        set_error("km_update_scatter: X, labels, sums, counts and C_out must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (!aligned(X, 16) || !aligned(sums, 16) || !aligned(C_out, 16) || !aligned(labels, 4) || !aligned(counts, 4)) {
+        set_error("km_update_scatter: X, sums and C_out must be 16-byte aligned, labels and counts 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    {
+        PhaseScope ph(st, KM_PHASE_OTHER, 0);
+        KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * (size_t)(B * K * d), st), "zero sums"));
+        KM_TRY(launched(cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)(B * K), st), "zero counts"));
+    }
+    {
+        PhaseScope ph(st, KM_PHASE_UPDATE, 1);
+        KM_TRY(launched(launch_scatter_update(X, dtype, labels, B, N, K, d, sums, counts, st), "scatter update"));
+    }
+    PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
+    return launched(launch_finalize(sums, nullptr, B, K, d, C_out, dtype, PreparedC(), nullptr, false, nullptr,
+                                    nullptr, st, counts),
+                    "centroid finalize");
+}
+
 km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
                    int iters, int32_t* labels, float* C_out, float* objective, void* stream) {
     g_err[0] = 0;

@@ -106,9 +106,15 @@ struct Params {
     int32_t* labels;
     float* mindist;
     double* obj_acc;  // [B] running sum of minimum distances, nullable
+    float* dense;     // dense mode: [B, padded K, N] scores, written instead of reduced
+    float* xnorm;     // dense mode: [B, N] ||x||^2
     int32_t* fault;
 };
 
+// kDense (the dense-distance ablation): the same MMA pipeline, but every
+// tile's scores are written to P.dense and ||x||^2 to P.xnorm instead of
+// being reduced on chip -- the N x K matrix round trip that FlashAssign avoids.
+template <bool kDense>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
                      const __grid_constant__ CUtensorMap tmap_e, const Params P) {
@@ -306,31 +312,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
+                if constexpr (kDense) {
+                    const int upb = (int)P.units_per_batch;
+                    const int b = u / upb;
+                    const int n = (u - b * upb) * kUnitRows + (int)rank * kRows + row;
+                    if (n < P.N) {
+                        // [B, K', N]: a warp's 32 consecutive points of one column are one 128-byte line
+                        float* out = P.dense + ((int64_t)b * P.ktiles * kTileK + kt * kTileK + h * kPartCols) * P.N + n;
 #pragma unroll
-                for (int g = 0; g < kPartCols / 32; ++g) {
-                    const float* w = v + 32 * g;
-                    // two interleaved 3-input chains: few live temporaries
-                    float ga = max3(w[0], w[1], w[2]), gb = max3(w[3], w[4], w[5]);
-#pragma unroll
-                    for (int t = 6; t < 30; t += 4) {
-                        ga = max3(ga, w[t], w[t + 1]);
-                        gb = max3(gb, w[t + 2], w[t + 3]);
+                        for (int j = 0; j < kPartCols; ++j) out[(int64_t)j * P.N] = v[j];
                     }
-                    const float gmax = max3(max3(ga, w[30], w[31]), gb, gb);
-                    const bool better = gmax > best;  // strict: an earlier group keeps ties
-                    if (__any_sync(0xffffffffu, better)) {
-                        // the first column of the group holding its maximum
-                        int j0 = 31;
+                } else {
 #pragma unroll
-                        for (int j = 31; j >= 0; --j) j0 = (w[j] == gmax) ? j : j0;
-                        if (better) {
-                            best = gmax;
-                            label = kt * kTileK + h * kPartCols + g * 32 + j0;
-                        }
-                    }
+                  for (int g = 0; g < kPartCols / 32; ++g) {
+                      const float* w = v + 32 * g;
+                      // two interleaved 3-input chains: few live temporaries
+                      float ga = max3(w[0], w[1], w[2]), gb = max3(w[3], w[4], w[5]);
+#pragma unroll
+                      for (int t = 6; t < 30; t += 4) {
+                          ga = max3(ga, w[t], w[t + 1]);
+                          gb = max3(gb, w[t + 2], w[t + 3]);
+                      }
+                      const float gmax = max3(max3(ga, w[30], w[31]), gb, gb);
+                      const bool better = gmax > best;  // strict: an earlier group keeps ties
+                      if (__any_sync(0xffffffffu, better)) {
+                          // the first column of the group holding its maximum
+                          int j0 = 31;
+#pragma unroll
+                          for (int j = 31; j >= 0; --j) j0 = (w[j] == gmax) ? j : j0;
+                          if (better) {
+                              best = gmax;
+                              label = kt * kTileK + h * kPartCols + g * 32 + j0;
+                          }
+                      }
+                  }
                 }
             }
             if (!ok) break;
+            if constexpr (kDense) {
+                const int upb = (int)P.units_per_batch;
+                const int b = u / upb;
+                const int n = (u - b * upb) * kUnitRows + (int)rank * kRows + row;
+                if (h == 0 && n < P.N) P.xnorm[(int64_t)b * P.N + n] = xnorm;
+                continue;
+            }
             // join the column slices of each row (larger score, then lower
             // index) through a double-buffered shared slot with bounded handoffs
             const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
@@ -394,15 +419,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 bool assign_tc_supported(int64_t d, int dtype) { return dtype == KM_F16 && d >= 64 && d <= 128 && d % 8 == 0; }
 
-cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
-                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st) {
+template <bool kDense>
+cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
+                      int64_t d, int32_t* labels, float* mindist, double* obj_acc, float* dense, float* xnorm, int sms,
+                      cudaStream_t st) {
     if (!assign_tc_supported(d, KM_F16)) return cudaErrorNotSupported;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, 2, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mc, chat, 2, B, K, d, kBoxK, kHalfTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&me, cext, 2, B, padded_k(K), 16, 16, kHalfTile, CU_TENSOR_MAP_SWIZZLE_32B))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e =
+        cudaFuncSetAttribute(assign_tc_kernel<kDense>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     Params P;
     P.B = B; P.N = N; P.K = K; P.d = d;
@@ -414,9 +442,11 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* 
     P.labels = labels;
     P.mindist = mindist;
     P.obj_acc = obj_acc;
+    P.dense = dense;
+    P.xnorm = xnorm;
     P.fault = fault_word();
     // co-resident CTA pairs (a GPC with an odd number of free SMs cannot host a whole pair)
-    static int pair_cache[64] = {0};
+    static int pair_cache[64] = {0};  // per instantiation
     int dev = 0;
     cudaGetDevice(&dev);
     int max_pairs = (dev >= 0 && dev < 64) ? pair_cache[dev] : 0;
@@ -426,7 +456,7 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* 
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = kSmemBytes;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, (void*)assign_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&n, (void*)assign_tc_kernel<kDense>, &cfg) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = sms / 2;
         }
@@ -434,7 +464,18 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* 
         if (dev >= 0 && dev < 64) pair_cache[dev] = max_pairs;
     }
     P.pairs = P.units < max_pairs ? P.units : max_pairs;
-    return launch_kernel(assign_tc_kernel, dim3((unsigned)(2 * P.pairs)), dim3(kThreads), kSmemBytes, st, mx, mc, me, P);
+    return launch_kernel(assign_tc_kernel<kDense>, dim3((unsigned)(2 * P.pairs)), dim3(kThreads), kSmemBytes, st, mx,
+                         mc, me, P);
+}
+
+cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
+                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st) {
+    return launch_tc<false>(X, chat, cext, B, N, K, d, labels, mindist, obj_acc, nullptr, nullptr, sms, st);
+}
+
+cudaError_t launch_assign_tc_dense(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N,
+                                   int64_t K, int64_t d, float* dense, float* xnorm, int sms, cudaStream_t st) {
+    return launch_tc<true>(X, chat, cext, B, N, K, d, nullptr, nullptr, nullptr, dense, xnorm, sms, st);
 }
 
 }  // namespace km

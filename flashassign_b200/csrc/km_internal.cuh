@@ -136,6 +136,19 @@ cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted
                                int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
                                cudaStream_t st, bool accumulate = false);
 
+// ---- baselines the method replaces (measurement only, never on its path) ----
+// The dense-distance assignment: the tensor-core kernel's MMA pipeline writing
+// every score s = x.c - ||c||^2/2 to dense [B, padded_k(K), N] fp32 and ||x||^2
+// to xnorm [B, N]; then a separate pass takes each row's argmax.
+cudaError_t launch_assign_tc_dense(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N,
+                                   int64_t K, int64_t d, float* dense, float* xnorm, int sms, cudaStream_t st);
+cudaError_t launch_dense_argmin(const float* D, const float* xnorm, int64_t B, int64_t N, int64_t K, int32_t* labels,
+                                float* mindist, cudaStream_t st);
+// The scatter-atomic update: sums and counts (zeroed by the caller) receive one
+// atomic addition per coordinate and one per point.
+cudaError_t launch_scatter_update(const void* X, int dtype, const int32_t* labels, int64_t B, int64_t N, int64_t K,
+                                  int64_t d, float* sums, int32_t* counts, cudaStream_t st);
+
 // counts[b][k] += offsets[b][k+1] - offsets[b][k] (chunked accumulation of cluster sizes).
 cudaError_t launch_add_counts(const int32_t* offsets, int64_t B, int64_t K, int32_t* counts, cudaStream_t st);
 

@@ -156,6 +156,33 @@ KM_API km_status km_assign_noalloc(const void* X, const float* C, int64_t B, int
                                    int dtype, int32_t* labels, float* mindist, void* stream);
 KM_API size_t km_assign_noalloc_limit(void);
 
+/*
+ * Baselines the method replaces, for measurement (papernotes.org page,
+ * 方法详解 and 关键设计 1-2: the standard implementations whose memory
+ * traffic and atomic contention Flash-KMeans removes).  Same results as
+ * km_assign and km_update, never used by km_lloyd.
+ *
+ * km_assign_dense: the distance matrix materialised.  The tensor-core
+ * assignment writes every score s = x.c - ||c||^2/2 to a [B, K', N] fp32
+ * scratch matrix in HBM (K' = K rounded up to 256; 4*B*N*K' bytes, taken with
+ * cudaMallocAsync: KM_E_NOMEM when it does not fit), then a second kernel
+ * reads it back and takes each point's argmax (lowest index among equal
+ * scores).  fp16 points with 64 <= d <= 128 only (else KM_E_UNSUPPORTED).
+ * Arguments as km_assign.
+ */
+KM_API km_status km_assign_dense(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                                 int32_t* labels, float* mindist, void* stream);
+
+/*
+ * km_update_scatter: the update with one atomic addition per point
+ * coordinate into its cluster's fp32 sum and one per point into its count
+ * (B*N*d + B*N atomics, contended on large clusters), then the same
+ * finalisation as km_update.  Arguments as km_update; labels must lie in
+ * [0, K) (others are skipped).
+ */
+KM_API km_status km_update_scatter(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d,
+                                   int dtype, float* sums, int32_t* counts, float* C_out, void* stream);
+
 /* Rows per chunk used by km_lloyd for host-resident X (0 restores the default, 2^23). */
 KM_API void km_set_chunk_rows(int64_t rows);
 

@@ -281,3 +281,43 @@ def test_injected_allocation_failure_is_reported_and_leaks_nothing(monkeypatch):
     assert abs(torch.cuda.mem_get_info()[0] - free0) < (64 << 20)
     km.lloyd(X, C, 1)  # still works
     torch.cuda.synchronize()
+
+
+# ---- the baselines the method replaces (measurement only) ----
+
+@pytest.mark.parametrize("B,N,K,d", [(2, 1000, 300, 128), (1, 129, 127, 64), (2, 257, 255, 96), (3, 511, 513, 128)])
+def test_dense_assign_baseline_matches_the_fused_kernel_and_the_oracle(B, N, K, d):
+    w = synth.small(B=B, N=N, d=d, K=K, dtype="f16", ncomp=max(1, K // 2), sigma=0.3, seed=2000 + N + K)
+    X = synth.points(w)
+    C = synth.init_centroids(w, X) if K <= N else np.random.default_rng(2).standard_normal((B, K, d)).astype(
+        np.float32)
+    lab_d, md_d = km.assign_dense(cuda(X), cuda(C))
+    lab_f, md_f = km.assign(cuda(X), cuda(C))
+    torch.cuda.synchronize()
+    assert km.device_fault() == 0
+    lab_d, md_d = lab_d.cpu().numpy(), md_d.cpu().numpy()
+    # the same scores from the same MMAs, reduced on chip or read back: identical results
+    assert np.array_equal(lab_d, lab_f.cpu().numpy())
+    assert np.array_equal(md_d, md_f.cpu().numpy())
+    check_labels(X, C, lab_d, md_d)
+
+
+def test_dense_assign_baseline_rejects_shapes_outside_the_tensor_core_range():
+    X = torch.zeros((1, 64, 16), dtype=torch.float16, device="cuda")
+    C = torch.zeros((1, 4, 16), dtype=torch.float32, device="cuda")
+    with pytest.raises(km.KMError) as e:
+        km.assign_dense(X, C)
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("B,N,K,d,dt", [(2, 3000, 100, 128, "f16"), (1, 4096, 8, 16, "f32"), (2, 2000, 500, 64, "f16")])
+def test_scatter_update_baseline_matches_the_oracle(B, N, K, d, dt):
+    w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=3000 + N + K)
+    X = synth.points(w)
+    C = synth.init_centroids(w, X)
+    lab, _ = run_assign(X, C)
+    C_s, sums_s, counts_s = km.update_scatter(cuda(X), cuda(lab), cuda(C))
+    C_u, sums_u, counts_u = km.update(cuda(X), cuda(lab), cuda(C))
+    torch.cuda.synchronize()
+    assert torch.equal(counts_s, counts_u)
+    check_centroids(X, lab, C, C_s.cpu().numpy(), counts_s.cpu().numpy())
