@@ -23,6 +23,7 @@ SIGNATURES = {
     "km_sort_labels": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P]),
     "km_update": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P, _P]),
     "km_lloyd": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _INT, _P, _P, _P, _P]),
+    "km_lloyd_tol": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _INT, ctypes.c_double, _P, _P, _P, _P, _P]),
     "km_set_chunk_rows": (None, [_I64]),
     "km_status_string": (ctypes.c_char_p, [_INT]),
     "km_last_error": (ctypes.c_char_p, []),
@@ -193,6 +194,27 @@ def lloyd(X, C_init, iters: int, labels=None, C_out=None, objective=None, stream
     check("km_lloyd", lib().km_lloyd(_ptr(X), _ptr(C_init), B, N, K, d, _dtype_code(X), iters, _ptr(labels),
                                      _ptr(C_out), _ptr(objective), _stream(stream)))
     return labels, C_out, objective
+
+
+def lloyd_tol(X, C_init, max_iters: int, tol: float, labels=None, C_out=None, objective=None, stream=None):
+    """Lloyd iterations until every batch's squared centroid shift is <= tol (or max_iters):
+    (labels, centroids, objective [max_iters, B] -- rows past the stop unwritten, iterations run)."""
+    torch = _torch()
+    B, N, d = X.shape
+    K = C_init.shape[1]
+    _require(C_init, (B, K, d), torch.float32, "C_init")
+    dev = C_init.device
+    if labels is None:
+        labels = torch.empty((B, N), dtype=torch.int32, device=dev)
+    if C_out is None:
+        C_out = torch.empty_like(C_init)
+    if objective is None:
+        objective = torch.full((max_iters, B), float("nan"), dtype=torch.float32, device=dev)
+    iters_run = torch.zeros(1, dtype=torch.int32, device=dev)
+    check("km_lloyd_tol", lib().km_lloyd_tol(_ptr(X), _ptr(C_init), B, N, K, d, _dtype_code(X), max_iters, float(tol),
+                                             _ptr(labels), _ptr(C_out), _ptr(objective), _ptr(iters_run),
+                                             _stream(stream)))
+    return labels, C_out, objective, iters_run
 
 
 def device_fault(stream=None) -> int:

@@ -208,12 +208,12 @@ km_status alloc_tc(Scratch& s, int dtype, int64_t B, int64_t K, int64_t d, int64
 // kernel, then the exact re-scan of the points it listed.
 km_status run_assign(const void* X, int dtype, const float* C, const TcScratch* tc, int64_t B, int64_t N, int64_t K,
                      int64_t d, int32_t* labels, float* mindist, double* obj_acc, const DeviceInfo& dev,
-                     cudaStream_t st) {
+                     cudaStream_t st, const int32_t* stop = nullptr) {
     if (tc && dtype == KM_F16) {
         PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
         return launched(launch_assign_tc((const __half*)X, static_cast<const __half*>(tc->prep.chat),
                                          static_cast<const __half*>(tc->prep.cext), B, N, K, d, labels, mindist,
-                                         obj_acc, dev.sms, st),
+                                         obj_acc, dev.sms, st, stop),
                         "assign (tensor cores)");
     }
     if (tc) {
@@ -221,15 +221,17 @@ km_status run_assign(const void* X, int dtype, const float* C, const TcScratch* 
         KM_TRY(launched(cudaMemsetAsync(tc->flag_count, 0, sizeof(int32_t) * (size_t)B, st), "zero re-scan counters"));
         KM_TRY(launched(launch_assign_tf32((const float*)X, static_cast<const float*>(tc->prep.chat),
                                            static_cast<const float*>(tc->prep.cext), tc->prep.cmax, B, N, K, d,
-                                           labels, mindist, obj_acc, tc->flag_count, tc->flag_rows, dev.sms, st),
+                                           labels, mindist, obj_acc, tc->flag_count, tc->flag_rows, dev.sms, st,
+                                           stop),
                         "assign (tf32 tensor cores)"));
         const int blocks = (int)std::max<int64_t>(1, 4 * (int64_t)dev.sms / B);
         return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st, tc->flag_rows,
-                                           tc->flag_count, blocks),
+                                           tc->flag_count, blocks, stop),
                         "assign (exact re-scan of listed points)");
     }
     PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
-    return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st),
+    return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st, nullptr, nullptr, 0,
+                                       stop),
                     "assign (CUDA cores)");
 }
 
@@ -391,6 +393,82 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
         }
     }  // scratch released on the stream
     return wait_stream(st, "km_lloyd (host-resident X)");
+}
+
+// Convergence control of the device-path iteration loop: after each
+// iteration the finalisation sums every batch's squared centroid shift on the
+// device, a one-block kernel counts the iteration into *iters_run and sets a
+// stop flag once every batch has shift <= tol, and every kernel of the later
+// iterations, already enqueued, reads the flag and returns at once -- no host
+// synchronisation per iteration.
+struct Converge {
+    double tol;
+    int32_t* iters_run;
+};
+
+// The device-path iteration loop of km_lloyd (cv == nullptr) and km_lloyd_tol.
+km_status lloyd_device(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, int dtype, int iters,
+                       int32_t* labels, float* C_out, float* objective, const DeviceInfo& dev, cudaStream_t st,
+                       const Converge* cv) {
+    const size_t ckd = (size_t)(B * K * d);
+    Scratch scratch(st);
+    const bool tc = uses_tc(dtype, d);
+    TcScratch tcs;
+    float* sums = nullptr;
+    double* obj_acc = nullptr;
+    int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
+    unsigned char* work = nullptr;
+    int32_t* stop = nullptr;
+    double* shift = nullptr;
+    if (tc) KM_TRY(alloc_tc(scratch, dtype, B, K, d, B * N, st, &tcs));
+    if (cv) {
+        KM_TRY(scratch.get(&stop, 1, "stop flag"));
+        KM_TRY(scratch.get(&shift, (size_t)B, "centroid shifts"));
+    }
+    if (objective) KM_TRY(scratch.get(&obj_acc, (size_t)B, "objective accumulator"));
+    KM_TRY(scratch.get(&sums, ckd, "cluster sums"));
+    KM_TRY(scratch.get(&offs, (size_t)(B * (K + 1)), "segment offsets"));
+    KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
+    KM_TRY(scratch.get(&sidx, (size_t)(B * N), "sorted indices"));
+    KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
+
+    if (tc) {
+        PhaseScope ph(st, KM_PHASE_PREP, 1);
+        KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
+    }
+    {
+        PhaseScope ph(st, KM_PHASE_OTHER, 0);
+        KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * ckd, st), "zero sums"));
+        if (obj_acc) KM_TRY(launched(cudaMemsetAsync(obj_acc, 0, sizeof(double) * B, st), "zero objective"));
+        if (cv) {
+            KM_TRY(launched(cudaMemsetAsync(stop, 0, sizeof(int32_t), st), "zero stop flag"));
+            KM_TRY(launched(cudaMemsetAsync(shift, 0, sizeof(double) * B, st), "zero shifts"));
+            KM_TRY(launched(cudaMemsetAsync(cv->iters_run, 0, sizeof(int32_t), st), "zero iteration count"));
+        }
+    }
+    const int sort_launches = sort_kernel_launches(N, K, false, false);
+    for (int t = 0; t < iters; ++t) {
+        KM_TRY(run_assign(X, dtype, C_out, tc ? &tcs : nullptr, B, N, K, d, labels, nullptr, obj_acc, dev, st, stop));
+        {
+            PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
+            KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, nullptr, work, st, false, stop),
+                            "label sort"));
+        }
+        {
+            PhaseScope ph(st, KM_PHASE_UPDATE, 1);
+            KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, offs, st, false, stop),
+                            "segmented update"));
+        }
+        const bool prep_next = tc && t + 1 < iters;
+        PhaseScope ph(st, KM_PHASE_FINALIZE, cv ? 2 : 1);
+        // the finalize zeroes the consumed sums, so the next update starts from 0
+        KM_TRY(launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, prep_next ? tcs.prep : PreparedC(),
+                                        nullptr, true, obj_acc,
+                                        objective ? objective + (size_t)t * B : nullptr, st, nullptr, stop, shift),
+                        "centroid finalize"));
+        if (cv) KM_TRY(launched(launch_converge_check(shift, B, cv->tol, stop, cv->iters_run, st), "convergence test"));
+    }
+    return KM_OK;
 }
 
 }  // namespace
@@ -668,52 +746,44 @@ km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t N, int
     if (iters == 0) return KM_OK;
     if (host_x) return lloyd_host(X, B, N, K, d, dtype, iters, labels, labels_on_host, C_out, objective, dev, st);
 
-    Scratch scratch(st);
-    const bool tc = uses_tc(dtype, d);
-    TcScratch tcs;
-    float* sums = nullptr;
-    double* obj_acc = nullptr;
-    int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
-    unsigned char* work = nullptr;
-    if (tc) KM_TRY(alloc_tc(scratch, dtype, B, K, d, B * N, st, &tcs));
-    if (objective) KM_TRY(scratch.get(&obj_acc, (size_t)B, "objective accumulator"));
-    KM_TRY(scratch.get(&sums, ckd, "cluster sums"));
-    KM_TRY(scratch.get(&offs, (size_t)(B * (K + 1)), "segment offsets"));
-    KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
-    KM_TRY(scratch.get(&sidx, (size_t)(B * N), "sorted indices"));
-    KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
+    return lloyd_device(X, B, N, K, d, dtype, iters, labels, C_out, objective, dev, st, nullptr);
+}
 
-    if (tc) {
-        PhaseScope ph(st, KM_PHASE_PREP, 1);
-        KM_TRY(launched(launch_prep_centroids(C_out, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
+km_status km_lloyd_tol(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                       int max_iters, double tol, int32_t* labels, float* C_out, float* objective, int32_t* iters_run,
+                       void* stream) {
+    g_err[0] = 0;
+    if (!X || !C_init || !labels || !C_out || !iters_run) {
+        set_error("km_lloyd_tol: X, C_init, labels, C_out and iters_run must be non-null");
+        return KM_E_INVALID;
     }
-    {
-        PhaseScope ph(st, KM_PHASE_OTHER, 0);
-        KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * ckd, st), "zero sums"));
-        if (obj_acc) KM_TRY(launched(cudaMemsetAsync(obj_acc, 0, sizeof(double) * B, st), "zero objective"));
+    if (max_iters < 1 || !(tol >= 0.0)) {
+        set_error("km_lloyd_tol: max_iters must be >= 1 and tol a number >= 0");
+        return KM_E_INVALID;
     }
-    const int sort_launches = sort_kernel_launches(N, K, false, false);
-    for (int t = 0; t < iters; ++t) {
-        KM_TRY(run_assign(X, dtype, C_out, tc ? &tcs : nullptr, B, N, K, d, labels, nullptr, obj_acc, dev, st));
-        {
-            PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
-            KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
-                            "label sort"));
-        }
-        {
-            PhaseScope ph(st, KM_PHASE_UPDATE, 1);
-            KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, offs, st),
-                            "segmented update"));
-        }
-        const bool prep_next = tc && t + 1 < iters;
-        PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
-        // the finalize zeroes the consumed sums, so the next update starts from 0
-        KM_TRY(launched(launch_finalize(sums, offs, B, K, d, C_out, dtype, prep_next ? tcs.prep : PreparedC(),
-                                        nullptr, true, obj_acc,
-                                        objective ? objective + (size_t)t * B : nullptr, st),
-                        "centroid finalize"));
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (!aligned(X, 16) || !aligned(C_init, 16) || !aligned(C_out, 16) || !aligned(labels, 4) ||
+        !aligned(iters_run, 4) || (objective && !aligned(objective, 4))) {
+        set_error("km_lloyd_tol: X, C_init and C_out must be 16-byte aligned, labels, iters_run and objective "
+                  "4-byte aligned");
+        return KM_E_UNSUPPORTED;
     }
-    return KM_OK;
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaPointerAttributes pa;
+    cudaError_t e = cudaPointerGetAttributes(&pa, X);
+    if (e != cudaSuccess) return cuda_error(e, "cudaPointerGetAttributes(X)");
+    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged) {
+        set_error("km_lloyd_tol: X must be device memory (host-resident X: use km_lloyd)");
+        return KM_E_UNSUPPORTED;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if (C_out != C_init)
+        KM_TRY(launched(cudaMemcpyAsync(C_out, C_init, sizeof(float) * (size_t)(B * K * d), cudaMemcpyDeviceToDevice,
+                                        st),
+                        "copy C_init"));
+    const Converge cv{tol, iters_run};
+    return lloyd_device(X, B, N, K, d, dtype, max_iters, labels, C_out, objective, dev, st, &cv);
 }
 
 void km_set_chunk_rows(int64_t rows) { g_chunk_rows.store(rows > 0 ? rows : 0); }

@@ -35,9 +35,11 @@ __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restri
                                                                const int32_t* __restrict__ list_count,
                                                                int32_t* __restrict__ labels,
                                                                float* __restrict__ mindist,
-                                                               double* __restrict__ obj_acc) {
+                                                               double* __restrict__ obj_acc,
+                                                               const int32_t* __restrict__ stop) {
     pdl_trigger();
     pdl_wait();
+    if (stop && *stop) return;
     __shared__ float xs[kThreads][kTileD + 1];
     __shared__ float cs[kTileK][kTileD + 1];
     __shared__ int64_t rows[kThreads];
@@ -109,15 +111,15 @@ __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restri
 
 cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
                                int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st, const int32_t* list,
-                               const int32_t* list_count, int max_blocks) {
+                               const int32_t* list_count, int max_blocks, const int32_t* stop) {
     int64_t gx = ceil_div(N, kThreads);
     if (list && max_blocks > 0 && gx > max_blocks) gx = max_blocks;
     const dim3 grid((unsigned)gx, (unsigned)B);
     if (dtype == KM_F16)
         return launch_kernel(assign_simt_kernel<__half>, grid, dim3(kThreads), 0, st, (const __half*)X, C, N, K, d,
-                             list, list_count, labels, mindist, obj_acc);
+                             list, list_count, labels, mindist, obj_acc, stop);
     return launch_kernel(assign_simt_kernel<float>, grid, dim3(kThreads), 0, st, (const float*)X, C, N, K, d, list,
-                         list_count, labels, mindist, obj_acc);
+                         list_count, labels, mindist, obj_acc, stop);
 }
 
 }  // namespace km

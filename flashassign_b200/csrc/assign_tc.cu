@@ -108,6 +108,7 @@ struct Params {
     double* obj_acc;  // [B] running sum of minimum distances, nullable
     float* dense;     // dense mode: [B, padded K, N] scores, written instead of reduced
     float* xnorm;     // dense mode: [B, N] ||x||^2
+    const int32_t* stop;  // nullable: when *stop, the launch does nothing
     int32_t* fault;
 };
 
@@ -179,6 +180,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // and the objective accumulator are written by it
     pdl_trigger();
     pdl_wait();
+    // a converged iteration loop has set the stop flag: no units (straight to the teardown)
+    const int64_t n_units = (P.stop && *P.stop) ? 0 : P.units;
 
     const int boxes = P.boxes;
     const uint32_t x_bytes_pair = (uint32_t)(2 * boxes * kBoxBytes);
@@ -191,7 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // tiles and their norm slices through the 4-stage ring.
         if (lane == 16) {
             uint32_t it_x = 0;
-            for (int64_t u = pair; u < P.units; u += P.pairs, ++it_x) {
+            for (int64_t u = pair; u < n_units; u += P.pairs, ++it_x) {
                 const int b = (int)(u / P.units_per_batch);
                 const int n0 = (int)((u % P.units_per_batch) * kUnitRows) + (int)rank * kRows;
                 const uint32_t xb = it_x % kXBufs;
@@ -204,7 +207,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         } else if (lane == 0) {
             uint32_t it_c = 0;
             bool ok = true;
-            for (int64_t u = pair; u < P.units && ok; u += P.pairs) {
+            for (int64_t u = pair; u < n_units && ok; u += P.pairs) {
                 const int b = (int)(u / P.units_per_batch);
                 for (int kt = 0; kt < P.ktiles; ++kt, ++it_c) {
                     const uint32_t cs = it_c % kCStages;
@@ -230,7 +233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (rank == 0 && lane == 0) {
             uint32_t it_x = 0, it_c = 0, it_a = 0;
             bool ok = true;
-            for (int64_t u = pair; u < P.units && ok; u += P.pairs, ++it_x) {
+            for (int64_t u = pair; u < n_units && ok; u += P.pairs, ++it_x) {
                 const uint32_t xb = it_x % kXBufs;
                 if (!(ok = mbar_wait(bar_x_full + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
                 const uint64_t a_desc0 = umma_desc_sw128(x_base + xb * kMaxBoxes * kBoxBytes);
@@ -269,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t acc_empty_leader0 = map_to_rank(bar_acc_empty, 0);
         uint32_t it_x = 0, it_a = 0;
         bool ok = true;
-        const int units = (int)P.units, pairs = (int)P.pairs;  // < 2^23: 32-bit counters
+        const int units = (int)n_units, pairs = (int)P.pairs;  // < 2^23: 32-bit counters
         for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
             const uint32_t xb = it_x % kXBufs;
             float xnorm = 0.f;
@@ -422,7 +425,7 @@ bool assign_tc_supported(int64_t d, int dtype) { return dtype == KM_F16 && d >= 
 template <bool kDense>
 cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
                       int64_t d, int32_t* labels, float* mindist, double* obj_acc, float* dense, float* xnorm, int sms,
-                      cudaStream_t st) {
+                      cudaStream_t st, const int32_t* stop) {
     if (!assign_tc_supported(d, KM_F16)) return cudaErrorNotSupported;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, 2, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -444,6 +447,7 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
     P.obj_acc = obj_acc;
     P.dense = dense;
     P.xnorm = xnorm;
+    P.stop = stop;
     P.fault = fault_word();
     // co-resident CTA pairs (a GPC with an odd number of free SMs cannot host a whole pair)
     static int pair_cache[64] = {0};  // per instantiation
@@ -469,13 +473,14 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
 }
 
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
-                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st) {
-    return launch_tc<false>(X, chat, cext, B, N, K, d, labels, mindist, obj_acc, nullptr, nullptr, sms, st);
+                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st,
+                             const int32_t* stop) {
+    return launch_tc<false>(X, chat, cext, B, N, K, d, labels, mindist, obj_acc, nullptr, nullptr, sms, st, stop);
 }
 
 cudaError_t launch_assign_tc_dense(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N,
                                    int64_t K, int64_t d, float* dense, float* xnorm, int sms, cudaStream_t st) {
-    return launch_tc<true>(X, chat, cext, B, N, K, d, nullptr, nullptr, nullptr, dense, xnorm, sms, st);
+    return launch_tc<true>(X, chat, cext, B, N, K, d, nullptr, nullptr, nullptr, dense, xnorm, sms, st, nullptr);
 }
 
 }  // namespace km

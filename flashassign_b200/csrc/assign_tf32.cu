@@ -145,6 +145,7 @@ struct Params {
     int32_t* flag_count;  // [B] points listed for the exact re-scan (zero on entry)
     int32_t* flag_rows;   // [B, N] their indices within the batch
     unsigned long long* rescans;  // running total of listed points (observability)
+    const int32_t* stop;  // nullable: when *stop, the launch does nothing
     int32_t* fault;
 };
 
@@ -210,6 +211,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // tiles, their norm bound and the flag counters are written by it
     pdl_trigger();
     pdl_wait();
+    // a converged iteration loop has set the stop flag: no units (straight to the teardown)
+    const int64_t n_units = (P.stop && *P.stop) ? 0 : P.units;
 
     const int boxes = P.boxes;
     const int dcols = (int)P.d;
@@ -220,7 +223,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 16) {
             // this CTA's X tiles, one unit at a time (the buffer is free once the unit's MMAs are done)
             uint32_t it_x = 0;
-            for (int64_t u = pair; u < P.units; u += P.pairs, ++it_x) {
+            for (int64_t u = pair; u < n_units; u += P.pairs, ++it_x) {
                 const int b = (int)(u / P.units_per_batch);
                 const int n0 = (int)((u % P.units_per_batch) * kUnitRows) + (int)rank * kRows;
                 if (!mbar_wait(bar_x_empty, (it_x & 1) ^ 1, abort_flag, P.fault)) break;
@@ -232,7 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // centroid chunks: head and tail boxes of 32 dimensions, the norm slice with the last
             uint32_t it_c = 0;
             bool ok = true;
-            for (int64_t u = pair; u < P.units && ok; u += P.pairs) {
+            for (int64_t u = pair; u < n_units && ok; u += P.pairs) {
                 const int b = (int)(u / P.units_per_batch);
                 for (int kt = 0; kt < P.ktiles && ok; ++kt) {
                     const int k0 = kt * kTileK + (int)rank * kHalfTile;
@@ -257,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (rank == 0 && lane == 0) {
             uint32_t it_x = 0, it_c = 0, it_a = 0;
             bool ok = true;
-            for (int64_t u = pair; u < P.units && ok; u += P.pairs, ++it_x) {
+            for (int64_t u = pair; u < n_units && ok; u += P.pairs, ++it_x) {
                 if (!(ok = mbar_wait_cluster(bar_x_split, it_x & 1, abort_flag, P.fault))) break;
                 tc_fence_after();
                 for (int kt = 0; kt < P.ktiles && ok; ++kt, ++it_a) {
@@ -302,7 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t x_split_leader = map_to_rank(bar_x_split, 0);
         uint32_t it_x = 0, it_a = 0;
         bool ok = true;
-        const int units = (int)P.units, pairs = (int)P.pairs;  // < 2^23: 32-bit counters
+        const int units = (int)n_units, pairs = (int)P.pairs;  // < 2^23: 32-bit counters
         for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
             // split this CTA's tile: head in place, tail to the second buffer; ||x||^2 on the way
             if (!(ok = mbar_wait(bar_x_full, it_x & 1, abort_flag, P.fault))) break;
@@ -429,7 +432,8 @@ bool assign_tf32_supported(int64_t d) { return d >= 32 && d <= 128 && d % 32 == 
 
 cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float* cext, const float* cmax, int64_t B,
                                int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
-                               int32_t* flag_count, int32_t* flag_rows, int sms, cudaStream_t st) {
+                               int32_t* flag_count, int32_t* flag_rows, int sms, cudaStream_t st,
+                               const int32_t* stop) {
     if (!assign_tf32_supported(d)) return cudaErrorNotSupported;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, 4, B, N, d, kBoxF, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -451,6 +455,7 @@ cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float*
     P.flag_count = flag_count;
     P.flag_rows = flag_rows;
     P.rescans = rescan_word();
+    P.stop = stop;
     P.fault = fault_word();
     // co-resident CTA pairs (a GPC with an odd number of free SMs cannot host a whole pair)
     static int pair_cache[64] = {0};

@@ -129,9 +129,11 @@ constexpr int kFinThreads = 256;
 __global__ void __launch_bounds__(kFinThreads) finalize_kernel(
     float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t K, int64_t Kp, int64_t d,
     float* __restrict__ C_out, int dtype, PreparedC next, int32_t* __restrict__ counts, int zero_sums,
-    double* __restrict__ obj_acc, float* __restrict__ obj_out, const int32_t* __restrict__ counts_in) {
+    double* __restrict__ obj_acc, float* __restrict__ obj_out, const int32_t* __restrict__ counts_in,
+    const int32_t* __restrict__ stop, double* __restrict__ shift) {
     pdl_trigger();
     pdl_wait();
+    if (stop && *stop) return;
     const int64_t b = blockIdx.y;
     const int sub = threadIdx.x % kFinLanes;
     const int64_t k = ((int64_t)blockIdx.x * kFinThreads + threadIdx.x) / kFinLanes;
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(
     if (valid && counts && sub == 0) counts[row] = n;
     const float inv = n > 0 ? 1.0f / (float)n : 0.f;  // the mean as s * (1/n): within 1 ulp of s / n
     const int64_t base = row * d;
-    double acc = 0.0;
+    double acc = 0.0, moved = 0.0;
     if (valid) {
         for (int64_t j = 4 * sub; j < d; j += 4 * kFinLanes) {
             // the sums are read whatever the count (zero for an empty cluster), so the
@@ -155,6 +157,12 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(
             float4 v;
             if (n > 0) {
                 v = make_float4(sv.x * inv, sv.y * inv, sv.z * inv, sv.w * inv);
+                if (shift) {  // this centroid's squared shift
+                    const float4 o = *reinterpret_cast<const float4*>(C_out + base + j);
+                    const double dx = (double)v.x - o.x, dy = (double)v.y - o.y, dz = (double)v.z - o.z,
+                                 dw = (double)v.w - o.w;
+                    moved += dx * dx + dy * dy + dz * dz + dw * dw;
+                }
                 *reinterpret_cast<float4*>(C_out + base + j) = v;
                 if (zero_sums) *reinterpret_cast<float4*>(sums + base + j) = make_float4(0.f, 0.f, 0.f, 0.f);
             } else {
@@ -181,6 +189,32 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(
 #pragma unroll
         for (int o = kFinLanes / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (valid && sub == 0) write_row_norm(next, dtype, b, b * Kp + k, acc);
+    }
+    if (shift) {  // the warp's four rows, one atomic
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) moved += __shfl_xor_sync(0xffffffffu, moved, o);
+        if ((threadIdx.x & 31) == 0 && moved != 0.0) atomicAdd(shift + b, moved);
+    }
+}
+
+// After an iteration: unless the loop has stopped, count the iteration and
+// stop it when every batch's centroid shift is within tol; reset the shifts.
+__global__ void converge_check_kernel(double* __restrict__ shift, int64_t B, double tol, int32_t* __restrict__ stop,
+                                      int32_t* __restrict__ iters_run) {
+    pdl_trigger();
+    pdl_wait();
+    __shared__ int all_in;
+    if (threadIdx.x == 0) all_in = 1;
+    __syncthreads();
+    const bool running = *stop == 0;
+    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+        if (!(shift[b] <= tol)) all_in = 0;  // benign race: every writer stores 0
+        shift[b] = 0.0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && running) {
+        *iters_run += 1;
+        if (all_in) *stop = 1;
     }
 }
 
@@ -212,10 +246,16 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
 
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
                             int dtype, PreparedC next, int32_t* counts, bool zero_sums, double* obj_acc,
-                            float* obj_out, cudaStream_t st, const int32_t* counts_in) {
+                            float* obj_out, cudaStream_t st, const int32_t* counts_in, const int32_t* stop,
+                            double* shift) {
     const dim3 grid((unsigned)ceil_div(K * kFinLanes, kFinThreads), (unsigned)B);
     return launch_kernel(finalize_kernel, grid, dim3(kFinThreads), 0, st, sums, offsets, K, padded_k(K), d, C_out, dtype,
-                         next, counts, zero_sums ? 1 : 0, obj_acc, obj_out, counts_in);
+                         next, counts, zero_sums ? 1 : 0, obj_acc, obj_out, counts_in, stop, shift);
+}
+
+cudaError_t launch_converge_check(double* shift, int64_t B, double tol, int32_t* stop, int32_t* iters_run,
+                                  cudaStream_t st) {
+    return launch_kernel(converge_check_kernel, dim3(1), dim3(256), 0, st, shift, B, tol, stop, iters_run);
 }
 
 }  // namespace km

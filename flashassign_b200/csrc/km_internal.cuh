@@ -91,16 +91,22 @@ cudaError_t launch_prep_centroids(const float* C, int64_t B, int64_t K, int64_t 
 // with zero_sums the sums are reset to 0 once consumed.
 // When obj_out is non-null, obj_out[b] = obj_acc[b] (as fp32) and obj_acc[b] = 0.
 // n_k is taken from counts_in when it is non-null, else from the offsets.
+// When shift is non-null, shift[b] += sum_k ||C_new[b][k] - C_old[b][k]||^2 (the
+// centroid shift of the iteration, for convergence tests).
+// Every launcher's `stop` (nullable): when *stop is set at run time, the
+// launch does nothing (a converged iteration loop, see launch_converge_check).
 cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int64_t K, int64_t d, float* C_out,
                             int dtype, PreparedC next, int32_t* counts, bool zero_sums, double* obj_acc,
-                            float* obj_out, cudaStream_t st, const int32_t* counts_in = nullptr);
+                            float* obj_out, cudaStream_t st, const int32_t* counts_in = nullptr,
+                            const int32_t* stop = nullptr, double* shift = nullptr);
 
 // Tensor-core assignment (fp16, 64 <= d <= 128).  Returns cudaErrorNotSupported
 // for shapes it does not take.
 bool assign_tc_supported(int64_t d, int dtype);
 // obj_acc (nullable, [B] double) accumulates the sum of minimum distances.
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
-                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st);
+                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st,
+                             const int32_t* stop = nullptr);
 
 // Tensor-core assignment of fp32 points (tf32 head/tail split, 32 <= d <= 128,
 // d % 32 == 0).  Points whose best two scores lie within the split's error
@@ -110,7 +116,8 @@ cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* 
 bool assign_tf32_supported(int64_t d);
 cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float* cext, const float* cmax, int64_t B,
                                int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
-                               int32_t* flag_count, int32_t* flag_rows, int sms, cudaStream_t st);
+                               int32_t* flag_count, int32_t* flag_rows, int sms, cudaStream_t st,
+                               const int32_t* stop = nullptr);
 
 // CUDA-core assignment for every supported shape: direct-difference
 // distances.  With `list`, only the list_count[b] points list[b * N + r] of
@@ -118,7 +125,7 @@ cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float*
 cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
                                int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st,
                                const int32_t* list = nullptr, const int32_t* list_count = nullptr,
-                               int max_blocks = 0);
+                               int max_blocks = 0, const int32_t* stop = nullptr);
 
 // Stable LSD radix argsort of labels in [0, K).  Scratch: sort_scratch_bytes().
 size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K);
@@ -127,14 +134,14 @@ int sort_kernel_launches(int64_t N, int64_t K, bool with_counts, bool bounds = t
 // (the update kernel writes them while it walks the sorted labels).
 cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* a_sorted,
                         int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st,
-                        bool bounds = true);
+                        bool bounds = true, const int32_t* stop = nullptr);
 
 // Segmented gather-reduce over the sorted order (sums must be zeroed first);
 // when offsets [B, K+1] is non-null it also writes the segment offsets.
 // With accumulate, the sums are added to (points streamed in chunks).
 cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
                                int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
-                               cudaStream_t st, bool accumulate = false);
+                               cudaStream_t st, bool accumulate = false, const int32_t* stop = nullptr);
 
 // ---- baselines the method replaces (measurement only, never on its path) ----
 // The dense-distance assignment: the tensor-core kernel's MMA pipeline writing
@@ -150,6 +157,11 @@ cudaError_t launch_scatter_update(const void* X, int dtype, const int32_t* label
                                   int64_t d, float* sums, int32_t* counts, cudaStream_t st);
 
 // counts[b][k] += offsets[b][k+1] - offsets[b][k] (chunked accumulation of cluster sizes).
+// Convergence test after an iteration's finalisation: unless *stop is already
+// set, ++*iters_run, and *stop = 1 when every batch's shift[b] <= tol; shift is
+// reset to 0.
+cudaError_t launch_converge_check(double* shift, int64_t B, double tol, int32_t* stop, int32_t* iters_run,
+                                  cudaStream_t st);
 cudaError_t launch_add_counts(const int32_t* offsets, int64_t B, int64_t K, int32_t* counts, cudaStream_t st);
 
 

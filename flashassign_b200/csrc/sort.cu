@@ -54,9 +54,11 @@ Plan make_plan(int64_t N, int64_t K) {
 bool small_hist(int bins, int64_t tiles) { return (int64_t)bins * tiles <= 8192; }
 
 __global__ void __launch_bounds__(kThreads) radix_hist_kernel(const int32_t* __restrict__ keys, int64_t N, int shift,
-                                                              int bits, int64_t T, int32_t* __restrict__ hist) {
+                                                              int bits, int64_t T, int32_t* __restrict__ hist,
+                                                              const int32_t* __restrict__ stop) {
     pdl_trigger();
     pdl_wait();
+    if (stop && *stop) return;
     __shared__ int s[256];
     const int64_t b = blockIdx.y, tile = blockIdx.x;
     const int bins = 1 << bits, mask = bins - 1;
@@ -73,9 +75,11 @@ __global__ void __launch_bounds__(kThreads) radix_hist_kernel(const int32_t* __r
 }
 
 // In-place exclusive scan of `len` ints per batch (one 1024-thread block per batch).
-__global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t* __restrict__ data, int64_t len) {
+__global__ void __launch_bounds__(1024) exclusive_scan_kernel(int32_t* __restrict__ data, int64_t len,
+                                                              const int32_t* __restrict__ stop) {
     pdl_trigger();
     pdl_wait();
+    if (stop && *stop) return;
     __shared__ int warp_tot[32];
     __shared__ int carry_s;
     int32_t* p = data + (int64_t)blockIdx.x * len;
@@ -118,9 +122,11 @@ __global__ void __launch_bounds__(kThreads) radix_scatter_kernel(const int32_t* 
                                                                  int32_t* __restrict__ vals_out, int64_t N, int shift,
                                                                  int bits, int64_t T,
                                                                  const int32_t* __restrict__ offs,
-                                                                 const int32_t* __restrict__ hist) {
+                                                                 const int32_t* __restrict__ hist,
+                                                                 const int32_t* __restrict__ stop) {
     pdl_trigger();
     pdl_wait();
+    if (stop && *stop) return;
     __shared__ int wh[kWarps][256];      // per-warp digit counts, then per-warp exclusive offsets
     __shared__ int gstart[256];          // global first position of each digit of this tile (hist path)
     __shared__ int tstart[256];          // first tile-local position of each digit
@@ -298,7 +304,7 @@ size_t sort_scratch_bytes(int64_t B, int64_t N, int64_t K) {
 
 cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* a_sorted,
                         int32_t* sorted_idx, int32_t* counts, int32_t* offsets, void* scratch, cudaStream_t st,
-                        bool bounds) {
+                        bool bounds, const int32_t* stop) {
     const Plan p = make_plan(N, K);
     int32_t* tmp_k = (int32_t*)scratch;
     int32_t* tmp_v = tmp_k + B * N;
@@ -315,17 +321,17 @@ cudaError_t launch_sort(const int32_t* labels, int64_t B, int64_t N, int64_t K, 
         int32_t* out_v = to_final ? sorted_idx : tmp_v;
         const int bins = 1 << p.bits[i];
         cudaError_t e = launch_kernel(radix_hist_kernel, grid, dim3(kThreads), 0, st, in_k, N, p.shift[i], p.bits[i],
-                                      p.tiles, hist);
+                                      p.tiles, hist, stop);
         if (e != cudaSuccess) return e;
         if (small_hist(bins, p.tiles)) {
             e = launch_kernel(radix_scatter_kernel, grid, dim3(kThreads), 0, st, in_k, in_v, out_k, out_v, N,
-                              p.shift[i], p.bits[i], p.tiles, (const int32_t*)nullptr, (const int32_t*)hist);
+                              p.shift[i], p.bits[i], p.tiles, (const int32_t*)nullptr, (const int32_t*)hist, stop);
         } else {
             e = launch_kernel(exclusive_scan_kernel, dim3((unsigned)B), dim3(1024), 0, st, hist,
-                              (int64_t)bins * p.tiles);
+                              (int64_t)bins * p.tiles, stop);
             if (e != cudaSuccess) return e;
             e = launch_kernel(radix_scatter_kernel, grid, dim3(kThreads), 0, st, in_k, in_v, out_k, out_v, N,
-                              p.shift[i], p.bits[i], p.tiles, (const int32_t*)hist, (const int32_t*)nullptr);
+                              p.shift[i], p.bits[i], p.tiles, (const int32_t*)hist, (const int32_t*)nullptr, stop);
         }
         if (e != cudaSuccess) return e;
         in_k = out_k;

@@ -62,9 +62,11 @@ template <typename T>
 __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, const int32_t* __restrict__ a_sorted,
                                                      const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
                                                      int64_t d, int tpr, int G, float* __restrict__ sums,
-                                                     int32_t* __restrict__ offsets, int accumulate) {
+                                                     int32_t* __restrict__ offsets, int accumulate,
+                                                     const int32_t* __restrict__ stop) {
     pdl_trigger();
     pdl_wait();
+    if (stop && *stop) return;
     constexpr int E = Chunk<T>::kElems;
     extern __shared__ __align__(16) unsigned char smem[];
     const int BN = G * kRowsPerLane;
@@ -207,7 +209,8 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
 
 template <typename T>
 cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sorted_idx, int64_t B, int64_t N,
-                     int64_t K, int64_t d, float* sums, int32_t* offsets, bool accumulate, cudaStream_t st) {
+                     int64_t K, int64_t d, float* sums, int32_t* offsets, bool accumulate, cudaStream_t st,
+                     const int32_t* stop) {
     const int tpr = (int)(d * (int64_t)sizeof(T) / 16);
     const int G = 256 / tpr;
     const int BN = G * kRowsPerLane;
@@ -218,16 +221,17 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
     }
     const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B);
     return launch_kernel(update_kernel<T>, grid, dim3(G * tpr), smem, st, (const T*)X, a_sorted, sorted_idx, N, K, d,
-                         tpr, G, sums, offsets, accumulate ? 1 : 0);
+                         tpr, G, sums, offsets, accumulate ? 1 : 0, stop);
 }
 
 }  // namespace
 
 cudaError_t launch_update_sums(const void* X, int dtype, const int32_t* a_sorted, const int32_t* sorted_idx,
                                int64_t B, int64_t N, int64_t K, int64_t d, float* sums, int32_t* offsets,
-                               cudaStream_t st, bool accumulate) {
-    if (dtype == KM_F16) return launch_t<__half>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, accumulate, st);
-    return launch_t<float>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, accumulate, st);
+                               cudaStream_t st, bool accumulate, const int32_t* stop) {
+    if (dtype == KM_F16)
+        return launch_t<__half>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, accumulate, st, stop);
+    return launch_t<float>(X, a_sorted, sorted_idx, B, N, K, d, sums, offsets, accumulate, st, stop);
 }
 
 }  // namespace km

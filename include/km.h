@@ -134,6 +134,31 @@ KM_API km_status km_lloyd(const void* X, const float* C_init, int64_t B, int64_t
                    int iters, int32_t* labels, float* C_out, float* objective, void* stream);
 
 /*
+ * km_lloyd until convergence (papernotes.org page, 整体框架 flowchart:
+ * iterate "until converged or the maximum number of iterations").  After each
+ * iteration the device sums, per batch, the squared shift of the centroids,
+ * shift_b = sum_k ||c_new - c_old||^2 (empty clusters do not move), and the
+ * loop stops once every batch has shift_b <= tol -- the decision is taken on
+ * the device: all max_iters iterations are enqueued at once and those after
+ * the stop return immediately (no host synchronisation per iteration).  All
+ * batches run the same number of iterations.  tol = 0 asks for an exact fixed
+ * point (no centroid moved); the update combines the partial sums of a
+ * cluster that spans several CTA runs with fp32 atomics, whose order can
+ * change the last bit from one iteration to the next, so a tol slightly above
+ * 0 is the robust way to ask for a settled state.
+ *   X        [B, N, d] dtype, device memory only (else KM_E_UNSUPPORTED).
+ *   iters_run int32, device, written: the number of iterations performed
+ *            (1..max_iters); labels, C_out and objective rows [0, iters_run)
+ *            are those of km_lloyd with iters = iters_run; later objective
+ *            rows are not written.
+ * Other arguments as km_lloyd.  max_iters >= 1 and tol >= 0 (else
+ * KM_E_INVALID).
+ */
+KM_API km_status km_lloyd_tol(const void* X, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d,
+                              int dtype, int max_iters, double tol, int32_t* labels, float* C_out, float* objective,
+                              int32_t* iters_run, void* stream);
+
+/*
  * km_assign without any device-memory allocation.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate --
  * e.g. a framework that has reserved the device's memory for its own pool,

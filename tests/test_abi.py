@@ -74,6 +74,11 @@ def test_update_and_sort_and_lloyd_reject_nulls():
     assert L.km_sort_labels(FAKE, 1, 10, 2, None, FAKE, None, None) == 1
     assert L.km_lloyd(FAKE, FAKE, 1, 10, 2, 16, 0, -1, FAKE, FAKE, None, None) == 1
     assert L.km_device_fault(None, None) == 1
+    assert L.km_lloyd_tol(FAKE, FAKE, 1, 10, 2, 16, 0, 5, 0.0, FAKE, FAKE, None, None, None) == 1
+    assert L.km_lloyd_tol(FAKE, FAKE, 1, 10, 2, 16, 0, 5, -1.0, FAKE, FAKE, None, FAKE, None) == 1
+    assert L.km_lloyd_tol(FAKE, FAKE, 1, 10, 2, 16, 0, 0, 0.0, FAKE, FAKE, None, FAKE, None) == 1
+    assert L.km_assign_dense(None, FAKE, 1, 10, 2, 64, 1, FAKE, None, None) == 1
+    assert L.km_update_scatter(FAKE, None, 1, 10, 2, 16, 0, FAKE, FAKE, FAKE, None) == 1
 
 
 def test_binding_raises_with_detail():

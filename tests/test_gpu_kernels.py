@@ -321,3 +321,68 @@ def test_scatter_update_baseline_matches_the_oracle(B, N, K, d, dt):
     torch.cuda.synchronize()
     assert torch.equal(counts_s, counts_u)
     check_centroids(X, lab, C, C_s.cpu().numpy(), counts_s.cpu().numpy())
+
+
+# ---- convergence-controlled iteration (device-side stop) ----
+
+def _shift(Ca, Cb):
+    return ((np.asarray(Ca, np.float64) - np.asarray(Cb, np.float64)) ** 2).sum(axis=(1, 2))
+
+
+@pytest.mark.parametrize("dt,d,K", [("f16", 128, 40), ("f32", 128, 40), ("f32", 16, 12)])
+def test_lloyd_tol_stops_when_the_centroids_settle_and_equals_plain_iterations(dt, d, K):
+    w = synth.small(B=3, N=3000, d=d, K=K, dtype=dt, ncomp=K, sigma=0.2, seed=4000 + d + K)
+    X = synth.points(w)
+    C0 = cuda(synth.init_centroids(w, X))
+    Xg = cuda(X)
+    tol = 1e-9  # above the last-bit wander of sums combined by atomics, far below any real move
+    lab, C, obj, n = km.lloyd_tol(Xg, C0, 60, tol)
+    torch.cuda.synchronize()
+    t = int(n.item())
+    assert 1 <= t < 60, f"not settled within 60 iterations ({t})"
+    lab_p, C_p, obj_p = km.lloyd(Xg, C0, t)
+    torch.cuda.synchronize()
+    # the same kernels in the same order as t plain iterations (up to the order of fp32 atomics)
+    assert (lab == lab_p).float().mean().item() > 0.9999
+    torch.testing.assert_close(C, C_p, rtol=1e-5, atol=1e-6)
+    torch.testing.assert_close(obj[:t], obj_p, rtol=1e-5, atol=0)
+    assert torch.isnan(obj[t:]).all()  # rows past the stop are not written
+    # the stop was earned: one more iteration moves the centroids by at most tol
+    _, C_next, _ = km.lloyd(Xg, C, 1)
+    torch.cuda.synchronize()
+    assert (_shift(C_next.cpu().numpy(), C.cpu().numpy()) <= 10 * tol).all()
+    assert km.device_fault() == 0
+
+
+def test_lloyd_tol_applies_the_shift_rule_and_the_iteration_cap():
+    w = synth.small(B=2, N=4000, d=64, K=60, dtype="f16", ncomp=60, sigma=0.3, seed=4101)
+    X = synth.points(w)
+    C0 = cuda(synth.init_centroids(w, X))
+    Xg = cuda(X)
+    runs = [km.lloyd(Xg, C0, t)[1].cpu().numpy() for t in range(1, 9)]  # C after t iterations
+    shifts = [_shift(runs[0], C0.cpu().numpy())] + [_shift(runs[t], runs[t - 1]) for t in range(1, 8)]
+    # a tolerance between two of the per-iteration shifts, away from either (the device sums in another order)
+    vals = sorted({float(s.max()) for s in shifts})
+    tol = 0.5 * (vals[len(vals) // 2 - 1] + vals[len(vals) // 2])
+    _, C, _, n = km.lloyd_tol(Xg, C0, 8, tol)
+    torch.cuda.synchronize()
+    t = int(n.item())
+    # stopped after the first iteration whose shift is within tol in every batch
+    first = next((i + 1 for i, s in enumerate(shifts) if (s <= tol).all()), 8)
+    assert t == first
+    assert np.array_equal(C.cpu().numpy(), runs[t - 1])
+    # the cap: two iterations at most
+    _, _, _, n2 = km.lloyd_tol(Xg, C0, 2, 0.0)
+    torch.cuda.synchronize()
+    assert int(n2.item()) == 2
+
+
+def test_lloyd_tol_rejects_bad_arguments():
+    X = torch.zeros((1, 256, 64), dtype=torch.float16, device="cuda")
+    C = torch.zeros((1, 4, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(km.KMError) as e:
+        km.lloyd_tol(X, C, 5, -1.0)
+    assert e.value.status == 1
+    with pytest.raises(km.KMError) as e:
+        km.lloyd_tol(X.cpu().pin_memory(), C, 5, 0.0)
+    assert e.value.status == 2
