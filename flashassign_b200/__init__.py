@@ -25,6 +25,7 @@ SIGNATURES = {
     "km_lloyd": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _INT, _P, _P, _P, _P]),
     "km_lloyd_tol": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _INT, ctypes.c_double, _P, _P, _P, _P, _P]),
     "km_set_chunk_rows": (None, [_I64]),
+    "km_release_cached": (_INT, []),
     "km_status_string": (ctypes.c_char_p, [_INT]),
     "km_last_error": (ctypes.c_char_p, []),
     "km_device_fault": (_INT, [ctypes.POINTER(ctypes.c_int32), _P]),

@@ -27,7 +27,40 @@ bool inject(const char* what) {
     return f && std::strcmp(f, what) == 0;
 }
 
-// Scratch taken stream-ordered on one stream, released on scope exit.
+// The library's stream-ordered memory pool on the current device, created on
+// first use.  Unlike the device's default pool it keeps the memory freed into
+// it (release threshold: unlimited), so a call does not map and unmap its
+// scratch every time; km_release_cached() returns it to the device.
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[64] = {nullptr};
+
+cudaError_t scratch_pool(cudaMemPool_t* out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    if (!g_pool[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess) return e;
+        uint64_t keep = ~uint64_t(0);
+        if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return e;
+        }
+        g_pool[dev] = pool;
+    }
+    *out = g_pool[dev];
+    return cudaSuccess;
+}
+
+// Scratch taken stream-ordered from the library's pool on one stream, released
+// (to the pool) on scope exit.
 class Scratch {
   public:
     explicit Scratch(cudaStream_t st) : st_(st) {}
@@ -39,7 +72,9 @@ class Scratch {
         *out = nullptr;
         if (count == 0) return KM_OK;
         void* p = nullptr;
-        cudaError_t e = inject("alloc") ? cudaErrorMemoryAllocation : cudaMallocAsync(&p, count * sizeof(T), st_);
+        cudaMemPool_t pool = nullptr;
+        cudaError_t e = inject("alloc") ? cudaErrorMemoryAllocation : scratch_pool(&pool);
+        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&p, count * sizeof(T), pool, st_);
         if (e != cudaSuccess) {
             cudaGetLastError();
             set_error("scratch allocation of %zu bytes for %s failed: %s", count * sizeof(T), what,
@@ -784,6 +819,17 @@ km_status km_lloyd_tol(const void* X, const float* C_init, int64_t B, int64_t N,
                         "copy C_init"));
     const Converge cv{tol, iters_run};
     return lloyd_device(X, B, N, K, d, dtype, max_iters, labels, C_out, objective, dev, st, &cv);
+}
+
+km_status km_release_cached(void) {
+    g_err[0] = 0;
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    for (int dev = 0; dev < 64; ++dev) {
+        if (!g_pool[dev]) continue;
+        cudaError_t e = cudaMemPoolTrimTo(g_pool[dev], 0);
+        if (e != cudaSuccess) return cuda_error(e, "cudaMemPoolTrimTo");
+    }
+    return KM_OK;
 }
 
 void km_set_chunk_rows(int64_t rows) { g_chunk_rows.store(rows > 0 ? rows : 0); }

@@ -17,9 +17,10 @@
  *   - The B problems are independent; each has its own K centroids.
  *   - Pointers are device pointers unless stated otherwise; the caller owns
  *     (allocates and frees) every array it passes.  Scratch memory is taken
- *     stream-ordered (cudaMallocAsync) on `stream` and released before return
- *     on the same stream.  No state survives a call except a per-device cache
- *     of the capability check.
+ *     stream-ordered from the library's memory pool on `stream` and released
+ *     to it before return on the same stream (see km_release_cached).  No
+ *     other state survives a call except a per-device cache of the capability
+ *     check.
  *   - `stream` is a cudaStream_t (NULL means the legacy default stream).
  *     Every call is asynchronous on it: results are ready once the stream is
  *     synchronised.  Argument errors return before any work is enqueued.
@@ -207,6 +208,16 @@ KM_API km_status km_assign_dense(const void* X, const float* C, int64_t B, int64
  */
 KM_API km_status km_update_scatter(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d,
                                    int dtype, float* sums, int32_t* counts, float* C_out, void* stream);
+
+/*
+ * Scratch memory comes from a stream-ordered memory pool of the library's own
+ * (one per device, created on first use) that keeps what its calls free, so
+ * repeated calls do not map and unmap device memory each time.  This returns
+ * the pools' unused memory to the devices (memory still in use by enqueued
+ * work is kept).  The pools hold at most the largest scratch of any one call
+ * per stream in flight.
+ */
+KM_API km_status km_release_cached(void);
 
 /* Rows per chunk used by km_lloyd for host-resident X (0 restores the default, 2^23). */
 KM_API void km_set_chunk_rows(int64_t rows);

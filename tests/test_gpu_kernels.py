@@ -386,3 +386,18 @@ def test_lloyd_tol_rejects_bad_arguments():
     with pytest.raises(km.KMError) as e:
         km.lloyd_tol(X.cpu().pin_memory(), C, 5, 0.0)
     assert e.value.status == 2
+
+
+def test_scratch_pool_keeps_memory_until_released():
+    # the dense baseline takes a 256 MiB score matrix as scratch; the library's pool keeps it after the call
+    w = synth.small(B=1, N=65536, d=128, K=1024, dtype="f16", seed=25)
+    X = cuda(synth.points(w))
+    C = cuda(synth.init_centroids(w, X.cpu().numpy()))
+    km.assign_dense(X, C)
+    torch.cuda.synchronize()
+    held = torch.cuda.mem_get_info()[0]
+    km.assign_dense(X, C)  # served from the pool: no new device memory
+    torch.cuda.synchronize()
+    assert abs(torch.cuda.mem_get_info()[0] - held) < (32 << 20)
+    km.check("km_release_cached", km.lib().km_release_cached())
+    assert torch.cuda.mem_get_info()[0] - held > (200 << 20)
