@@ -25,22 +25,29 @@
 //   * Persistent grid of pairs; a work unit is 256 consecutive points of one
 //     batch; units are strided over the pairs so that pairs running at the
 //     same time share their batch's centroids in L2.
-//   * Warp roles per CTA: warp 0 issues TMA loads (one thread: X tiles of the
-//     units into two buffers; another: centroid tiles plus their norm slices
-//     into a 4-stage ring), completing on the leader CTA's barriers; warp 1
-//     allocates TMEM for the pair; in the leader CTA, warps 1 and 10 issue
-//     the MMAs (alternate tiles: one thread issues at most ~1 MMA per 100
-//     cycles) and commit them to both CTAs' barriers; warps 2..9 are the
-//     epilogue: TMEM lane = point row, two warps per row split each tile's
-//     256 columns in 128-column slices, read in one 128-column TMEM load; the
-//     accumulator is released as soon as they are in registers.
+//   * Warp roles per CTA (12 warps): warp 0 issues TMA loads (one thread:
+//     X tiles of the units into three buffers; another: centroid tiles plus
+//     their norm slices into a 3-stage ring), completing on the leader CTA's
+//     barriers; warp 1 allocates TMEM for the pair; in the leader CTA, warps
+//     1 and 10 issue the MMAs (alternate tiles) and commit them to both CTAs'
+//     barriers; warps 2..9 are the epilogue: TMEM lane = point row, two warps
+//     per row split each tile's 256 columns in 128-column slices, read in one
+//     128-column TMEM load, the accumulator released as soon as they are in
+//     registers; warp 11 finishes each unit (below), so that nothing but tile
+//     work sits between two accumulator releases of the epilogue warps.
 //   * Epilogue: per 32-column group, the group maximum (3-input max) is
 //     compared with the running best; only when it improves (in any lane of
 //     the warp) is the group scanned for its first column equal to the
-//     maximum, which becomes the running label.  The
-//     two column slices of a row are joined in shared memory (larger score,
-//     then lower index).  mindist = ||x||^2 - 2 * best, ||x||^2 summed from
-//     the staged X tile.
+//     maximum, which becomes the running label.  At the end of a unit each
+//     epilogue warp posts its (score, label) to a double-buffered shared slot.
+//   * Unit finish (warp 11): ||x||^2 of each row summed from the staged X
+//     tile (then the X buffer is released), the two column slices joined
+//     (larger score, then lower index), labels, mindist = ||x||^2 - 2 * best,
+//     and the objective (one atomic per unit).
+//   * Measured on B200: at the 1 kW power cap the SM clock settles near
+//     1.4 GHz (K = 4096) to 1.7 GHz (K = 1024) and a tile costs ~1.1 us of
+//     wall time either way: the kernel runs at the power limit, so fewer
+//     cycles per tile buy a lower clock rather than time.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records a fault code in the device fault word, stops issuing work, frees
 // its TMEM and returns.
@@ -56,16 +63,17 @@ constexpr int kTileK = kAssignTileK;            // centroids per K tile (MMA N) 
 constexpr int kHalfTile = kTileK / 2;           // centroids staged per CTA per tile (128)
 constexpr int kBoxK = 64;                       // fp16 elements per 128-byte swizzle row
 constexpr int kMaxBoxes = 2;                    // d <= 128
-constexpr int kCStages = 4;
-constexpr int kXBufs = 2;
+constexpr int kCStages = 3;
+constexpr int kXBufs = 3;
 constexpr int kAccSets = 2;                     // 2 x 256 TMEM columns
 constexpr int kBoxBytes = 128 * 128;            // X: [128 rows x 64 fp16], 128-byte swizzled
 constexpr int kCBoxBytes = kHalfTile * 128;     // C: [128 centroids x 64 fp16], 128-byte swizzled
 constexpr int kExtBytes = 128 * 32;             // ones: [128 rows x 16 fp16], 32-byte swizzled
 constexpr int kCExtBytes = kHalfTile * 32;      // norm slice: [128 centroids x 16 fp16], 32-byte swizzled
-constexpr int kThreads = 352;                   // 11 warps: producers, MMA issuer A, 8 epilogue, MMA issuer B
+constexpr int kThreads = 384;                   // 12 warps: producers, MMA issuer A, 8 epilogue, issuer B, merge
 constexpr int kEpiWarp0 = 2;
 constexpr int kMmaWarpB = 10;                   // second issuer, on another SMSP than warp 1
+constexpr int kMergeWarp = 11;                  // joins the halves, ||x||^2, outputs (warps go in fours: no extra registers)
 constexpr int kEpiWarps = 8;                    // at most 3 warps per SMSP: up to 168 registers each
 constexpr int kColParts = kEpiWarps / 4;        // warps per TMEM lane quarter, each with a column slice
 constexpr int kPartCols = kTileK / kColParts;   // 128 columns of each tile per epilogue warp
@@ -78,8 +86,8 @@ constexpr int kCOff = kXOff + kXBytes;
 constexpr int kCStageBytes = kMaxBoxes * kCBoxBytes + kCExtBytes;  // 36 KB: centroid boxes + norm slice
 constexpr int kCBytes = kCStages * kCStageBytes;                    // 144 KB
 constexpr int kAOnesOff = kCOff + kCBytes;                          // 4 KB of ones (the points' extra slice)
-constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 1 part x 128 rows x (score, label)
-constexpr int kMergeBytes = 2 * (kColParts - 1) * kRows * 8;
+constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 2 halves x 128 rows x (score, label)
+constexpr int kMergeBytes = 2 * kColParts * kRows * 8;
 constexpr int kBarOff = kMergeOff + kMergeBytes;
 constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 4;  // + merge handoff (2 slots x full/empty)
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;      // + tmem slot, flag, alignment slack
@@ -133,8 +141,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t bar_m_full = bar_acc_empty + 8 * kAccSets, bar_m_empty = bar_m_full + 16;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + kNumBars * 8 + 4);
-    float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                 // [2][parts-1][128]
-    int* merge_label = reinterpret_cast<int*>(smem + kMergeOff + kMergeBytes / 2);  // [2][parts-1][128]
+    float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                 // [2][parts][128]
+    int* merge_label = reinterpret_cast<int*>(smem + kMergeOff + kMergeBytes / 2);  // [2][parts][128]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cta_rank();         // 0: leader CTA of the pair (issues the MMAs)
@@ -143,7 +151,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kXBufs; ++i) {
             mbar_init(bar_x_full + 8 * i, 1);               // leader: its expect_tx; bytes from both CTAs
-            mbar_init(bar_x_empty + 8 * i, 2 + kEpiWarps);  // both issuers' end-of-unit commits + local epilogue warps
+            mbar_init(bar_x_empty + 8 * i, 3);              // both issuers' end-of-unit commits + the merge warp
         }
         for (int i = 0; i < kCStages; ++i) {
             mbar_init(bar_c_full + 8 * i, 1);
@@ -154,8 +162,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(bar_acc_empty + 8 * i, 2 * kEpiWarps);  // leader: epilogue warps of both CTAs
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(bar_m_full + 8 * i, kEpiWarps - 4);  // the warps of column slices 1..3
-            mbar_init(bar_m_empty + 8 * i, 4);             // the warps of column slice 0
+            mbar_init(bar_m_full + 8 * i, kEpiWarps);      // every epilogue warp has posted its half
+            mbar_init(bar_m_empty + 8 * i, 1);             // the merge warp has read the slot
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -265,6 +273,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
         // ------------------------------ epilogue (both CTAs) ------------------------------
+        // Per tile: read this warp's 128 columns, hand the accumulator back,
+        // reduce.  Per unit only the (score, label) of this half is posted to
+        // the merge warp, so nothing but tile work sits between two releases.
         const int e = warp - kEpiWarp0;
         const int q = warp % 4;   // TMEM lane quarter this warp may access
         const int h = e / 4;      // which 128-column slice of each 256-column tile
@@ -274,8 +285,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         bool ok = true;
         const int units = (int)n_units, pairs = (int)P.pairs;  // < 2^23: 32-bit counters
         for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
-            const uint32_t xb = it_x % kXBufs;
-            float xnorm = 0.f;
             float best = -INFINITY;
             int label = -1;    // column of the running best
             for (int kt = 0; kt < P.ktiles; ++kt, ++it_a) {
@@ -284,30 +293,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 __syncwarp();  // tcgen05.ld below is warp-collective
                 tc_fence_after();
                 const uint32_t tcol = tmem_base + ((uint32_t)(q * 32) << 16) + s * kTileK + h * kPartCols;
-                if (kt == 0) {
-                    // The MMA has consumed this unit's X tile, so it is in place.
-                    // ||x||^2 from it: the swizzle permutes 16-byte chunks within a
-                    // 128-byte row, so each row's bytes are all in that row.
-                    if (h == 0) {
-                        for (int kb = 0; kb < boxes; ++kb) {
-                            const uint4* rowp =
-                                reinterpret_cast<const uint4*>(smem + kXOff + (xb * kMaxBoxes + kb) * kBoxBytes + row * 128);
-#pragma unroll
-                            for (int cch = 0; cch < 8; ++cch) {
-                                const uint4 xv = rowp[(cch + lane) & 7];  // lanes start on different banks
-                                const __half2* hh = reinterpret_cast<const __half2*>(&xv);
-#pragma unroll
-                                for (int t = 0; t < 4; ++t) {
-                                    const float2 f = __half22float2(hh[t]);
-                                    xnorm = fmaf(f.x, f.x, xnorm);
-                                    xnorm = fmaf(f.y, f.y, xnorm);
-                                }
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
-                }
                 // this warp's 128 columns in one load; the accumulator is handed
                 // back as soon as they are in registers, before their arithmetic
                 float v[kPartCols];
@@ -352,54 +337,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) break;
-            if constexpr (kDense) {
-                const int upb = (int)P.units_per_batch;
-                const int b = u / upb;
-                const int n = (u - b * upb) * kUnitRows + (int)rank * kRows + row;
-                if (h == 0 && n < P.N) P.xnorm[(int64_t)b * P.N + n] = xnorm;
-                continue;
-            }
-            // join the column slices of each row (larger score, then lower
-            // index) through a double-buffered shared slot with bounded handoffs
+            // post this half's result (the dense mode posts only the arrival)
             const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
-            if (h > 0) {
-                if (!(ok = mbar_wait(bar_m_empty + 8 * ms, mph ^ 1, abort_flag, P.fault))) break;
-                const int slot = ((int)ms * (kColParts - 1) + (h - 1)) * kRows + row;
+            if (!(ok = mbar_wait(bar_m_empty + 8 * ms, mph ^ 1, abort_flag, P.fault))) break;
+            if constexpr (!kDense) {
+                const int slot = ((int)ms * kColParts + h) * kRows + row;
                 merge_score[slot] = best;
                 merge_label[slot] = label;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_m_full + 8 * ms);
-            } else {
-                if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
-                float fb = best;
-                int fl = label;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_m_full + 8 * ms);
+        }
+    } else if (warp == kMergeWarp) {
+        // ------------------------------ merge warp (both CTAs) ------------------------------
+        // Once every epilogue warp has posted unit u (so its MMAs, done with
+        // the X tile, are complete): ||x||^2 of each row from the staged tile
+        // (the swizzle permutes 16-byte chunks within a 128-byte row, so each
+        // row's bytes are all in that row), the X buffer released, the two
+        // column halves joined (larger score, then the lower index; half 0
+        // holds the lower columns), the labels, mindist and the objective.
+        uint32_t it_x = 0;
+        bool ok = true;
+        const int units = (int)n_units, pairs = (int)P.pairs;
+        const int upb = (int)P.units_per_batch;
+        for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
+            const uint32_t xb = it_x % kXBufs;
+            const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
+            if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
+            const int b = u / upb;
+            const int n0 = (u - b * upb) * kUnitRows + (int)rank * kRows;
+            double obj = 0.0;
+            for (int rq = 0; rq < kRows / 32; ++rq) {
+                const int r = rq * 32 + lane;
+                float xnorm = 0.f;
+                for (int kb = 0; kb < boxes; ++kb) {
+                    const uint4* rowp =
+                        reinterpret_cast<const uint4*>(smem + kXOff + (xb * kMaxBoxes + kb) * kBoxBytes + r * 128);
 #pragma unroll
-                for (int part = 0; part < kColParts - 1; ++part) {
-                    const int slot = ((int)ms * (kColParts - 1) + part) * kRows + row;
-                    const float ob = merge_score[slot];
-                    const int ol = merge_label[slot];
-                    if (ob > fb || (ob == fb && ol >= 0 && (fl < 0 || ol < fl))) {
-                        fb = ob;
-                        fl = ol;
+                    for (int cch = 0; cch < 8; ++cch) {
+                        const uint4 xv = rowp[(cch + lane) & 7];  // lanes start on different banks
+                        const __half2* hh = reinterpret_cast<const __half2*>(&xv);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const float2 f = __half22float2(hh[t]);
+                            xnorm = fmaf(f.x, f.x, xnorm);
+                            xnorm = fmaf(f.y, f.y, xnorm);
+                        }
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
-                const int upb = (int)P.units_per_batch;
-                const int b = u / upb;
-                const int n = (u - b * upb) * kUnitRows + (int)rank * kRows + row;
-                const float md = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
-                if (n < P.N) {
-                    const int64_t o = (int64_t)b * P.N + n;
-                    P.labels[o] = fl;
-                    if (P.mindist) P.mindist[o] = md;
-                }
-                if (P.obj_acc) {  // the objective: this warp's 32 rows, one atomic per warp
-                    double part = n < P.N ? (double)md : 0.0;
+                const int n = n0 + r;
+                if constexpr (kDense) {
+                    if (n < P.N) P.xnorm[(int64_t)b * P.N + n] = xnorm;
+                } else {
+                    float fb = merge_score[((int)ms * kColParts) * kRows + r];
+                    int fl = merge_label[((int)ms * kColParts) * kRows + r];
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-                    if (lane == 0) atomicAdd(P.obj_acc + b, part);
+                    for (int part = 1; part < kColParts; ++part) {
+                        const int slot = ((int)ms * kColParts + part) * kRows + r;
+                        const float ob = merge_score[slot];
+                        const int ol = merge_label[slot];
+                        if (ob > fb || (ob == fb && ol >= 0 && (fl < 0 || ol < fl))) {
+                            fb = ob;
+                            fl = ol;
+                        }
+                    }
+                    const float md = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
+                    if (n < P.N) {
+                        const int64_t o = (int64_t)b * P.N + n;
+                        P.labels[o] = fl;
+                        if (P.mindist) P.mindist[o] = md;
+                        obj += (double)md;
+                    }
                 }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar_x_empty + 8 * xb);
+                mbar_arrive(bar_m_empty + 8 * ms);
+            }
+            if (!kDense && P.obj_acc) {  // the objective of the unit's 128 rows, one atomic
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) obj += __shfl_xor_sync(0xffffffffu, obj, o);
+                if (lane == 0) atomicAdd(P.obj_acc + b, obj);
             }
         }
     }
