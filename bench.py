@@ -380,8 +380,15 @@ def run_ours(args, w):
     t_other = phases["other"][0] / args.steps
     tflops = wk["flops_assign"] / (t_assign * 1e-3) / 1e12
     upd_gbs = wk["bytes_update"] / (t_update * 1e-3) / 1e9
-    peak_tf = peaks["bf16_tflops"]  # fp16 dense rate equals bf16; burst figure (short timed region)
+    # fp16 dense rate equals bf16.  The assignment is timed inside a long loop of back-to-back
+    # iterations that runs at the 1 kW power cap (sw_power_cap in the clock record; the SM clock
+    # settles near 1.4-1.7 GHz), so its denominator is the sustained GEMM figure; the burst figure
+    # is reported beside it.
+    peak_tf = peaks["bf16_tflops_sustained"]
+    peak_burst = peaks["bf16_tflops"]
     peak_bw = peaks["hbm_gbs"]
+    t_roof_burst = (max(wk["flops_assign"] / (peak_burst * 1e12), wk["bytes_assign"] / (peak_bw * 1e9)) +
+                    (wk["bytes_update"] + wk["bytes_sort"] + wk["bytes_finalize"]) / (peak_bw * 1e9)) * 1e3
     t_roof = (max(wk["flops_assign"] / (peak_tf * 1e12), wk["bytes_assign"] / (peak_bw * 1e9)) +
               (wk["bytes_update"] + wk["bytes_sort"] + wk["bytes_finalize"]) / (peak_bw * 1e9)) * 1e3
     launches = sum(c for _, c in phases.values())
@@ -400,13 +407,16 @@ def run_ours(args, w):
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(tflops / peak_tf, 4), "traffic": traffic_for(ASSIGN_TRAFFIC),
                      "kernel": "assign_tc_kernel",
-                     "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)",
+                     "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate equals bf16); the kernel runs "
+                                    f"inside a long power-capped loop",
+                     "frac_of_burst_peak": round(tflops / peak_burst, 4), "burst_peak": peak_burst,
                      "ms_per_launch": round(t_assign, 4)},
         "roofline_update": {"bound": "hbm", "achieved": round(upd_gbs, 1), "peak": peak_bw, "unit": "GB/s",
                             "frac": round(upd_gbs / peak_bw, 4), "kernel": "update_kernel",
                             "traffic": traffic_for(UPDATE_TRAFFIC),
                             "ms_per_launch": round(t_update, 4), "peak_source": peak_src},
-        "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4)},
+        "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4),
+                               "frac_with_burst_tensor_peak": round(t_roof_burst / ms_iter, 4)},
         "phases_ms_per_iter": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
         "traced_ms_per_iter": round(traced_ms_iter, 4),
         "gpu_launches": launches,
