@@ -44,6 +44,8 @@ def lockstep(w, iters, nsample):
         check_centroids(X, lab, C, C_next)
         C = C_next
     assert km.device_fault() == 0
+    print(f"{w.name}: {near} near-tie points (relative top-2 gap below the label tolerance) "
+          f"in {iters} iterations x {min(nsample, w.B * w.N)} checked rows")
     return X, C, near
 
 
@@ -85,6 +87,7 @@ def test_workload5_host_resident_fp32_chunked():
     C = synth.init_centroids(w, X)
     lab_h = torch.empty((w.B, w.N), dtype=torch.int32).pin_memory()
     km.lib().km_set_chunk_rows(w.chunk_rows)
+    km.assign_rescans()
     try:
         for t in range(2):
             t0 = time.perf_counter()
@@ -93,7 +96,9 @@ def test_workload5_host_resident_fp32_chunked():
             print(f"workload 5 iteration {t}: {time.perf_counter() - t0:.2f} s")
             lab = lab_h.numpy()
             C_next = C_next.cpu().numpy()
-            check_labels(X, C, lab, rows=sample_rows(w.B, w.N, 8192, seed=50 + t))
+            near = check_labels(X, C, lab, rows=sample_rows(w.B, w.N, 8192, seed=50 + t))
+            print(f"workload 5 iteration {t}: {near} near-tie points of 8192 checked rows, "
+                  f"{km.assign_rescans()} points re-scanned exactly")
             # argsort and counts over every point
             sidx, counts, offs = km.sort_labels(torch.from_numpy(lab).cuda(), w.K)
             check_sort(lab, w.K, sidx.cpu().numpy(), counts.cpu().numpy(), offs.cpu().numpy())
