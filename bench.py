@@ -34,13 +34,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captures summarised in profiles/assign_tc_kernel_b32_n65536_k1024_d128_f16.md and
 # profiles/update_kernel_b32_n65536_k1024_d128_f16.md, each valid only for the kernel source it was
 # taken on (sha1 of the .cu file); reported as null once that source changes.
-ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "3015919e48a9e44baf28be864699cba7d20ad824",
+ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "7e5a00a8cfdf487024aadac22ffd70cd463ccd10",
                             "tc_ptx.cuh": "ee9645b484e88174263ad58b26408994fd536d40",
-                            "km_internal.cuh": "475c6be450de2a4cc966941be94fbf1e05e59b0b"},
-                  "bytes": 546.350592e6 + 10.823680e6}
-UPDATE_TRAFFIC = {"files": {"update.cu": "c9054cceeb01068c671f1d62d9236f6ddc985079",
-                            "km_internal.cuh": "f0924f98116dbe93ff46af367ce72068d83b6d27"},
-                  "bytes": 557.689088e6 + 16.940288e6}
+                            "km_internal.cuh": "2c304a53203d0a8b6b4daae5b52fe75657c97a48"},
+                  "bytes": 546.353920e6 + 10.674432e6}
+UPDATE_TRAFFIC = {"files": {"update.cu": "e782d07783850ee11aed345f376d4c4a44fc6f24",
+                            "km_internal.cuh": "2c304a53203d0a8b6b4daae5b52fe75657c97a48"},
+                  "bytes": 557.689344e6 + 16.603648e6}
 
 
 def traffic_for(rec: dict):
@@ -63,6 +63,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", type=int, default=2, help="workload id (2 = the metric's configuration)")
+    p.add_argument("--n", type=int, default=0,
+                   help="points per problem instead of the workload's (a smaller case of it, e.g. for a profiler)")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-e2e", action="store_true")
@@ -401,9 +403,10 @@ def run_ours(args, w):
     out = {
         "metric": METRIC, "value": round(ms_iter, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_iter, 4), "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "global_problems": w.B * world,
-                   "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (X is 512 MiB)"},
+                   "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2 (X is {w.B * w.N * w.d * w.elem_bytes / 2**20:.0f} MiB)"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(tflops / peak_tf, 4), "traffic": traffic_for(ASSIGN_TRAFFIC),
                      "kernel": "assign_tc_kernel",
@@ -436,6 +439,8 @@ def main():
     args = parse()
     import synth
     w = synth.WORKLOADS[args.workload]
+    if args.n > 0:
+        w = w.with_(N=args.n, name=f"{w.name}_n{args.n}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)
