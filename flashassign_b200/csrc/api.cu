@@ -188,7 +188,8 @@ km_status launched(cudaError_t e, const char* what) {
     } while (0)
 
 bool uses_tc(int dtype, int64_t d) {
-    return dtype == KM_F16 ? assign_tc_supported(d, dtype) : assign_tf32_supported(d);
+    return dtype == KM_F16 ? (assign_tc_supported(d, dtype) || assign_wide_supported(d, dtype))
+                           : assign_tf32_supported(d);
 }
 
 // Scratch of a tensor-core assignment: the prepared centroids and, for fp32,
@@ -244,6 +245,13 @@ km_status alloc_tc(Scratch& s, int dtype, int64_t B, int64_t K, int64_t d, int64
 km_status run_assign(const void* X, int dtype, const float* C, const TcScratch* tc, int64_t B, int64_t N, int64_t K,
                      int64_t d, int32_t* labels, float* mindist, double* obj_acc, const DeviceInfo& dev,
                      cudaStream_t st, const int32_t* stop = nullptr) {
+    if (tc && dtype == KM_F16 && assign_wide_supported(d, dtype)) {
+        PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
+        return launched(launch_assign_wide((const __half*)X, static_cast<const __half*>(tc->prep.chat),
+                                           static_cast<const __half*>(tc->prep.cext), B, N, K, d, labels, mindist,
+                                           obj_acc, dev.sms, st, stop),
+                        "assign (tensor cores, d split in chunks)");
+    }
     if (tc && dtype == KM_F16) {
         PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
         return launched(launch_assign_tc((const __half*)X, static_cast<const __half*>(tc->prep.chat),

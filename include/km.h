@@ -68,6 +68,8 @@ typedef enum {
  * matrix is never written to memory.  The centroids are first rounded
  * (round-to-nearest-even) to `dtype`, and x.c is accumulated in fp32:
  *   - fp16, 64 <= d <= 128: on the tensor cores;
+ *   - fp16, d in {192, 256, ..., 512}: on the tensor cores, the centroids
+ *     streamed in 64-dimension chunks;
  *   - fp32, d in {32, 64, 96, 128}: on the tensor cores from tf32 head/tail
  *     splits of both operands (three products); a point whose best two scores
  *     lie within the split's error bound is re-scanned exactly on the CUDA

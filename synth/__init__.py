@@ -117,6 +117,9 @@ WORKLOADS = {
                 sigma=0.25, iters=5, seed=0x6B6D0004),
     5: Workload("b1_n134217728_d128_k4096_f32_host", 1, 1 << 27, 128, 4096, "f32", ncomp=4096,
                 sigma=0.3, iters=3, seed=0x6B6D0005, host=True, chunk_rows=1 << 23),
+    # wide points: the d = 512 shape of the papernotes.org page's end-to-end table (N = 1M, K = 65536)
+    6: Workload("b1_n1048576_d512_k65536_f16", 1, 1 << 20, 512, 65536, "f16", ncomp=65536,
+                sigma=0.25, iters=3, seed=0x6B6D0006),
 }
 
 

@@ -42,7 +42,12 @@ ASSIGN_SHAPES = [
     (2, 777, 257, 64, "f16"),
     (2, 600, 200, 96, "f16"),
     (2, 500, 100, 16, "f16"),    # below the tensor-core range: CUDA-core kernel
-    (2, 300, 50, 256, "f16"),    # above it
+    (2, 300, 50, 256, "f16"),    # wide points: centroids streamed in 64-dimension chunks
+    (1, 129, 127, 192, "f16"),
+    (2, 1000, 300, 512, "f16"),
+    (3, 257, 513, 320, "f16"),
+    (2, 500, 100, 448, "f16"),
+    (1, 200, 30, 136, "f16"),    # not a multiple of 64: CUDA-core kernel
     (1, 4096, 8, 16, "f32"),     # fp32 below the tf32 tensor-core range (d % 32 != 0): CUDA cores
     (2, 129, 33, 4, "f32"),
     (1, 1, 1, 32, "f32"),        # fp32 on tf32 tensor cores: d in {32, 64, 96, 128}
@@ -66,7 +71,7 @@ def test_assign_matches_oracle(B, N, K, d, dt):
     check_labels(X, C, lab, md)
 
 
-@pytest.mark.parametrize("dt,d", [("f16", 128), ("f32", 16), ("f32", 128)])
+@pytest.mark.parametrize("dt,d", [("f16", 128), ("f16", 256), ("f32", 16), ("f32", 128)])
 def test_assign_ties_go_to_the_lowest_index(dt, d):
     # integer coordinates and duplicate centroids give exact ties in every precision
     rng = np.random.default_rng(11)
@@ -196,7 +201,8 @@ def test_update_matches_oracle(B, N, K, d, dt, case):
 
 
 @pytest.mark.parametrize("B,N,K,d,dt", [(2, 3000, 50, 128, "f16"), (1, 4096, 8, 16, "f32"), (2, 1000, 300, 64, "f16"),
-                                        (2, 3000, 50, 128, "f32"), (1, 2000, 257, 32, "f32")])
+                                        (2, 3000, 50, 128, "f32"), (1, 2000, 257, 32, "f32"),
+                                        (1, 3000, 300, 512, "f16"), (2, 1000, 100, 256, "f16")])
 def test_lloyd_lockstep_with_oracle(B, N, K, d, dt):
     """Each iteration: the oracle takes the GPU's centroids and checks that iteration's labels and update."""
     w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=5 + K)

@@ -76,6 +76,12 @@ def test_workload4_large_k():
     lockstep(w, 2, nsample=384)
 
 
+def test_wide_points_d512_k65536():
+    # the d = 512 shape of the page's end-to-end table, on the chunked tensor-core path
+    w = synth.WORKLOADS[6]
+    lockstep(w, 1, nsample=256)
+
+
 def test_workload5_host_resident_fp32_chunked():
     """2^27 x 128 fp32 points (64 GiB) in pinned host memory, streamed in 2^23-row chunks."""
     import time
