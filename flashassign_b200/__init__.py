@@ -32,6 +32,8 @@ SIGNATURES = {
     "km_assign_rescans": (_INT, [ctypes.POINTER(ctypes.c_int64), _P]),
     "km_assign_noalloc": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
     "km_assign_dense": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "km_update_sums": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "km_finalize": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "km_update_scatter": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P, _P]),
     "km_assign_noalloc_limit": (ctypes.c_size_t, []),
     "km_trace_enable": (None, [_INT]),
@@ -176,6 +178,29 @@ def update(X, labels, C_prev, stream=None):
     check("km_update", lib().km_update(_ptr(X), _ptr(labels), B, N, K, d, _dtype_code(X), _ptr(sums), _ptr(counts),
                                        _ptr(C_out), _stream(stream)))
     return C_out, sums, counts
+
+
+def update_sums(X, labels, K: int, stream=None):
+    """The first half of the update: (sums [B,K,d] fp32, counts [B,K] int32); no centroid is written."""
+    torch = _torch()
+    B, N, d = X.shape
+    _require(labels, (B, N), torch.int32, "labels")
+    sums = torch.empty((B, K, d), dtype=torch.float32, device=X.device)
+    counts = torch.empty((B, K), dtype=torch.int32, device=X.device)
+    check("km_update_sums", lib().km_update_sums(_ptr(X), _ptr(labels), B, N, K, d, _dtype_code(X), _ptr(sums),
+                                                 _ptr(counts), _stream(stream)))
+    return sums, counts
+
+
+def finalize(sums, counts, C_prev, stream=None):
+    """The second half: sums / counts where counts > 0, else the previous centroid."""
+    torch = _torch()
+    B, K, d = C_prev.shape
+    _require(sums, (B, K, d), torch.float32, "sums")
+    _require(counts, (B, K), torch.int32, "counts")
+    C_out = C_prev.clone()
+    check("km_finalize", lib().km_finalize(_ptr(sums), _ptr(counts), B, K, d, _ptr(C_out), _stream(stream)))
+    return C_out
 
 
 def lloyd(X, C_init, iters: int, labels=None, C_out=None, objective=None, stream=None):

@@ -677,6 +677,64 @@ km_status km_update(const void* X, const int32_t* labels, int64_t B, int64_t N, 
         "centroid finalize");
 }
 
+km_status km_update_sums(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                         float* sums, int32_t* counts, void* stream) {
+    g_err[0] = 0;
+    if (!X || !labels || !sums || !counts) {
+        set_error("km_update_sums: X, labels, sums and counts must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (!aligned(X, 16) || !aligned(sums, 16) || !aligned(labels, 4) || !aligned(counts, 4)) {
+        set_error("km_update_sums: X and sums must be 16-byte aligned, labels and counts 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    Scratch scratch(st);
+    int32_t *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr;
+    unsigned char* work = nullptr;
+    KM_TRY(scratch.get(&a_sorted, (size_t)(B * N), "sorted labels"));
+    KM_TRY(scratch.get(&sidx, (size_t)(B * N), "sorted indices"));
+    KM_TRY(scratch.get(&offs, (size_t)(B * (K + 1)), "segment offsets"));
+    KM_TRY(scratch.get(&work, sort_scratch_bytes(B, N, K), "radix sort buffers"));
+    {
+        PhaseScope ph(st, KM_PHASE_OTHER, 0);
+        KM_TRY(launched(cudaMemsetAsync(sums, 0, sizeof(float) * (size_t)(B * K * d), st), "zero sums"));
+        KM_TRY(launched(cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)(B * K), st), "zero counts"));
+    }
+    {
+        PhaseScope ph(st, KM_PHASE_SORT, sort_kernel_launches(N, K, false, false));
+        KM_TRY(launched(launch_sort(labels, B, N, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
+                        "label sort"));
+    }
+    PhaseScope ph(st, KM_PHASE_UPDATE, 2);
+    KM_TRY(launched(launch_update_sums(X, dtype, a_sorted, sidx, B, N, K, d, sums, offs, st), "segmented update"));
+    return launched(launch_add_counts(offs, B, K, counts, st), "cluster counts");
+}
+
+km_status km_finalize(const float* sums, const int32_t* counts, int64_t B, int64_t K, int64_t d, float* C_out,
+                      void* stream) {
+    g_err[0] = 0;
+    if (!sums || !counts || !C_out) {
+        set_error("km_finalize: sums, counts and C_out must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, 1, K, d, KM_F32));
+    if (!aligned(sums, 16) || !aligned(C_out, 16) || !aligned(counts, 4)) {
+        set_error("km_finalize: sums and C_out must be 16-byte aligned, counts 4-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    PhaseScope ph(st, KM_PHASE_FINALIZE, 1);
+    return launched(launch_finalize(const_cast<float*>(sums), nullptr, B, K, d, C_out, KM_F32, PreparedC(), nullptr,
+                                    false, nullptr, nullptr, st, counts),
+                    "centroid finalize");
+}
+
 km_status km_assign_dense(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
                           int32_t* labels, float* mindist, void* stream) {
     g_err[0] = 0;

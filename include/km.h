@@ -185,6 +185,21 @@ KM_API km_status km_assign_noalloc(const void* X, const float* C, int64_t B, int
 KM_API size_t km_assign_noalloc_limit(void);
 
 /*
+ * The update split in its two halves, for callers that combine the sums of
+ * several shards of the points before dividing (e.g. one shard per GPU with
+ * an all-reduce in between; see flashassign_b200.sharded).
+ * km_update_sums: sort the labels and gather-reduce as km_update does,
+ *   sums[b][k] = sum of the rows labelled k, counts[b][k] = their number;
+ *   no centroid is written.  Arguments as km_update.
+ * km_finalize: C_out[b][k] = sums[b][k] / counts[b][k] where counts > 0, else
+ *   unchanged (C_out is in/out, [B, K, d] fp32, 16-byte aligned).
+ */
+KM_API km_status km_update_sums(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d,
+                                int dtype, float* sums, int32_t* counts, void* stream);
+KM_API km_status km_finalize(const float* sums, const int32_t* counts, int64_t B, int64_t K, int64_t d, float* C_out,
+                             void* stream);
+
+/*
  * Baselines the method replaces, for measurement (papernotes.org page,
  * 方法详解 and 关键设计 1-2: the standard implementations whose memory
  * traffic and atomic contention Flash-KMeans removes).  Same results as
