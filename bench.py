@@ -37,15 +37,30 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "7e5a00a8cfdf487024aadac22ffd70cd463ccd10",
                             "tc_ptx.cuh": "ee9645b484e88174263ad58b26408994fd536d40",
                             "km_internal.cuh": "2c304a53203d0a8b6b4daae5b52fe75657c97a48"},
-                  "bytes": 546.353920e6 + 10.674432e6}
+                  "bytes": 546.353920e6 + 10.674432e6, "workload": "b32_n65536_d128_k1024_f16"}
 UPDATE_TRAFFIC = {"files": {"update.cu": "e782d07783850ee11aed345f376d4c4a44fc6f24",
                             "km_internal.cuh": "2c304a53203d0a8b6b4daae5b52fe75657c97a48"},
-                  "bytes": 557.689344e6 + 16.603648e6}
+                  "bytes": 557.689344e6 + 16.603648e6, "workload": "b32_n65536_d128_k1024_f16"}
 
 
-def traffic_for(rec: dict):
-    """The recorded traffic while every source file the kernel is built from is unchanged."""
+def assign_kernel_name(w) -> str:
+    """The assignment kernel the library dispatches for this workload's dtype and d."""
+    if w.dtype == "f16":
+        if 64 <= w.d <= 128 and w.d % 8 == 0:
+            return "assign_tc_kernel"
+        if w.d % 64 == 0 and w.d > 128:
+            return "assign_wide_kernel" if w.d <= 512 else "assign_split_kernel"
+    elif 32 <= w.d <= 128 and w.d % 32 == 0:
+        return "assign_tf32_kernel"
+    return "assign_simt_kernel"
+
+
+def traffic_for(rec: dict, workload: str):
+    """The recorded traffic of the workload it was taken on, while every source file the kernel is
+    built from is unchanged."""
     import hashlib
+    if workload != rec["workload"]:
+        return None
     for name, want in rec["files"].items():
         try:
             with open(os.path.join(ROOT, "flashassign_b200", "csrc", name), "rb") as f:
@@ -408,15 +423,15 @@ def run_ours(args, w):
                    "parallelism": f"replicas{world}",
                    "l2": f"inputs larger than L2 (X is {w.B * w.N * w.d * w.elem_bytes / 2**20:.0f} MiB)"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": round(tflops / peak_tf, 4), "traffic": traffic_for(ASSIGN_TRAFFIC),
-                     "kernel": "assign_tc_kernel",
+                     "frac": round(tflops / peak_tf, 4), "traffic": traffic_for(ASSIGN_TRAFFIC, w.name),
+                     "kernel": assign_kernel_name(w),
                      "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate equals bf16); the kernel runs "
                                     f"inside a long power-capped loop",
                      "frac_of_burst_peak": round(tflops / peak_burst, 4), "burst_peak": peak_burst,
                      "ms_per_launch": round(t_assign, 4)},
         "roofline_update": {"bound": "hbm", "achieved": round(upd_gbs, 1), "peak": peak_bw, "unit": "GB/s",
                             "frac": round(upd_gbs / peak_bw, 4), "kernel": "update_kernel",
-                            "traffic": traffic_for(UPDATE_TRAFFIC),
+                            "traffic": traffic_for(UPDATE_TRAFFIC, w.name),
                             "ms_per_launch": round(t_update, 4), "peak_source": peak_src},
         "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4),
                                "frac_with_burst_tensor_peak": round(t_roof_burst / ms_iter, 4)},

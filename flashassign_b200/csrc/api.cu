@@ -140,6 +140,8 @@ class PhaseScope {
     cudaEvent_t a_ = nullptr;
 };
 
+constexpr int kMaxDim = 16384;
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 km_status check_shape(int64_t B, int64_t N, int64_t K, int64_t d, int dtype) {
@@ -152,8 +154,8 @@ km_status check_shape(int64_t B, int64_t N, int64_t K, int64_t d, int dtype) {
         set_error("unknown dtype %d", dtype);
         return KM_E_INVALID;
     }
-    if (B > 65535 || B * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 24) || d > 512) {
-        set_error("outside the supported range: B <= 65535, B*N < 2^31, K < 2^24, d <= 512");
+    if (B > 65535 || B * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 24) || d > kMaxDim) {
+        set_error("outside the supported range: B <= 65535, B*N < 2^31, K < 2^24, d <= %d", kMaxDim);
         return KM_E_UNSUPPORTED;
     }
     const int64_t s = dtype == KM_F16 ? 2 : 4;
@@ -188,7 +190,8 @@ km_status launched(cudaError_t e, const char* what) {
     } while (0)
 
 bool uses_tc(int dtype, int64_t d) {
-    return dtype == KM_F16 ? (assign_tc_supported(d, dtype) || assign_wide_supported(d, dtype))
+    return dtype == KM_F16 ? (assign_tc_supported(d, dtype) || assign_wide_supported(d, dtype) ||
+                              assign_split_supported(d, dtype))
                            : assign_tf32_supported(d);
 }
 
@@ -245,6 +248,13 @@ km_status alloc_tc(Scratch& s, int dtype, int64_t B, int64_t K, int64_t d, int64
 km_status run_assign(const void* X, int dtype, const float* C, const TcScratch* tc, int64_t B, int64_t N, int64_t K,
                      int64_t d, int32_t* labels, float* mindist, double* obj_acc, const DeviceInfo& dev,
                      cudaStream_t st, const int32_t* stop = nullptr) {
+    if (tc && dtype == KM_F16 && assign_split_supported(d, dtype)) {
+        PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
+        return launched(launch_assign_split((const __half*)X, static_cast<const __half*>(tc->prep.chat),
+                                            static_cast<const __half*>(tc->prep.cext), B, N, K, d, labels, mindist,
+                                            obj_acc, dev.sms, st, stop),
+                        "assign (tensor cores, points and centroids streamed along d)");
+    }
     if (tc && dtype == KM_F16 && assign_wide_supported(d, dtype)) {
         PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
         return launched(launch_assign_wide((const __half*)X, static_cast<const __half*>(tc->prep.chat),
@@ -280,6 +290,7 @@ km_status run_assign(const void* X, int dtype, const float* C, const TcScratch* 
 
 std::atomic<int64_t> g_chunk_rows{0};
 constexpr int64_t kDefaultChunkRows = int64_t(1) << 23;
+constexpr int64_t kDefaultChunkBytes = int64_t(1) << 32;  // the default chunk also stays within 4 GiB
 constexpr int kSlots = 2;
 
 // Host-side wait for a stream, polled against a deadline (KM_HOST_TIMEOUT_S,
@@ -342,7 +353,7 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
                      cudaStream_t st) {
     const int64_t s = dtype == KM_F16 ? 2 : 4;
     int64_t R = g_chunk_rows.load();
-    if (R <= 0) R = kDefaultChunkRows;
+    if (R <= 0) R = std::max<int64_t>(1, std::min(kDefaultChunkRows, kDefaultChunkBytes / (d * s)));
     if (R > N) R = N;
     const bool tc = uses_tc(dtype, d);
     const int64_t Kp = padded_k(K);

@@ -116,16 +116,17 @@ __global__ void prep_kernel(const float* __restrict__ C, int64_t B, int64_t K, i
     if (lane == 0) write_row_norm(p, dtype, b, row, acc);
 }
 
-// Lanes per centroid row in the finalisation: each lane takes every eighth
-// 4-wide chunk of the row, a warp finalises four rows at once.
-constexpr int kFinLanes = 8;
+// Lanes per centroid row in the finalisation (L = 8 below d = 512, where a
+// warp finalises four rows at once; L = 32, a warp per row, from d = 512 on):
+// each lane takes every L-th 4-wide chunk of the row.
 constexpr int kFinThreads = 256;
 
 // n_k comes from the sort's segment offsets (offsets[k+1] - offsets[k]); it is
 // also written to counts when that is non-null.  With zero_sums the consumed
 // sums are reset to 0, ready for the next iteration's boundary atomics.  When
 // `next` holds buffers, the new centroids are prepared for the next
-// assignment as prep_kernel does.  Grid: (rows of a batch / 32, B).
+// assignment as prep_kernel does.  Grid: (rows of a batch * L / 256, B).
+template <int kFinLanes>
 __global__ void __launch_bounds__(kFinThreads) finalize_kernel(
     float* __restrict__ sums, const int32_t* __restrict__ offsets, int64_t K, int64_t Kp, int64_t d,
     float* __restrict__ C_out, int dtype, PreparedC next, int32_t* __restrict__ counts, int zero_sums,
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(
         for (int o = kFinLanes / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (valid && sub == 0) write_row_norm(next, dtype, b, b * Kp + k, acc);
     }
-    if (shift) {  // the warp's four rows, one atomic
+    if (shift) {  // the warp's rows, one atomic
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) moved += __shfl_xor_sync(0xffffffffu, moved, o);
         if ((threadIdx.x & 31) == 0 && moved != 0.0) atomicAdd(shift + b, moved);
@@ -248,9 +249,14 @@ cudaError_t launch_finalize(float* sums, const int32_t* offsets, int64_t B, int6
                             int dtype, PreparedC next, int32_t* counts, bool zero_sums, double* obj_acc,
                             float* obj_out, cudaStream_t st, const int32_t* counts_in, const int32_t* stop,
                             double* shift) {
-    const dim3 grid((unsigned)ceil_div(K * kFinLanes, kFinThreads), (unsigned)B);
-    return launch_kernel(finalize_kernel, grid, dim3(kFinThreads), 0, st, sums, offsets, K, padded_k(K), d, C_out, dtype,
-                         next, counts, zero_sums ? 1 : 0, obj_acc, obj_out, counts_in, stop, shift);
+    if (d >= 512) {
+        const dim3 grid((unsigned)ceil_div(K * 32, kFinThreads), (unsigned)B);
+        return launch_kernel(finalize_kernel<32>, grid, dim3(kFinThreads), 0, st, sums, offsets, K, padded_k(K), d,
+                             C_out, dtype, next, counts, zero_sums ? 1 : 0, obj_acc, obj_out, counts_in, stop, shift);
+    }
+    const dim3 grid((unsigned)ceil_div(K * 8, kFinThreads), (unsigned)B);
+    return launch_kernel(finalize_kernel<8>, grid, dim3(kFinThreads), 0, st, sums, offsets, K, padded_k(K), d, C_out,
+                         dtype, next, counts, zero_sums ? 1 : 0, obj_acc, obj_out, counts_in, stop, shift);
 }
 
 cudaError_t launch_converge_check(double* shift, int64_t B, double tol, int32_t* stop, int32_t* iters_run,

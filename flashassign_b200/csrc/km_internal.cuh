@@ -116,6 +116,14 @@ cudaError_t launch_assign_wide(const __half* X, const __half* chat, const __half
                                int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms,
                                cudaStream_t st, const int32_t* stop = nullptr);
 
+// Tensor-core assignment of fp16 points with d > 512 (d % 64 == 0): points and
+// centroids both stream in 64-dimension chunks, each point chunk meeting two
+// centroid tiles.  Same prepared centroids and results as launch_assign_tc.
+bool assign_split_supported(int64_t d, int dtype);
+cudaError_t launch_assign_split(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N,
+                                int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms,
+                                cudaStream_t st, const int32_t* stop = nullptr);
+
 // Tensor-core assignment of fp32 points (tf32 head/tail split, 32 <= d <= 128,
 // d % 32 == 0).  Points whose best two scores lie within the split's error
 // bound are not resolved: they are appended to flag_rows[b * N + ...]

@@ -65,8 +65,8 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
         return KM_E_INVALID;
     }
     const int64_t s = dtype == KM_F16 ? 2 : 4;
-    if (B > 65535 || B * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 24) || d > 512 || (d * s) % 16 != 0) {
-        set_error("km_assign_noalloc: outside the supported range (B <= 65535, B*N < 2^31, K < 2^24, d <= 512, "
+    if (B > 65535 || B * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 24) || d > 16384 || (d * s) % 16 != 0) {
+        set_error("km_assign_noalloc: outside the supported range (B <= 65535, B*N < 2^31, K < 2^24, d <= 16384, "
                   "d * sizeof(dtype) a multiple of 16 bytes)");
         return KM_E_UNSUPPORTED;
     }
@@ -84,7 +84,8 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
         return KM_E_UNSUPPORTED;
     }
     cudaStream_t stm = (cudaStream_t)stream;
-    const bool tc = dtype == KM_F16 && assign_tc_supported(d, dtype);
+    const bool tc = dtype == KM_F16 && (assign_tc_supported(d, dtype) || assign_wide_supported(d, dtype) ||
+                                        assign_split_supported(d, dtype));
     if (!tc) {  // the CUDA-core kernel reads C directly and needs no scratch
         cudaError_t e = launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, nullptr, stm);
         return e == cudaSuccess ? KM_OK : cuda_error(e, "km_assign_noalloc: assign (CUDA cores)");
@@ -92,7 +93,7 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
     const size_t chat_bytes = round_up(sizeof(__half) * (size_t)(B * K * d), 256);
     const size_t cext_bytes = sizeof(__half) * (size_t)(B * padded_k(K) * 16);
     if (chat_bytes + cext_bytes > kNoAllocScratchBytes) {
-        set_error("km_assign_noalloc: needs %zu bytes of scratch (2*B*K*d + 32*B*ceil(K/128)*128), above the "
+        set_error("km_assign_noalloc: needs %zu bytes of scratch (2*B*K*d + 32*B*ceil(K/256)*256), above the "
                   "fixed %zu-byte array; use km_assign",
                   chat_bytes + cext_bytes, kNoAllocScratchBytes);
         return KM_E_UNSUPPORTED;
@@ -107,7 +108,12 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
     prep.cext = cext;
     cudaError_t e = launch_prep_centroids(C, B, K, d, dtype, prep, stm);
     if (e != cudaSuccess) return cuda_error(e, "km_assign_noalloc: centroid preparation");
-    e = launch_assign_tc(static_cast<const __half*>(X), chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms,
-                         stm);
+    const __half* Xh = static_cast<const __half*>(X);
+    if (assign_split_supported(d, dtype))
+        e = launch_assign_split(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms, stm);
+    else if (assign_wide_supported(d, dtype))
+        e = launch_assign_wide(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms, stm);
+    else
+        e = launch_assign_tc(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms, stm);
     return e == cudaSuccess ? KM_OK : cuda_error(e, "km_assign_noalloc: assign (tensor cores)");
 }

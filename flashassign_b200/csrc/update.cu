@@ -12,7 +12,10 @@
 // counter atomics and no separate pass are needed.
 //
 // Layout of a CTA (16-byte chunks of a row per thread):
-//   tpr = d * sizeof(T) / 16 threads cover one row; G = 256 / tpr row-lanes;
+//   rows longer than 1 KB are split into 1 KB slices of W dimensions, one
+//   slice per grid z (the same positions in every slice), so a CTA covers W = d
+//   or W = 1024 / sizeof(T) dimensions of each row;
+//   tpr = W * sizeof(T) / 16 threads cover one row; G = 256 / tpr row-lanes;
 //   row-lane g walks 16 consecutive sorted positions (B_N = 16 G), issuing
 //   four independent 16-byte gathers at a time and keeping a running fp32
 //   partial sum in registers.  A label change inside the walk ends a piece:
@@ -61,7 +64,7 @@ struct Chunk<float> {
 template <typename T>
 __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, const int32_t* __restrict__ a_sorted,
                                                      const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
-                                                     int64_t d, int tpr, int G, float* __restrict__ sums,
+                                                     int64_t d, int64_t W, int tpr, int G, float* __restrict__ sums,
                                                      int32_t* __restrict__ offsets, int accumulate,
                                                      const int32_t* __restrict__ stop) {
     pdl_trigger();
@@ -70,14 +73,16 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     constexpr int E = Chunk<T>::kElems;
     extern __shared__ __align__(16) unsigned char smem[];
     const int BN = G * kRowsPerLane;
-    float* head_vec = reinterpret_cast<float*>(smem);    // [G][d]
-    float* tail_vec = head_vec + (size_t)G * d;          // [G][d]
-    int* s_lab = reinterpret_cast<int*>(tail_vec + (size_t)G * d);  // [BN]
+    float* head_vec = reinterpret_cast<float*>(smem);    // [G][W]
+    float* tail_vec = head_vec + (size_t)G * W;          // [G][W]
+    int* s_lab = reinterpret_cast<int*>(tail_vec + (size_t)G * W);  // [BN]
     int* s_idx = s_lab + BN;                             // [BN]
     int* head_lab = s_idx + BN;                          // [G]
     int* tail_lab = head_lab + G;                        // [G]
 
     const int64_t b = blockIdx.y;
+    const int64_t z0 = (int64_t)blockIdx.z * W;          // first dimension of this slice
+    const int Wz = (int)min(W, d - z0);                  // its width
     const int64_t p0 = (int64_t)blockIdx.x * BN;
     const int64_t pend = min(p0 + BN, N);
     const int n = (int)(pend - p0);
@@ -87,7 +92,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         s_idx[t] = sorted_idx[b * N + p0 + t];
     }
     __syncthreads();
-    if (offsets) {
+    if (offsets && blockIdx.z == 0) {
         // Segment offsets of the sorted labels: position p starts every label k
         // with a[p-1] < k <= a[p] (labels clamped so nothing is written out of
         // bounds); the last run also closes labels above a[N-1] at N.
@@ -105,11 +110,11 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
 
     const int g = threadIdx.x / tpr, c = threadIdx.x % tpr;
     const int r0 = g * kRowsPerLane, r1 = min(r0 + kRowsPerLane, n);
-    float* sums_b = sums + b * K * d + (int64_t)c * E;
+    float* sums_b = sums + b * K * d + z0 + (int64_t)c * E;
     if (r0 >= r1) {
         if (c == 0) head_lab[g] = tail_lab[g] = -1;
-    } else {
-        const T* xb = X + b * N * d + (int64_t)c * E;
+    } else if (c * E < Wz) {  // (chunks past a narrower last slice idle; c = 0 never does)
+        const T* xb = X + b * N * d + z0 + (int64_t)c * E;
         float acc[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = 0.f;
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
                     if (piece == 0) {
                         if (c == 0) head_lab[g] = cur;
 #pragma unroll
-                        for (int e = 0; e < E; ++e) head_vec[(size_t)g * d + c * E + e] = acc[e];
+                        for (int e = 0; e < E; ++e) head_vec[(size_t)g * W + c * E + e] = acc[e];
                     } else if (cur >= 0 && cur < K) {  // a whole cluster inside this walk
 #pragma unroll
                         for (int e = 0; e < E; e += 4) {
@@ -155,18 +160,18 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
                 tail_lab[g] = -1;
             }
 #pragma unroll
-            for (int e = 0; e < E; ++e) head_vec[(size_t)g * d + c * E + e] = acc[e];
+            for (int e = 0; e < E; ++e) head_vec[(size_t)g * W + c * E + e] = acc[e];
         } else {
             if (c == 0) tail_lab[g] = cur;
 #pragma unroll
-            for (int e = 0; e < E; ++e) tail_vec[(size_t)g * d + c * E + e] = acc[e];
+            for (int e = 0; e < E; ++e) tail_vec[(size_t)g * W + c * E + e] = acc[e];
         }
     }
     __syncthreads();
 
     // Join the boundary pieces in position order; one thread per 4 dims.
     const int j4 = threadIdx.x * 4;
-    if (j4 >= d) return;
+    if (j4 >= Wz) return;
     const int before = p0 > 0 ? ab[p0 - 1] : -1;   // label just before the run
     const int after = pend < N ? ab[pend] : -1;    // label just after it
     int run_lab = -1;
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         if (lab < 0 || lab >= K) return;
         const bool shared_left = first && before == lab;
         const bool shared_right = last && after == lab;
-        float* dst = sums + (b * K + lab) * d + j4;
+        float* dst = sums + (b * K + lab) * d + z0 + j4;
         if (shared_left || shared_right) {
             atomicAdd(reinterpret_cast<float4*>(dst), v);
         } else if (accumulate) {
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         for (int which = 0; which < 2; ++which) {
             const int lab = which == 0 ? head_lab[gg] : tail_lab[gg];
             if (lab < 0) continue;
-            const float4 v = *reinterpret_cast<const float4*>((which == 0 ? head_vec : tail_vec) + (size_t)gg * d + j4);
+            const float4 v = *reinterpret_cast<const float4*>((which == 0 ? head_vec : tail_vec) + (size_t)gg * W + j4);
             if (seen && lab == run_lab) {
                 run.x += v.x; run.y += v.y; run.z += v.z; run.w += v.w;
             } else {
@@ -211,17 +216,18 @@ template <typename T>
 cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sorted_idx, int64_t B, int64_t N,
                      int64_t K, int64_t d, float* sums, int32_t* offsets, bool accumulate, cudaStream_t st,
                      const int32_t* stop) {
-    const int tpr = (int)(d * (int64_t)sizeof(T) / 16);
-    const int G = 256 / tpr;
+    const int64_t W = d * (int64_t)sizeof(T) <= 1024 ? d : 1024 / (int64_t)sizeof(T);  // dims per slice
+    const int tpr = (int)(W * (int64_t)sizeof(T) / 16);                                 // <= 64
+    const int G = 256 / tpr;                                                              // >= 4
     const int BN = G * kRowsPerLane;
-    const size_t smem = sizeof(float) * 2 * (size_t)G * d + sizeof(int) * (2 * (size_t)BN + 2 * (size_t)G);
+    const size_t smem = sizeof(float) * 2 * (size_t)G * W + sizeof(int) * (2 * (size_t)BN + 2 * (size_t)G);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(update_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B);
+    const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B, (unsigned)ceil_div(d, W));
     return launch_kernel(update_kernel<T>, grid, dim3(G * tpr), smem, st, (const T*)X, a_sorted, sorted_idx, N, K, d,
-                         tpr, G, sums, offsets, accumulate ? 1 : 0, stop);
+                         W, tpr, G, sums, offsets, accumulate ? 1 : 0, stop);
 }
 
 }  // namespace

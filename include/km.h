@@ -24,7 +24,7 @@
  *   - `stream` is a cudaStream_t (NULL means the legacy default stream).
  *     Every call is asynchronous on it: results are ready once the stream is
  *     synchronised.  Argument errors return before any work is enqueued.
- *   - Supported: B >= 1, N >= 1, K >= 1, B*N < 2^31, K < 2^24, 1 <= d <= 512,
+ *   - Supported: B >= 1, N >= 1, K >= 1, B*N < 2^31, K < 2^24, 1 <= d <= 16384,
  *     d * sizeof(dtype) a multiple of 16 bytes, X and the [B, K, d] arrays
  *     (C, C_init, C_out, sums) 16-byte aligned, every other array 4-byte
  *     aligned, a device of compute capability 10.0.
@@ -70,6 +70,9 @@ typedef enum {
  *   - fp16, 64 <= d <= 128: on the tensor cores;
  *   - fp16, d in {192, 256, ..., 512}: on the tensor cores, the centroids
  *     streamed in 64-dimension chunks;
+ *   - fp16, d a multiple of 64 above 512 (the split-D path of the 7minutos.es
+ *     article, "Usándolo"): on the tensor cores, points and centroids both
+ *     streamed in 64-dimension chunks, each point chunk meeting 512 centroids;
  *   - fp32, d in {32, 64, 96, 128}: on the tensor cores from tf32 head/tail
  *     splits of both operands (three products); a point whose best two scores
  *     lie within the split's error bound is re-scanned exactly on the CUDA
@@ -170,8 +173,9 @@ KM_API km_status km_lloyd_tol(const void* X, const float* C_init, int64_t B, int
  * km_assign; the scratch (fp16 centroids and their norm slices) lives in one
  * fixed array of km_assign_noalloc_limit() bytes (16 MiB) compiled into the
  * library, which every GPU that loads the library holds until exit.
- *   - Needs 2*B*K*d + 32*B*ceil(K/128)*128 bytes for fp16 inputs with
- *     64 <= d <= 128 (none otherwise); larger problems return
+ *   - Needs 2*B*K*d + 32*B*ceil(K/256)*256 bytes for fp16 inputs on the
+ *     tensor-core paths (64 <= d <= 128, or d a multiple of 64 above 128;
+ *     none otherwise); larger problems return
  *     KM_E_UNSUPPORTED with the sizes in km_last_error().
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
@@ -236,7 +240,8 @@ KM_API km_status km_update_scatter(const void* X, const int32_t* labels, int64_t
  */
 KM_API km_status km_release_cached(void);
 
-/* Rows per chunk used by km_lloyd for host-resident X (0 restores the default, 2^23). */
+/* Rows per chunk used by km_lloyd for host-resident X (0 restores the default:
+ * 2^23 rows, fewer when that would exceed 4 GiB, i.e. min(2^23, 2^32 / (d * sizeof(dtype)))). */
 KM_API void km_set_chunk_rows(int64_t rows);
 
 /*

@@ -120,6 +120,10 @@ WORKLOADS = {
     # wide points: the d = 512 shape of the papernotes.org page's end-to-end table (N = 1M, K = 65536)
     6: Workload("b1_n1048576_d512_k65536_f16", 1, 1 << 20, 512, 65536, "f16", ncomp=65536,
                 sigma=0.25, iters=3, seed=0x6B6D0006),
+    # very wide points: d = 4096, the dense multimodal width the papernotes.org page names as the limit
+    # of on-chip tiles (局限与展望), served by the split-D path
+    7: Workload("b1_n262144_d4096_k4096_f16", 1, 1 << 18, 4096, 4096, "f16", ncomp=4096,
+                sigma=0.25, iters=3, seed=0x6B6D0007),
 }
 
 

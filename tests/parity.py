@@ -5,8 +5,11 @@ Tolerances (the stated bar for this method):
     at least TAU_LABEL (1e-3 for fp16 inputs, 1e-5 for fp32); below it, the GPU
     label must be a near-minimiser, dist(gpu label) <= d1 + tau * d2.  The
     number of such near ties is returned for reporting.
-  * mindist: |m_gpu - m_oracle(gpu label)| <= 1e-5 * (||x||^2 + ||c||^2) + 1e-6,
-    the fp32 rounding scale of the expansion ||x||^2 + ||c||^2 - 2 x.c.
+  * mindist: |m_gpu - m_oracle(gpu label)| <= tau_m(d) * (||x||^2 + ||c||^2) + 1e-6,
+    the fp32 rounding scale of the expansion ||x||^2 + ||c||^2 - 2 x.c, with
+    tau_m(d) = max(1e-5, d * 2^-24): x.c and ||x||^2 are fp32 sums of d terms, whose
+    first-order error bound is gamma_d ~ d * u (u = 2^-24) times the sum of the
+    terms' magnitudes, itself at most (||x||^2 + ||c||^2) / 2 for x.c.
   * sort, counts, offsets: bit-exact.
   * centroids: ||c_gpu - c_ref||_inf <= 1e-4 * max(||c_ref||_inf, 1e-6) per
     centroid; empty clusters bit-identical to the previous centroid.
@@ -19,6 +22,10 @@ import oracle
 
 TAU_LABEL = {"f16": 1e-3, "f32": 1e-5}
 TAU_MIND = 1e-5
+
+
+def tau_mind(d: int) -> float:
+    return max(TAU_MIND, d * 2.0 ** -24)
 TAU_CENTROID = 1e-4
 
 
@@ -55,7 +62,7 @@ def check_labels(X, C, gpu_labels, gpu_mindist=None, rows=None):
         gm = np.asarray(gpu_mindist).reshape(-1)[flat].astype(np.float64)
         scale = (xs ** 2).sum(axis=1) + (cg ** 2).sum(axis=1)
         err = np.abs(gm - dist_g)
-        lim = TAU_MIND * scale + 1e-6
+        lim = tau_mind(d) * scale + 1e-6
         worst = np.argmax(err / lim)
         assert (err <= lim).all(), (f"mindist off: row {flat[worst]} gpu {gm[worst]} ref {dist_g[worst]} "
                                     f"err {err[worst]} lim {lim[worst]}")

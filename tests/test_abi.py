@@ -49,7 +49,7 @@ FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: validati
     (dict(K=0), 1),
     (dict(dtype=7), 1),
     (dict(d=12), 2),          # 24 bytes of fp16 per row: not a multiple of 16
-    (dict(d=520), 2),         # d > 512
+    (dict(d=16392), 2),       # d > 16384
     (dict(B=70000), 2),
     (dict(K=1 << 24), 2),
     (dict(X=ctypes.c_void_p(0x10008)), 2),  # X not 16-byte aligned

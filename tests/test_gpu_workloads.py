@@ -82,6 +82,12 @@ def test_wide_points_d512_k65536():
     lockstep(w, 1, nsample=256)
 
 
+def test_very_wide_points_d4096_split_d():
+    # d = 4096 on the split-D tensor-core path (points and centroids both streamed along d)
+    w = synth.WORKLOADS[7]
+    lockstep(w, 2, nsample=256)
+
+
 def test_workload5_host_resident_fp32_chunked():
     """2^27 x 128 fp32 points (64 GiB) in pinned host memory, streamed in 2^23-row chunks."""
     import time
