@@ -75,8 +75,9 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     const int BN = G * kRowsPerLane;
     float* head_vec = reinterpret_cast<float*>(smem);    // [G][W]
     float* tail_vec = head_vec + (size_t)G * W;          // [G][W]
-    int* s_lab = reinterpret_cast<int*>(tail_vec + (size_t)G * W);  // [BN]
-    int* s_idx = s_lab + BN;                             // [BN]
+    // the run's labels with one neighbour on each side: s_lab[-1 .. BN], -1 outside [0, N)
+    int* s_lab = reinterpret_cast<int*>(tail_vec + (size_t)G * W) + 1;
+    int* s_idx = s_lab + BN + 1;                         // [BN]
     int* head_lab = s_idx + BN;                          // [G]
     int* tail_lab = head_lab + G;                        // [G]
 
@@ -87,9 +88,10 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     const int64_t pend = min(p0 + BN, N);
     const int n = (int)(pend - p0);
     const int32_t* ab = a_sorted + b * N;
-    for (int t = threadIdx.x; t < n; t += blockDim.x) {
-        s_lab[t] = ab[p0 + t];
-        s_idx[t] = sorted_idx[b * N + p0 + t];
+    for (int t = (int)threadIdx.x - 1; t <= n; t += blockDim.x) {
+        const int64_t p = p0 + t;
+        s_lab[t] = (p >= 0 && p < N) ? ab[p] : -1;
+        if (t >= 0 && t < n) s_idx[t] = sorted_idx[b * N + p];
     }
     __syncthreads();
     if (offsets && blockIdx.z == 0) {
@@ -100,7 +102,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         for (int t = threadIdx.x; t <= n; t += blockDim.x) {
             const int64_t p = p0 + t;
             if (t == n && p != N) break;
-            int64_t prev = t > 0 ? s_lab[t - 1] : (p0 > 0 ? ab[p0 - 1] : -1);
+            int64_t prev = s_lab[t - 1];
             int64_t cur = p == N ? K : s_lab[t];
             prev = min(max(prev, (int64_t)-1), K);
             cur = min(max(cur, (int64_t)-1), K);
@@ -172,8 +174,8 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     // Join the boundary pieces in position order; one thread per 4 dims.
     const int j4 = threadIdx.x * 4;
     if (j4 >= Wz) return;
-    const int before = p0 > 0 ? ab[p0 - 1] : -1;   // label just before the run
-    const int after = pend < N ? ab[pend] : -1;    // label just after it
+    const int before = s_lab[-1];  // label just before the run
+    const int after = s_lab[n];    // label just after it
     int run_lab = -1;
     bool run_first = false;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -220,7 +222,7 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
     const int tpr = (int)(W * (int64_t)sizeof(T) / 16);                                 // <= 64
     const int G = 256 / tpr;                                                              // >= 4
     const int BN = G * kRowsPerLane;
-    const size_t smem = sizeof(float) * 2 * (size_t)G * W + sizeof(int) * (2 * (size_t)BN + 2 * (size_t)G);
+    const size_t smem = sizeof(float) * 2 * (size_t)G * W + sizeof(int) * (2 * (size_t)BN + 2 + 2 * (size_t)G);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(update_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
