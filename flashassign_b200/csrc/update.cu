@@ -61,7 +61,13 @@ struct Chunk<float> {
     }
 };
 
-template <typename T>
+// kSliced: rows are cut into slices of W dimensions along grid z; otherwise a
+// CTA covers whole rows (W = d) and every slice term folds away at compile time.
+// The gathers are latency-bound, so the number of resident warps sets the
+// bandwidth: the whole-row form compiles to 48 registers (five CTAs per SM);
+// folding the slice terms in at run time cost it four registers, one CTA per
+// SM and 17% of its speed at d = 128.
+template <typename T, bool kSliced>
 __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, const int32_t* __restrict__ a_sorted,
                                                      const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
                                                      int64_t d, int64_t W, int tpr, int G, float* __restrict__ sums,
@@ -73,28 +79,27 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     constexpr int E = Chunk<T>::kElems;
     extern __shared__ __align__(16) unsigned char smem[];
     const int BN = G * kRowsPerLane;
-    float* head_vec = reinterpret_cast<float*>(smem);    // [G][W]
-    float* tail_vec = head_vec + (size_t)G * W;          // [G][W]
-    // the run's labels with one neighbour on each side: s_lab[-1 .. BN], -1 outside [0, N)
-    int* s_lab = reinterpret_cast<int*>(tail_vec + (size_t)G * W) + 1;
-    int* s_idx = s_lab + BN + 1;                         // [BN]
+    const int64_t Wd = kSliced ? W : d;                  // dimensions per CTA
+    float* head_vec = reinterpret_cast<float*>(smem);    // [G][Wd]
+    float* tail_vec = head_vec + (size_t)G * Wd;         // [G][Wd]
+    int* s_lab = reinterpret_cast<int*>(tail_vec + (size_t)G * Wd);  // [BN]
+    int* s_idx = s_lab + BN;                             // [BN]
     int* head_lab = s_idx + BN;                          // [G]
     int* tail_lab = head_lab + G;                        // [G]
 
     const int64_t b = blockIdx.y;
-    const int64_t z0 = (int64_t)blockIdx.z * W;          // first dimension of this slice
-    const int Wz = (int)min(W, d - z0);                  // its width
+    const int64_t z0 = kSliced ? (int64_t)blockIdx.z * W : 0;  // first dimension of this slice
+    const int Wz = kSliced ? (int)min(W, d - z0) : (int)d;      // its width
     const int64_t p0 = (int64_t)blockIdx.x * BN;
     const int64_t pend = min(p0 + BN, N);
     const int n = (int)(pend - p0);
     const int32_t* ab = a_sorted + b * N;
-    for (int t = (int)threadIdx.x - 1; t <= n; t += blockDim.x) {
-        const int64_t p = p0 + t;
-        s_lab[t] = (p >= 0 && p < N) ? ab[p] : -1;
-        if (t >= 0 && t < n) s_idx[t] = sorted_idx[b * N + p];
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+        s_lab[t] = ab[p0 + t];
+        s_idx[t] = sorted_idx[b * N + p0 + t];
     }
     __syncthreads();
-    if (offsets && blockIdx.z == 0) {
+    if (offsets && (!kSliced || blockIdx.z == 0)) {
         // Segment offsets of the sorted labels: position p starts every label k
         // with a[p-1] < k <= a[p] (labels clamped so nothing is written out of
         // bounds); the last run also closes labels above a[N-1] at N.
@@ -102,7 +107,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         for (int t = threadIdx.x; t <= n; t += blockDim.x) {
             const int64_t p = p0 + t;
             if (t == n && p != N) break;
-            int64_t prev = s_lab[t - 1];
+            int64_t prev = t > 0 ? s_lab[t - 1] : (p0 > 0 ? ab[p0 - 1] : -1);
             int64_t cur = p == N ? K : s_lab[t];
             prev = min(max(prev, (int64_t)-1), K);
             cur = min(max(cur, (int64_t)-1), K);
@@ -115,7 +120,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     float* sums_b = sums + b * K * d + z0 + (int64_t)c * E;
     if (r0 >= r1) {
         if (c == 0) head_lab[g] = tail_lab[g] = -1;
-    } else if (c * E < Wz) {  // (chunks past a narrower last slice idle; c = 0 never does)
+    } else if (!kSliced || c * E < Wz) {  // (chunks past a narrower last slice idle; c = 0 never does)
         const T* xb = X + b * N * d + z0 + (int64_t)c * E;
         float acc[E];
 #pragma unroll
@@ -135,7 +140,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
                     if (piece == 0) {
                         if (c == 0) head_lab[g] = cur;
 #pragma unroll
-                        for (int e = 0; e < E; ++e) head_vec[(size_t)g * W + c * E + e] = acc[e];
+                        for (int e = 0; e < E; ++e) head_vec[(size_t)g * Wd + c * E + e] = acc[e];
                     } else if (cur >= 0 && cur < K) {  // a whole cluster inside this walk
 #pragma unroll
                         for (int e = 0; e < E; e += 4) {
@@ -162,11 +167,11 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
                 tail_lab[g] = -1;
             }
 #pragma unroll
-            for (int e = 0; e < E; ++e) head_vec[(size_t)g * W + c * E + e] = acc[e];
+            for (int e = 0; e < E; ++e) head_vec[(size_t)g * Wd + c * E + e] = acc[e];
         } else {
             if (c == 0) tail_lab[g] = cur;
 #pragma unroll
-            for (int e = 0; e < E; ++e) tail_vec[(size_t)g * W + c * E + e] = acc[e];
+            for (int e = 0; e < E; ++e) tail_vec[(size_t)g * Wd + c * E + e] = acc[e];
         }
     }
     __syncthreads();
@@ -174,8 +179,8 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     // Join the boundary pieces in position order; one thread per 4 dims.
     const int j4 = threadIdx.x * 4;
     if (j4 >= Wz) return;
-    const int before = s_lab[-1];  // label just before the run
-    const int after = s_lab[n];    // label just after it
+    const int before = p0 > 0 ? ab[p0 - 1] : -1;   // label just before the run
+    const int after = pend < N ? ab[pend] : -1;    // label just after it
     int run_lab = -1;
     bool run_first = false;
     float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -199,7 +204,7 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         for (int which = 0; which < 2; ++which) {
             const int lab = which == 0 ? head_lab[gg] : tail_lab[gg];
             if (lab < 0) continue;
-            const float4 v = *reinterpret_cast<const float4*>((which == 0 ? head_vec : tail_vec) + (size_t)gg * W + j4);
+            const float4 v = *reinterpret_cast<const float4*>((which == 0 ? head_vec : tail_vec) + (size_t)gg * Wd + j4);
             if (seen && lab == run_lab) {
                 run.x += v.x; run.y += v.y; run.z += v.z; run.w += v.w;
             } else {
@@ -222,14 +227,17 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
     const int tpr = (int)(W * (int64_t)sizeof(T) / 16);                                 // <= 64
     const int G = 256 / tpr;                                                              // >= 4
     const int BN = G * kRowsPerLane;
-    const size_t smem = sizeof(float) * 2 * (size_t)G * W + sizeof(int) * (2 * (size_t)BN + 2 + 2 * (size_t)G);
+    const size_t smem = sizeof(float) * 2 * (size_t)G * W + sizeof(int) * (2 * (size_t)BN + 2 * (size_t)G);
+    const bool sliced = W != d;
+    void (*kernel)(const T*, const int32_t*, const int32_t*, int64_t, int64_t, int64_t, int64_t, int, int, float*,
+                   int32_t*, int, const int32_t*) = sliced ? update_kernel<T, true> : update_kernel<T, false>;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(update_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     const dim3 grid((unsigned)ceil_div(N, BN), (unsigned)B, (unsigned)ceil_div(d, W));
-    return launch_kernel(update_kernel<T>, grid, dim3(G * tpr), smem, st, (const T*)X, a_sorted, sorted_idx, N, K, d,
-                         W, tpr, G, sums, offsets, accumulate ? 1 : 0, stop);
+    return launch_kernel(kernel, grid, dim3(G * tpr), smem, st, (const T*)X, a_sorted, sorted_idx, N, K, d, W, tpr, G,
+                         sums, offsets, accumulate ? 1 : 0, stop);
 }
 
 }  // namespace
