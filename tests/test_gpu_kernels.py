@@ -53,6 +53,8 @@ ASSIGN_SHAPES = [
     (3, 300, 513, 768, "f16"),
     (1, 513, 1024, 2048, "f16"),
     (1, 300, 60, 4096, "f16"),
+    (1, 700, 2100, 4096, "f16"),  # ... 9 centroid tiles: 5 passes, the last with one tile
+    (2, 300, 1500, 3072, "f16"),  # ... 6 tiles, 3 full passes, two batches
     (1, 200, 20, 1000, "f16"),   # d > 512, not a multiple of 64: CUDA-core kernel
     (1, 100, 20, 1000, "f32"),
     (1, 200, 30, 136, "f16"),    # not a multiple of 64: CUDA-core kernel
@@ -215,7 +217,8 @@ def test_update_matches_oracle(B, N, K, d, dt, case):
 @pytest.mark.parametrize("B,N,K,d,dt", [(2, 3000, 50, 128, "f16"), (1, 4096, 8, 16, "f32"), (2, 1000, 300, 64, "f16"),
                                         (2, 3000, 50, 128, "f32"), (1, 2000, 257, 32, "f32"),
                                         (1, 3000, 300, 512, "f16"), (2, 1000, 100, 256, "f16"),
-                                        (1, 1500, 100, 1024, "f16"), (1, 800, 40, 4096, "f16")])
+                                        (1, 1500, 100, 1024, "f16"), (1, 800, 40, 4096, "f16"),
+                                        (1, 1500, 1100, 2048, "f16")])
 def test_lloyd_lockstep_with_oracle(B, N, K, d, dt):
     """Each iteration: the oracle takes the GPU's centroids and checks that iteration's labels and update."""
     w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=5 + K)
