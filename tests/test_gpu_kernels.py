@@ -138,7 +138,8 @@ def test_assign_single_centroid_and_far_centroids():
 
 
 @pytest.mark.parametrize("case", ["random", "all_equal", "k1", "sorted", "skewed", "big_k", "ragged",
-                                  "one_pass_max", "one_pass_tiles", "one_pass_tail", "k4096", "long_small_k"])
+                                  "one_pass_max", "one_pass_tiles", "one_pass_tail", "k4096", "long_small_k",
+                                  "small_max", "small_odd", "small_one", "small_33", "small_reversed", "just_over"])
 def test_sort_is_bit_exact(case):
     rng = np.random.default_rng(13)
     B, N, K = 3, 5000, 1024
@@ -170,6 +171,25 @@ def test_sort_is_bit_exact(case):
         lab = rng.integers(0, K, (B, N))
     elif case == "one_pass_tail":
         B, N, K = 3, 4097, 5  # one key past a 4096-key tile, a few labels
+        lab = rng.integers(0, K, (B, N))
+    # single batches at and around 2^16 points
+    elif case == "small_max":
+        B, N, K = 2, 65536, 1024
+        lab = rng.integers(0, K, (B, N))
+    elif case == "small_odd":
+        B, N, K = 3, 65535, 1000  # odd length, skewed labels
+        lab = np.minimum(rng.zipf(1.2, (B, N)) - 1, K - 1)
+    elif case == "small_one":
+        B, N, K = 2, 1, 1
+        lab = np.zeros((B, N))
+    elif case == "small_33":
+        B, N, K = 2, 33, 7  # one full warp group and one lane of the next
+        lab = rng.integers(0, K, (B, N))
+    elif case == "small_reversed":
+        B, N, K = 1, 40000, 1024
+        lab = np.sort(rng.integers(0, K, (B, N)), axis=1)[:, ::-1]
+    elif case == "just_over":
+        B, N, K = 1, 65537, 1024  # one point past 2^16
         lab = rng.integers(0, K, (B, N))
     else:
         B, N, K = 2, 20000, 4096  # two 6-bit passes
