@@ -376,7 +376,8 @@ def _shift(Ca, Cb):
     return ((np.asarray(Ca, np.float64) - np.asarray(Cb, np.float64)) ** 2).sum(axis=(1, 2))
 
 
-@pytest.mark.parametrize("dt,d,K", [("f16", 128, 40), ("f32", 128, 40), ("f32", 16, 12)])
+@pytest.mark.parametrize("dt,d,K", [("f16", 128, 40), ("f32", 128, 40), ("f32", 16, 12), ("f16", 256, 40),
+                                    ("f16", 1024, 40)])
 def test_lloyd_tol_stops_when_the_centroids_settle_and_equals_plain_iterations(dt, d, K):
     w = synth.small(B=3, N=3000, d=d, K=K, dtype=dt, ncomp=K, sigma=0.2, seed=4000 + d + K)
     X = synth.points(w)

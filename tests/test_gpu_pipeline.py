@@ -27,7 +27,7 @@ def pinned(a):
     return torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
 
 
-@pytest.mark.parametrize("dtype,d", [("f16", 128), ("f32", 16), ("f32", 128)])
+@pytest.mark.parametrize("dtype,d", [("f16", 128), ("f32", 16), ("f32", 128), ("f16", 320), ("f16", 1024)])
 @pytest.mark.parametrize("chunk_rows", [0, 1500, 1000, 777])  # 0: default (one chunk per batch here)
 def test_host_pipeline_matches_device_path(dtype, d, chunk_rows):
     w = synth.small(B=2, N=3000, d=d, K=70, dtype=dtype, ncomp=70, seed=31 + d)

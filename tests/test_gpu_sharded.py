@@ -33,7 +33,7 @@ def nccl_group():
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("dt,d,K", [("f16", 128, 300), ("f32", 128, 100), ("f32", 16, 10)])
+@pytest.mark.parametrize("dt,d,K", [("f16", 128, 300), ("f32", 128, 100), ("f32", 16, 10), ("f16", 1024, 600)])
 def test_one_rank_sharded_loop_equals_lloyd(nccl_group, dt, d, K):
     w = synth.small(B=2, N=3000, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=6000 + d + K)
     X = synth.points(w)

@@ -30,7 +30,7 @@ def noalloc(X, C, labels, mindist):
                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("dtype,d", [("f16", 128), ("f16", 96), ("f32", 16)])
+@pytest.mark.parametrize("dtype,d", [("f16", 128), ("f16", 96), ("f32", 16), ("f16", 256), ("f16", 1024)])
 def test_noalloc_matches_km_assign_on_two_calls_in_a_row(dtype, d):
     w = synth.small(B=3, N=2500, d=d, K=300, dtype=dtype, seed=777 + d)
     X = torch.from_numpy(synth.points(w)).cuda()
