@@ -554,7 +554,10 @@ unsigned long long* rescan_word() {
 }
 
 km_status device_info(DeviceInfo* out) {
+    // per-device attributes, filled on first use; the lock keeps a reader from
+    // seeing an entry that another thread is still writing
     static DeviceInfo cache[64];
+    static std::mutex mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
@@ -562,6 +565,7 @@ km_status device_info(DeviceInfo* out) {
         set_error("device ordinal %d out of range", dev);
         return KM_E_UNSUPPORTED;
     }
+    std::lock_guard<std::mutex> lk(mu);
     DeviceInfo& c = cache[dev];
     if (c.device != dev) {
         DeviceInfo n;

@@ -457,24 +457,8 @@ cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float*
     P.rescans = rescan_word();
     P.stop = stop;
     P.fault = fault_word();
-    // co-resident CTA pairs (a GPC with an odd number of free SMs cannot host a whole pair)
-    static int pair_cache[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    int max_pairs = (dev >= 0 && dev < 64) ? pair_cache[dev] : 0;
-    if (max_pairs <= 0) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(sms & ~1), 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = kSmemBytes;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, (void*)assign_tf32_kernel, &cfg) != cudaSuccess || n <= 0) {
-            cudaGetLastError();
-            n = sms / 2;
-        }
-        max_pairs = n < sms / 2 ? n : sms / 2;
-        if (dev >= 0 && dev < 64) pair_cache[dev] = max_pairs;
-    }
+    static std::atomic<int> pair_cache[kMaxDevices];
+    const int max_pairs = co_resident_pairs((const void*)assign_tf32_kernel, kThreads, kSmemBytes, sms, pair_cache);
     P.pairs = P.units < max_pairs ? P.units : max_pairs;
     return launch_kernel(assign_tf32_kernel, dim3((unsigned)(2 * P.pairs)), dim3(kThreads), kSmemBytes, st, mx, mc, me,
                          P);

@@ -8,12 +8,15 @@
 
 #include <cuda.h>
 
+#include <atomic>
+
 namespace km {
 namespace ptx {
 
 // Every mbarrier wait gives up after this long (the kernel then records a
 // fault code, stops issuing work, frees its TMEM and returns).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr int kMaxDevices = 64;  // per-device host caches
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -149,19 +152,44 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
 }
 
 // ---- host side ------------------------------------------------------------------
+// CTA pairs of a cluster-of-2 kernel that can be resident at once on the
+// current device (a GPC with an odd number of free SMs cannot host a whole
+// pair), at most sms / 2.  `cache` holds one entry per device (0 = not yet
+// known); concurrent callers may both query, and store the same value.
+inline int co_resident_pairs(const void* kernel, int threads, int smem_bytes, int sms, std::atomic<int>* cache) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::atomic<int>* slot = (dev >= 0 && dev < kMaxDevices) ? cache + dev : nullptr;
+    int pairs = slot ? slot->load(std::memory_order_relaxed) : 0;
+    if (pairs > 0) return pairs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sms & ~1), 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)smem_bytes;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = sms / 2;
+    }
+    pairs = n < sms / 2 ? n : sms / 2;
+    if (slot) slot->store(pairs, std::memory_order_relaxed);
+    return pairs;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (a thread-safe static initialisation).
 inline EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return nullptr;
+    }();
     return fn;
 }
 

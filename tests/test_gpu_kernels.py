@@ -449,3 +449,47 @@ def test_scratch_pool_keeps_memory_until_released():
     assert abs(torch.cuda.mem_get_info()[0] - held) < (32 << 20)
     km.check("km_release_cached", km.lib().km_release_cached())
     assert torch.cuda.mem_get_info()[0] - held > (200 << 20)
+
+
+def test_concurrent_host_threads_on_their_own_streams_match_sequential_calls():
+    """The entry points are reentrant: host threads calling them at once, each on its own stream,
+    share the library's caches and scratch pool and get the results of the same calls made one by one."""
+    import threading
+    shapes = [(2, 3000, 100, 128, "f16"), (1, 2000, 300, 256, "f16"), (2, 1500, 50, 64, "f32"),
+              (1, 1000, 40, 1024, "f16")]
+    inputs = []
+    for i, (B, N, K, d, dt) in enumerate(shapes):
+        w = synth.small(B=B, N=N, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=9000 + i)
+        X = synth.points(w)
+        inputs.append((cuda(X), cuda(synth.init_centroids(w, X))))
+    ref = []
+    for X, C in inputs:
+        lab, C_next, _ = km.lloyd(X, C, 3)
+        torch.cuda.synchronize()
+        ref.append((lab.cpu(), C_next.cpu()))
+    out = [None] * len(inputs)
+    errors = []
+
+    def work(i):
+        try:
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                X, C = inputs[i]
+                for _ in range(4):
+                    lab, C_next, _ = km.lloyd(X, C, 3, stream=s)
+                s.synchronize()
+                out[i] = (lab.cpu(), C_next.cpu())
+        except Exception as e:  # reported below, on the test's thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=work, args=(i,)) for i in range(len(inputs))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    assert km.device_fault() == 0
+    for (lab, C_next), (ref_lab, ref_C) in zip(out, ref):
+        # the same kernels on the same inputs; only the order of fp32 atomics may differ
+        assert (lab == ref_lab).float().mean().item() > 0.999
+        torch.testing.assert_close(C_next, ref_C, rtol=1e-5, atol=1e-6)
