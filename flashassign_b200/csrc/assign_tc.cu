@@ -26,9 +26,10 @@
 //     batch; units are strided over the pairs so that pairs running at the
 //     same time share their batch's centroids in L2.
 //   * Warp roles per CTA (12 warps): warp 0 issues TMA loads (one thread:
-//     X tiles of the units into three buffers; another: centroid tiles plus
-//     their norm slices into a 3-stage ring), completing on the leader CTA's
-//     barriers; warp 1 allocates TMEM for the pair; in the leader CTA, warps
+//     X tiles of the units into two buffers; another: centroid tiles plus
+//     their norm slices into a 4-stage ring, so that with two tiles in the
+//     tensor pipe two more are in flight from L2), completing on the leader
+//     CTA's barriers; warp 1 allocates TMEM for the pair; in the leader CTA, warps
 //     1 and 10 issue the MMAs (alternate tiles) and commit them to both CTAs'
 //     barriers; warps 2..9 are the epilogue: TMEM lane = point row, two warps
 //     per row split each tile's 256 columns in 128-column slices, read in one
@@ -40,10 +41,14 @@
 //     the warp) is the group scanned for its first column equal to the
 //     maximum, which becomes the running label.  At the end of a unit each
 //     epilogue warp posts its (score, label) to a double-buffered shared slot.
-//   * Unit finish (warp 11): ||x||^2 of each row summed from the staged X
-//     tile (then the X buffer is released), the two column slices joined
-//     (larger score, then lower index), labels, mindist = ||x||^2 - 2 * best,
-//     and the objective (one atomic per unit).
+//   * Unit finish (warp 11): as soon as the unit's first tile of MMAs has
+//     completed (a commit on a per-buffer barrier), ||x||^2 of each row is
+//     summed from the staged X tile and the X buffer is released while the
+//     unit's other tiles run (two X buffers then suffice); at the unit's end
+//     the two column slices are joined (larger score, then lower index), and
+//     labels, mindist = ||x||^2 - 2 * best and the objective (one atomic per
+//     unit) are written.  Three X buffers with the release at the unit's end
+//     left room for only three centroid stages: 5% slower at K = 1024.
 //   * Measured on B200: at the 1 kW power cap the SM clock settles near
 //     1.4 GHz (K = 4096) to 1.7 GHz (K = 1024) and a tile costs ~1.1 us of
 //     wall time either way: the kernel runs at the power limit, so fewer
@@ -63,8 +68,8 @@ constexpr int kTileK = kAssignTileK;            // centroids per K tile (MMA N) 
 constexpr int kHalfTile = kTileK / 2;           // centroids staged per CTA per tile (128)
 constexpr int kBoxK = 64;                       // fp16 elements per 128-byte swizzle row
 constexpr int kMaxBoxes = 2;                    // d <= 128
-constexpr int kCStages = 3;
-constexpr int kXBufs = 3;
+constexpr int kCStages = 4;
+constexpr int kXBufs = 2;
 constexpr int kAccSets = 2;                     // 2 x 256 TMEM columns
 constexpr int kBoxBytes = 128 * 128;            // X: [128 rows x 64 fp16], 128-byte swizzled
 constexpr int kCBoxBytes = kHalfTile * 128;     // C: [128 centroids x 64 fp16], 128-byte swizzled
@@ -89,7 +94,8 @@ constexpr int kAOnesOff = kCOff + kCBytes;                          // 4 KB of o
 constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 2 halves x 128 rows x (score, label)
 constexpr int kMergeBytes = 2 * kColParts * kRows * 8;
 constexpr int kBarOff = kMergeOff + kMergeBytes;
-constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 4;  // + merge handoff (2 slots x full/empty)
+// x_full/x_empty, c_full/c_empty, acc_full/acc_empty, merge handoff (2 slots x full/empty), x_used
+constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 4 + kXBufs;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;      // + tmem slot, flag, alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA exceeded");
 static_assert(kCStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
@@ -139,6 +145,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t bar_c_full = bars + 16 * kXBufs, bar_c_empty = bar_c_full + 8 * kCStages;
     const uint32_t bar_acc_full = bar_c_empty + 8 * kCStages, bar_acc_empty = bar_acc_full + 8 * kAccSets;
     const uint32_t bar_m_full = bar_acc_empty + 8 * kAccSets, bar_m_empty = bar_m_full + 16;
+    const uint32_t bar_x_used = bar_m_empty + 16;  // a unit's first tile of MMAs has completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + kNumBars * 8 + 4);
     float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                 // [2][parts][128]
@@ -165,6 +172,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(bar_m_full + 8 * i, kEpiWarps);      // every epilogue warp has posted its half
             mbar_init(bar_m_empty + 8 * i, 1);             // the merge warp has read the slot
         }
+        for (int i = 0; i < kXBufs; ++i) mbar_init(bar_x_used + 8 * i, 1);  // the issuer of a unit's first tile
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -267,6 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                   1u);
                     umma_commit_pair(bar_c_empty + 8 * cs);
                     umma_commit_pair(bar_acc_full + 8 * s);
+                    if (kt == 0) umma_commit_pair(bar_x_used + 8 * xb);  // the unit's X tile is in place
                 }
                 if (ok) umma_commit_pair(bar_x_empty + 8 * xb);
             }
@@ -350,11 +359,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMergeWarp) {
         // ------------------------------ merge warp (both CTAs) ------------------------------
-        // Once every epilogue warp has posted unit u (so its MMAs, done with
-        // the X tile, are complete): ||x||^2 of each row from the staged tile
-        // (the swizzle permutes 16-byte chunks within a 128-byte row, so each
-        // row's bytes are all in that row), the X buffer released, the two
-        // column halves joined (larger score, then the lower index; half 0
+        // ||x||^2 of each row from the staged tile (the swizzle permutes
+        // 16-byte chunks within a 128-byte row, so each row's bytes are all in
+        // that row), then, once every epilogue warp has posted unit u, the
+        // column slices joined (larger score, then the lower index; slice 0
         // holds the lower columns), the labels, mindist and the objective.
         uint32_t it_x = 0;
         bool ok = true;
@@ -363,10 +371,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
             const uint32_t xb = it_x % kXBufs;
             const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
-            if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
             const int b = u / upb;
             const int n0 = (u - b * upb) * kUnitRows + (int)rank * kRows;
-            double obj = 0.0;
+            // ||x||^2 as soon as the unit's first tile of MMAs has completed
+            // (its X tile is then in place in both CTAs); the X buffer is
+            // released right after, while the unit's other tiles run
+            if (!(ok = mbar_wait(bar_x_used + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
+            float xn[kRows / 32];
+#pragma unroll
             for (int rq = 0; rq < kRows / 32; ++rq) {
                 const int r = rq * 32 + lane;
                 float xnorm = 0.f;
@@ -385,10 +397,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                const int n = n0 + r;
+                xn[rq] = xnorm;
                 if constexpr (kDense) {
-                    if (n < P.N) P.xnorm[(int64_t)b * P.N + n] = xnorm;
-                } else {
+                    if (n0 + r < P.N) P.xnorm[(int64_t)b * P.N + n0 + r] = xnorm;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
+            // the unit's results, once every epilogue warp has posted its column slice
+            if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
+            double obj = 0.0;
+            if constexpr (!kDense) {
+#pragma unroll
+                for (int rq = 0; rq < kRows / 32; ++rq) {
+                    const int r = rq * 32 + lane;
                     float fb = merge_score[((int)ms * kColParts) * kRows + r];
                     int fl = merge_label[((int)ms * kColParts) * kRows + r];
 #pragma unroll
@@ -401,7 +423,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             fl = ol;
                         }
                     }
-                    const float md = fmaxf(fmaf(-2.f, fb, xnorm), 0.f);
+                    const float md = fmaxf(fmaf(-2.f, fb, xn[rq]), 0.f);
+                    const int n = n0 + r;
                     if (n < P.N) {
                         const int64_t o = (int64_t)b * P.N + n;
                         P.labels[o] = fl;
@@ -411,10 +434,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar_x_empty + 8 * xb);
-                mbar_arrive(bar_m_empty + 8 * ms);
-            }
+            if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
             if (!kDense && P.obj_acc) {  // the objective of the unit's 128 rows, one atomic
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) obj += __shfl_xor_sync(0xffffffffu, obj, o);
