@@ -88,7 +88,9 @@ KM_API km_status km_assign(const void* X, const float* C, int64_t B, int64_t N, 
 
 /*
  * Label argsort (papernotes.org page, 关键设计 2: the labels alone are sorted;
- * X is never permuted).  A stable device LSD radix sort of each batch's labels:
+ * X is never permuted).  A stable device sort of each batch's labels (one
+ * launch, a thread-block cluster per batch, for N <= 65536 and K <= 1024;
+ * otherwise an LSD radix sort):
  *   sorted_idx[b][p] = index of the point at sorted position p (ascending
  *                      label, ties by ascending point index; unique),
  *   counts[b][k]     = number of points with label k,

@@ -139,7 +139,8 @@ def test_assign_single_centroid_and_far_centroids():
 
 @pytest.mark.parametrize("case", ["random", "all_equal", "k1", "sorted", "skewed", "big_k", "ragged",
                                   "one_pass_max", "one_pass_tiles", "one_pass_tail", "k4096", "long_small_k",
-                                  "small_max", "small_odd", "small_one", "small_33", "small_reversed", "just_over"])
+                                  "small_max", "small_odd", "small_one", "small_33", "small_reversed", "just_over",
+                                  "cluster_13", "cluster_tail_one", "top_bin"])
 def test_sort_is_bit_exact(case):
     rng = np.random.default_rng(13)
     B, N, K = 3, 5000, 1024
@@ -191,6 +192,17 @@ def test_sort_is_bit_exact(case):
     elif case == "just_over":
         B, N, K = 1, 65537, 1024  # one point past 2^16
         lab = rng.integers(0, K, (B, N))
+    # single-launch cluster sort: one CTA per 4096 points of a batch
+    elif case == "cluster_13":
+        B, N, K = 2, 50000, 600  # a cluster of 13 CTAs, 10-bit labels not filling their range
+        lab = rng.integers(0, K, (B, N))
+    elif case == "cluster_tail_one":
+        B, N, K = 3, 8193, 1024  # the third CTA holds one point
+        lab = rng.integers(0, K, (B, N))
+    elif case == "top_bin":
+        B, N, K = 2, 65536, 1024  # nearly every label in the last bin, a few in the first
+        lab = np.full((B, N), K - 1)
+        lab[:, rng.integers(0, N, 100)] = 0
     else:
         B, N, K = 2, 20000, 4096  # two 6-bit passes
         lab = np.minimum(rng.zipf(1.1, (B, N)) - 1, K - 1)
