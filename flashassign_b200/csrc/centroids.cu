@@ -150,40 +150,51 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(
     const float inv = n > 0 ? 1.0f / (float)n : 0.f;  // the mean as s * (1/n): within 1 ulp of s / n
     const int64_t base = row * d;
     double acc = 0.0, moved = 0.0;
+    constexpr int kAhead = 4;  // float4 steps of a row loaded before any is stored
     if (valid) {
-        for (int64_t j = 4 * sub; j < d; j += 4 * kFinLanes) {
-            // the sums are read whatever the count (zero for an empty cluster), so the
-            // load does not wait for the offsets
-            const float4 sv = *reinterpret_cast<const float4*>(sums + base + j);
-            float4 v;
-            if (n > 0) {
-                v = make_float4(sv.x * inv, sv.y * inv, sv.z * inv, sv.w * inv);
-                if (shift) {  // this centroid's squared shift
-                    const float4 o = *reinterpret_cast<const float4*>(C_out + base + j);
-                    const double dx = (double)v.x - o.x, dy = (double)v.y - o.y, dz = (double)v.z - o.z,
-                                 dw = (double)v.w - o.w;
-                    moved += dx * dx + dy * dy + dz * dz + dw * dw;
+        for (int64_t j0 = 4 * sub; j0 < d; j0 += kAhead * 4 * kFinLanes) {
+            // The loads of a group are issued together: the stores below go through
+            // pointers the compiler cannot separate from these, so a load after a
+            // store would wait for it.  An empty cluster keeps its centroid.
+            float4 sv[kAhead];
+#pragma unroll
+            for (int u = 0; u < kAhead; ++u) {
+                const int64_t j = j0 + (int64_t)u * 4 * kFinLanes;
+                if (j < d) sv[u] = *reinterpret_cast<const float4*>((n > 0 ? sums : C_out) + base + j);
+            }
+#pragma unroll
+            for (int u = 0; u < kAhead; ++u) {
+                const int64_t j = j0 + (int64_t)u * 4 * kFinLanes;
+                if (j >= d) break;
+                float4 v = sv[u];
+                if (n > 0) {
+                    v = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+                    if (shift) {  // this centroid's squared shift
+                        const float4 o = *reinterpret_cast<const float4*>(C_out + base + j);
+                        const double dx = (double)v.x - o.x, dy = (double)v.y - o.y, dz = (double)v.z - o.z,
+                                     dw = (double)v.w - o.w;
+                        moved += dx * dx + dy * dy + dz * dz + dw * dw;
+                    }
+                    *reinterpret_cast<float4*>(C_out + base + j) = v;
+                    if (zero_sums) *reinterpret_cast<float4*>(sums + base + j) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                *reinterpret_cast<float4*>(C_out + base + j) = v;
-                if (zero_sums) *reinterpret_cast<float4*>(sums + base + j) = make_float4(0.f, 0.f, 0.f, 0.f);
-            } else {
-                v = *reinterpret_cast<const float4*>(C_out + base + j);
+                if (!next.cext) continue;
+                if (dtype == KM_F16) {
+                    const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+                    __half* chat = static_cast<__half*>(next.chat);
+                    *reinterpret_cast<__half2*>(chat + base + j) = h01;
+                    *reinterpret_cast<__half2*>(chat + base + j + 2) = h23;
+                    const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+                    v = make_float4(f01.x, f01.y, f23.x, f23.y);
+                } else {
+                    float* row2 = static_cast<float*>(next.chat) + 2 * base;
+                    const float4 hv = make_float4(tf32_head(v.x), tf32_head(v.y), tf32_head(v.z), tf32_head(v.w));
+                    *reinterpret_cast<float4*>(row2 + j) = hv;
+                    *reinterpret_cast<float4*>(row2 + d + j) =
+                        make_float4(v.x - hv.x, v.y - hv.y, v.z - hv.z, v.w - hv.w);
+                }
+                acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
             }
-            if (!next.cext) continue;
-            if (dtype == KM_F16) {
-                const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
-                __half* chat = static_cast<__half*>(next.chat);
-                *reinterpret_cast<__half2*>(chat + base + j) = h01;
-                *reinterpret_cast<__half2*>(chat + base + j + 2) = h23;
-                const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-                v = make_float4(f01.x, f01.y, f23.x, f23.y);
-            } else {
-                float* row2 = static_cast<float*>(next.chat) + 2 * base;
-                const float4 hv = make_float4(tf32_head(v.x), tf32_head(v.y), tf32_head(v.z), tf32_head(v.w));
-                *reinterpret_cast<float4*>(row2 + j) = hv;
-                *reinterpret_cast<float4*>(row2 + d + j) = make_float4(v.x - hv.x, v.y - hv.y, v.z - hv.z, v.w - hv.w);
-            }
-            acc += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
         }
     }
     if (next.cext) {
