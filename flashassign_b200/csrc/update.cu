@@ -16,9 +16,11 @@
 //   slice per grid z (the same positions in every slice), so a CTA covers W = d
 //   or W = 1024 / sizeof(T) dimensions of each row;
 //   tpr = W * sizeof(T) / 16 threads cover one row; G = 256 / tpr row-lanes;
-//   row-lane g walks 16 consecutive sorted positions (B_N = 16 G), issuing
-//   four independent 16-byte gathers at a time and keeping a running fp32
-//   partial sum in registers.  A label change inside the walk ends a piece:
+//   row-lane g walks 32 consecutive sorted positions (B_N = 32 G); each
+//   thread streams its 16-byte chunk of the walk's rows through a ring of
+//   four asynchronous copies in shared memory (so the bytes in flight cost
+//   no registers) and keeps a running fp32 partial sum in registers.  A label
+//   change inside the walk ends a piece:
 //   pieces strictly inside the walk are whole clusters and are stored at once;
 //   the first and last piece of each walk go to shared memory, where one pass
 //   in position order joins equal labels across row-lanes and decides, from
@@ -32,8 +34,31 @@
 namespace km {
 namespace {
 
-constexpr int kRowsPerLane = 16;
-constexpr int kUnroll = 4;
+constexpr int kRowsPerLane = 32;
+constexpr int kRing = 4;  // row chunks in flight per thread (a shared-memory ring, not registers)
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t smem_u32addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+// 0, computed from v: an instruction that must wait for v, placed before a
+// copy that reuses v's ring slot
+__device__ __forceinline__ int zero_after(const uint4& v) {
+    int z;
+    asm volatile("and.b32 %0, %1, 0;" : "=r"(z) : "r"(v.x));
+    return z;
+}
 
 template <typename T>
 struct Chunk;
@@ -63,10 +88,11 @@ struct Chunk<float> {
 
 // kSliced: rows are cut into slices of W dimensions along grid z; otherwise a
 // CTA covers whole rows (W = d) and every slice term folds away at compile time.
-// The gathers are latency-bound, so the number of resident warps sets the
-// bandwidth: the whole-row form compiles to 48 registers (five CTAs per SM);
-// folding the slice terms in at run time cost it four registers, one CTA per
-// SM and 17% of its speed at d = 128.
+// The gathers are latency-bound: resident warps and bytes in flight set the
+// bandwidth.  At d = 128 (fp16) the whole-row form takes 40 registers and
+// 36 KB of shared memory, six CTAs per SM; rings of 2 or 8 slots, or walks of
+// 16 or 64 rows, measured slower.  Folding the slice terms in at run time
+// (register-held gathers then) cost four registers, one CTA per SM and 17%.
 template <typename T, bool kSliced>
 __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, const int32_t* __restrict__ a_sorted,
                                                      const int32_t* __restrict__ sorted_idx, int64_t N, int64_t K,
@@ -86,6 +112,8 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
     int* s_idx = s_lab + BN;                             // [BN]
     int* head_lab = s_idx + BN;                          // [G]
     int* tail_lab = head_lab + G;                        // [G]
+    // [kRing][threads] 16-byte slots: slot i of thread t at ring0 + (i * threads + t) * 16
+    const uint32_t ring0 = (smem_u32addr(tail_lab + G) + 15u) & ~15u;
 
     const int64_t b = blockIdx.y;
     const int64_t z0 = kSliced ? (int64_t)blockIdx.z * W : 0;  // first dimension of this slice
@@ -127,15 +155,24 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
         for (int e = 0; e < E; ++e) acc[e] = 0.f;
         int cur = s_lab[r0];
         int piece = 0;
-        for (int r = r0; r < r1; r += kUnroll) {
-            uint4 v[kUnroll];
+        // The walk's rows stream through a ring of kRing 16-byte slots per
+        // thread (asynchronous copies, one commit group per row, empty past
+        // the walk's end): the chunks in flight cost shared memory, not registers.
+        const uint32_t slot_stride = blockDim.x * 16u;
+        const uint32_t ring = ring0 + threadIdx.x * 16u;
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u)
-                if (r + u < r1) v[u] = __ldg(reinterpret_cast<const uint4*>(xb + (int64_t)s_idx[r + u] * d));
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                if (r + u >= r1) break;
-                const int lab = s_lab[r + u];
+        for (int i = 0; i < kRing; ++i) {
+            if (r0 + i < r1) cp_async16(ring + i * slot_stride, xb + (int64_t)s_idx[r0 + i] * d);
+            cp_async_commit();
+        }
+        for (int r = r0; r < r1; ++r) {
+            cp_async_wait<kRing - 1>();  // row r's group has landed
+            const uint32_t slot = ring + (uint32_t)((r - r0) & (kRing - 1)) * slot_stride;
+            const uint4 vr = lds128(slot);
+            if (r + kRing < r1) cp_async16(slot, xb + ((int64_t)s_idx[r + kRing] + zero_after(vr)) * d);
+            cp_async_commit();
+            {
+                const int lab = s_lab[r];
                 if (lab != cur) {
                     if (piece == 0) {
                         if (c == 0) head_lab[g] = cur;
@@ -158,9 +195,10 @@ __global__ void __launch_bounds__(256) update_kernel(const T* __restrict__ X, co
                     for (int e = 0; e < E; ++e) acc[e] = 0.f;
                     cur = lab;
                 }
-                Chunk<T>::add(acc, v[u]);
+                Chunk<T>::add(acc, vr);
             }
         }
+        cp_async_wait<0>();
         if (piece == 0) {  // the whole walk is one label: a head piece with no tail
             if (c == 0) {
                 head_lab[g] = cur;
@@ -227,7 +265,8 @@ cudaError_t launch_t(const void* X, const int32_t* a_sorted, const int32_t* sort
     const int tpr = (int)(W * (int64_t)sizeof(T) / 16);                                 // <= 64
     const int G = 256 / tpr;                                                              // >= 4
     const int BN = G * kRowsPerLane;
-    const size_t smem = sizeof(float) * 2 * (size_t)G * W + sizeof(int) * (2 * (size_t)BN + 2 * (size_t)G);
+    const size_t smem = sizeof(float) * 2 * (size_t)G * W + sizeof(int) * (2 * (size_t)BN + 2 * (size_t)G) + 16 +
+                        (size_t)kRing * (size_t)(G * tpr) * 16;
     const bool sliced = W != d;
     void (*kernel)(const T*, const int32_t*, const int32_t*, int64_t, int64_t, int64_t, int64_t, int, int, float*,
                    int32_t*, int, const int32_t*) = sliced ? update_kernel<T, true> : update_kernel<T, false>;
