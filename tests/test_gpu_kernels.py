@@ -295,6 +295,29 @@ def test_lloyd_many_iterations_equal_one_at_a_time():
     np.testing.assert_allclose(obj6.cpu().numpy(), torch.cat(objs).cpu().numpy(), rtol=1e-5)
 
 
+@pytest.mark.parametrize("B,N,K,launches", [(32, 65536, 1024, 1), (3, 4097, 8, 1), (2, 65537, 1024, 6),
+                                            (2, 20000, 2048, 6)])
+def test_sort_path_by_shape(B, N, K, launches):
+    """Batches of at most 65,536 labels below 1024 are sorted in one launch (a thread-block cluster per
+    batch); longer batches or wider labels take the radix passes (a histogram and a scatter per pass)
+    plus the boundary and count kernels.  Both give the oracle's bit-exact result."""
+    rng = np.random.default_rng(B * N + K)
+    lab = rng.integers(0, K, (B, N)).astype(np.int32)
+    g = cuda(lab)
+    km.sort_labels(g, K)
+    torch.cuda.synchronize()
+    km.trace_enable(True)
+    try:
+        km.trace_read()
+        sidx, counts, offsets = km.sort_labels(g, K)
+        torch.cuda.synchronize()
+        rec = km.trace_read()
+    finally:
+        km.trace_enable(False)
+    assert rec["sort"][1] == launches
+    check_sort(lab, K, sidx.cpu().numpy(), counts.cpu().numpy(), offsets.cpu().numpy())
+
+
 def test_labels_counts_and_sort_are_deterministic():
     w = synth.small(B=2, N=5000, d=128, K=200, dtype="f16", seed=22)
     X = cuda(synth.points(w))
