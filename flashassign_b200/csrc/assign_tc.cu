@@ -24,7 +24,10 @@
 //     Two 256-column accumulator sets fill the 512 TMEM columns.
 //   * Persistent grid of pairs; a work unit is 256 consecutive points of one
 //     batch; units are strided over the pairs so that pairs running at the
-//     same time share their batch's centroids in L2.
+//     same time share their batch's centroids in L2.  When a batch's tiles
+//     fit the ring one per stage (an even count, at most four: K in
+//     (256, 512] or (768, 1024]) they stay resident over a pair's run of units
+//     in one batch instead of being reloaded for every unit (4% at K = 1024).
 //   * Warp roles per CTA (12 warps): warp 0 issues TMA loads (one thread:
 //     X tiles of the units into two buffers; another: centroid tiles plus
 //     their norm slices into a 4-stage ring, so that with two tiles in the
@@ -117,6 +120,7 @@ struct Params {
     int64_t B, N, K, d;
     int64_t units_per_batch, units, pairs;
     int ktiles, ksteps, boxes;
+    int resident;  // the batch's centroid tiles stay in the ring across the units of a batch (see the producer)
     int32_t* labels;
     float* mindist;
     double* obj_acc;  // [B] running sum of minimum distances, nullable
@@ -221,13 +225,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tma_load_pair(x_base + (xb * kMaxBoxes + kb) * kBoxBytes, &tmap_x, kb * kBoxK, n0, b, xfull_leader);
             }
         } else if (lane == 0) {
-            uint32_t it_c = 0;
+            // Resident mode (an even number of tiles, at most one per stage): tile
+            // kt of the batch lives in stage kt and is loaded once per run of the
+            // pair's units in one batch (an epoch), not once per unit; a stage is
+            // refilled after the epoch's last MMA on it, so a batch change still
+            // streams tile by tile.
+            uint32_t it_c = 0, ep = 0;
+            int prev_b = -1;
             bool ok = true;
             for (int64_t u = pair; u < n_units && ok; u += P.pairs) {
                 const int b = (int)(u / P.units_per_batch);
+                if (P.resident) {
+                    if (b == prev_b) continue;  // this batch's tiles are in place
+                    if (prev_b >= 0) ++ep;
+                    prev_b = b;
+                }
                 for (int kt = 0; kt < P.ktiles; ++kt, ++it_c) {
-                    const uint32_t cs = it_c % kCStages;
-                    if (!(ok = mbar_wait(bar_c_empty + 8 * cs, ((it_c / kCStages) & 1) ^ 1, abort_flag, P.fault)))
+                    const uint32_t cs = P.resident ? (uint32_t)kt : it_c % kCStages;
+                    const uint32_t epar = P.resident ? (ep & 1) ^ 1 : ((it_c / kCStages) & 1) ^ 1;
+                    if (!(ok = mbar_wait(bar_c_empty + 8 * cs, epar, abort_flag, P.fault)))
                         break;
                     if (rank == 0) mbar_expect_tx(bar_c_full + 8 * cs, c_bytes_pair);
                     const uint32_t cfull_leader = map_to_rank(bar_c_full + 8 * cs, 0);
@@ -247,17 +263,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // C stage is only ever used by one of them (4 stages, 2 issuers).
         const uint32_t mine = warp == 1 ? 0u : 1u;
         if (rank == 0 && lane == 0) {
-            uint32_t it_x = 0, it_c = 0, it_a = 0;
+            uint32_t it_x = 0, it_c = 0, it_a = 0, ep = 0;
+            int prev_b = -1;
             bool ok = true;
             for (int64_t u = pair; u < n_units && ok; u += P.pairs, ++it_x) {
                 const uint32_t xb = it_x % kXBufs;
+                const int b = (int)(u / P.units_per_batch);
+                if (P.resident && b != prev_b) {
+                    if (prev_b >= 0) ++ep;
+                    prev_b = b;
+                }
+                // resident mode: the stages are released only after the epoch's last unit
+                // (with an even tile count each stage has one issuer, whose commit covers
+                // all of its earlier MMAs on that stage)
+                const bool release_c =
+                    !P.resident || u + P.pairs >= n_units || (int)((u + P.pairs) / P.units_per_batch) != b;
                 if (!(ok = mbar_wait(bar_x_full + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
                 const uint64_t a_desc0 = umma_desc_sw128(x_base + xb * kMaxBoxes * kBoxBytes);
                 for (int kt = 0; kt < P.ktiles; ++kt, ++it_c, ++it_a) {
                     if ((it_a & 1u) != mine) continue;
-                    const uint32_t cs = it_c % kCStages;
+                    const uint32_t cs = P.resident ? (uint32_t)kt : it_c % kCStages;
                     const uint32_t s = it_a % kAccSets;
-                    if (!(ok = mbar_wait(bar_c_full + 8 * cs, (it_c / kCStages) & 1, abort_flag, P.fault))) break;
+                    const uint32_t fpar = P.resident ? (ep & 1) : (it_c / kCStages) & 1;
+                    if (!(ok = mbar_wait(bar_c_full + 8 * cs, fpar, abort_flag, P.fault))) break;
                     if (!(ok = mbar_wait(bar_acc_empty + 8 * s, ((it_a / kAccSets) & 1) ^ 1, abort_flag, P.fault)))
                         break;
                     tc_fence_after();
@@ -273,7 +301,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     // the norm slice: ones (points) x (-||c||^2/2 pieces) (centroids)
                     umma_pair_f16(d_tmem, umma_desc_sw32(ones_base), umma_desc_sw32(stage + kMaxBoxes * kCBoxBytes),
                                   1u);
-                    umma_commit_pair(bar_c_empty + 8 * cs);
+                    if (release_c) umma_commit_pair(bar_c_empty + 8 * cs);
                     umma_commit_pair(bar_acc_full + 8 * s);
                     if (kt == 0) umma_commit_pair(bar_x_used + 8 * xb);  // the unit's X tile is in place
                 }
@@ -481,6 +509,7 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
     P.ktiles = (int)ceil_div(K, kTileK);
     P.ksteps = (int)ceil_div(d, 16);
     P.boxes = (int)ceil_div(d, kBoxK);
+    P.resident = (P.ktiles % 2 == 0 && P.ktiles <= kCStages) ? 1 : 0;
     P.labels = labels;
     P.mindist = mindist;
     P.obj_acc = obj_acc;

@@ -39,6 +39,8 @@ ASSIGN_SHAPES = [
     (2, 256, 129, 128, "f16"),
     (2, 257, 255, 128, "f16"),
     (3, 1000, 300, 128, "f16"),
+    (2, 20000, 1000, 128, "f16"),  # four centroid tiles kept in the ring over a pair's units of one batch
+    (40, 1000, 500, 128, "f16"),   # two resident tiles, reloaded as a pair's units change batch
     (2, 777, 257, 64, "f16"),
     (2, 600, 200, 96, "f16"),
     (2, 500, 100, 16, "f16"),    # below the tensor-core range: CUDA-core kernel
