@@ -562,10 +562,9 @@ bool use_cluster_sort(int64_t N, int64_t K) {
     int total = 1;
     while (total < 31 && (int64_t(1) << total) < K) ++total;
     if (total > kCsMaxBits) return false;
-    constexpr int kDevices = 64;  // devices with a cached answer; others take the radix path
-    static std::atomic<int> state[kDevices];  // per device: 0 not yet known, 1 usable, 2 not usable
+    static std::atomic<int> state[64];  // per device: 0 not yet known, 1 usable, 2 not usable
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return false;
     }
