@@ -369,7 +369,8 @@ def test_injected_allocation_failure_is_reported_and_leaks_nothing(monkeypatch):
 
 # ---- the baselines the method replaces (measurement only) ----
 
-@pytest.mark.parametrize("B,N,K,d", [(2, 1000, 300, 128), (1, 129, 127, 64), (2, 257, 255, 96), (3, 511, 513, 128)])
+@pytest.mark.parametrize("B,N,K,d", [(2, 1000, 300, 128), (1, 129, 127, 64), (2, 257, 255, 96), (3, 511, 513, 128),
+                                     (4, 20000, 1000, 128)])  # resident centroid tiles over several units per pair
 def test_dense_assign_baseline_matches_the_fused_kernel_and_the_oracle(B, N, K, d):
     w = synth.small(B=B, N=N, d=d, K=K, dtype="f16", ncomp=max(1, K // 2), sigma=0.3, seed=2000 + N + K)
     X = synth.points(w)
