@@ -52,6 +52,9 @@ def _load():
         lib.oracle_cost.argtypes = [_P, ctypes.c_int, _P, _P, _I, _I, _I, _I, _P]
         lib.oracle_lloyd.restype = ctypes.c_int
         lib.oracle_lloyd.argtypes = [_P, ctypes.c_int, _P, _I, _I, _I, _I, ctypes.c_int, _P, _P, _P, ctypes.c_int]
+        lib.oracle_lloyd_tol.restype = ctypes.c_int
+        lib.oracle_lloyd_tol.argtypes = [_P, ctypes.c_int, _P, _I, _I, _I, _I, ctypes.c_int, ctypes.c_double, _P, _P,
+                                         _P, _P, _P, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -185,3 +188,27 @@ def lloyd(X: np.ndarray, C_init: np.ndarray, iters: int, nthreads: int | None = 
     if rc:
         raise ValueError(f"oracle_lloyd failed ({rc})")
     return labels, C_out, obj
+
+
+def lloyd_tol(X: np.ndarray, C_init: np.ndarray, max_iters: int, tol: float, nthreads: int | None = None):
+    """Lloyd iterations until every batch's squared centroid shift is <= tol (or max_iters).
+
+    Returns (iters_run, labels of the last assignment, final C, objective [iters_run, B],
+    shift [iters_run, B]).
+    """
+    X = _c(X)
+    B, N, d = X.shape
+    K = C_init.shape[1]
+    C_init = _c(C_init, np.float32)
+    labels = np.empty((B, N), dtype=np.int32)
+    C_out = np.empty_like(C_init)
+    obj = np.empty((max_iters, B), dtype=np.float64)
+    shift = np.empty((max_iters, B), dtype=np.float64)
+    run = np.zeros(1, dtype=np.int32)
+    rc = _load().oracle_lloyd_tol(X.ctypes.data, _dtype_code(X), C_init.ctypes.data, B, N, K, d, max_iters,
+                                  float(tol), labels.ctypes.data, C_out.ctypes.data, obj.ctypes.data,
+                                  run.ctypes.data, shift.ctypes.data, nthreads or threads())
+    if rc:
+        raise ValueError(f"oracle_lloyd_tol failed ({rc})")
+    t = int(run[0])
+    return t, labels, C_out, obj[:t], shift[:t]

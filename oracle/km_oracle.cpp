@@ -284,4 +284,52 @@ int oracle_lloyd(const void* X, int dtype, const float* C_init, int64_t B, int64
     return 0;
 }
 
+// Lloyd iterations until convergence (papernotes.org page, 整体框架 flowchart:
+// after each update, "converged?" either ends the loop or returns to the
+// assignment).  The pages give no test; the reading taken: after iteration t,
+// every batch's squared centroid shift shift_b = sum_k ||C_{t+1,k} - C_{t,k}||^2
+// (fp32 centroids, summed in double; an empty cluster keeps its centroid and
+// so does not move) is compared with tol, and the loop ends after the first
+// iteration at which shift_b <= tol holds for every batch, or after max_iters.
+// *iters_run = the number of iterations performed; labels, C_out and the
+// objective rows [0, *iters_run) are those of oracle_lloyd with that count;
+// shift[t * B + b] (nullable, [max_iters, B]) = shift_b of iteration t.
+int oracle_lloyd_tol(const void* X, int dtype, const float* C_init, int64_t B, int64_t N, int64_t K, int64_t d,
+                     int max_iters, double tol, int32_t* labels, float* C_out, double* objective, int32_t* iters_run,
+                     double* shift, int nthreads) {
+    if (!X || !C_init || !labels || !C_out || !iters_run || max_iters < 1) return 1;
+    std::vector<float> C(C_init, C_init + B * K * d), Cn(B * K * d);
+    std::vector<double> chat(B * K * d), d1(B * N);
+    int t = 0;
+    bool settled = false;
+    while (t < max_iters && !settled) {
+        oracle_round_centroids(C.data(), dtype, B * K * d, chat.data());
+        int rc = oracle_assign(X, dtype, chat.data(), B, N, K, d, nullptr, 0, labels, d1.data(), nullptr, nthreads);
+        if (rc) return rc;
+        if (objective)
+            for (int64_t b = 0; b < B; ++b) {
+                double j = 0.0;
+                for (int64_t i = 0; i < N; ++i) j += d1[b * N + i];
+                objective[t * B + b] = j;
+            }
+        rc = oracle_update(X, dtype, labels, B, N, K, d, C.data(), Cn.data(), nullptr, nullptr, nthreads);
+        if (rc) return rc;
+        settled = true;
+        for (int64_t b = 0; b < B; ++b) {
+            double sb = 0.0;
+            for (int64_t e = b * K * d; e < (b + 1) * K * d; ++e) {
+                const double diff = static_cast<double>(Cn[e]) - static_cast<double>(C[e]);
+                sb += diff * diff;
+            }
+            if (shift) shift[t * B + b] = sb;
+            if (!(sb <= tol)) settled = false;
+        }
+        C.swap(Cn);
+        ++t;
+    }
+    *iters_run = t;
+    std::memcpy(C_out, C.data(), sizeof(float) * B * K * d);
+    return 0;
+}
+
 }  // extern "C"

@@ -217,6 +217,45 @@ def test_hand_worked_examples(dt):
         assert np.array_equal(C_end, C)
 
 
+@pytest.mark.parametrize("dt", [np.float32, np.float16])
+def test_convergence_stopping_follows_the_hand_worked_shifts(dt):
+    spec = json.load(open(GOLDEN))
+    examples = {ex["name"]: ex for ex in spec["examples"]}
+    for case in spec["stopping"]["cases"]:
+        ex = examples[case["example"]]
+        X = np.array(ex["X"], dtype=np.float64)[None].astype(dt)
+        C0 = np.array(ex["C0"], dtype=np.float32)[None]
+        want = [float(Fraction(v)) for v in case["shifts"]]
+        for run in case["runs"]:
+            tol = float(Fraction(run["tol"]))
+            t, lab, C, obj, shift = oracle.lloyd_tol(X, C0, run["max_iters"], tol)
+            assert t == run["iters_run"], (case["example"], run, t)
+            # the shifts of the iterations run (centroids are fp32: 20/3 is rounded)
+            for i in range(t):
+                assert abs(shift[i, 0] - want[i]) <= 1e-6 * max(1.0, want[i]), (case["example"], i, shift[i, 0])
+            # and the state is that of the plain loop run for the same number of iterations
+            lab_p, C_p, obj_p = oracle.lloyd(X, C0, t)
+            assert np.array_equal(lab, lab_p) and np.array_equal(C, C_p) and np.array_equal(obj, obj_p)
+
+
+def test_convergence_stopping_waits_for_every_batch_and_respects_the_cap():
+    # two batches: the first settles after 2 iterations (the 2-d square), the second after 3
+    # (the 1-d clusters, embedded in 2-d with a zero coordinate); the loop stops for both at 3
+    Xa = np.array([[0, 0], [0, 2], [4, 0], [4, 2]], dtype=np.float32)
+    Xb = np.array([[0, 0], [1, 0], [9, 0], [10, 0]], dtype=np.float32)
+    X = np.stack([Xa, Xb])
+    C0 = np.stack([Xa[[0, 1]], Xb[[0, 1]]]).astype(np.float32)
+    t, lab, C, obj, shift = oracle.lloyd_tol(X, C0, 10, 0.0)
+    assert t == 3
+    assert shift[1, 0] == 0.0 and shift[1, 1] > 0.0 and (shift[2] == 0.0).all()
+    t, *_ = oracle.lloyd_tol(X, C0, 2, 0.0)
+    assert t == 2
+    # a negative tolerance is never met: the loop runs to the cap, like the plain loop
+    t, lab, C, obj, shift = oracle.lloyd_tol(X, C0, 4, -1.0)
+    lab_p, C_p, obj_p = oracle.lloyd(X, C0, 4)
+    assert t == 4 and np.array_equal(lab, lab_p) and np.array_equal(C, C_p)
+
+
 def test_lloyd_reaches_the_global_optimum_on_separable_data():
     # three tight, far-apart groups; from one seed point per group, Lloyd's
     # fixed point is the optimal 3-partition, which enumeration finds exactly.
