@@ -20,6 +20,7 @@ STATUS = {0: "KM_OK", 1: "KM_E_INVALID", 2: "KM_E_UNSUPPORTED", 3: "KM_E_NOMEM",
 _P, _I64, _INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 SIGNATURES = {
     "km_assign": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P]),
+    "km_assign_objective": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P, _P]),
     "km_sort_labels": (_INT, [_P, _I64, _I64, _I64, _P, _P, _P, _P]),
     "km_update": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _P, _P, _P, _P]),
     "km_lloyd": (_INT, [_P, _P, _I64, _I64, _I64, _I64, _INT, _INT, _P, _P, _P, _P]),
@@ -120,6 +121,23 @@ def assign(X, C, labels=None, mindist=None, stream=None):
     check("km_assign", lib().km_assign(_ptr(X), _ptr(C), B, N, K, d, _dtype_code(X), _ptr(labels), _ptr(mindist),
                                        _stream(stream)))
     return labels, mindist
+
+
+def assign_objective(X, C, labels=None, mindist=None, stream=None):
+    """assign() plus the per-problem objective sum_i mindist (fp64 [B]) from the assignment kernels."""
+    torch = _torch()
+    B, N, d = X.shape
+    K = C.shape[1]
+    _require(C, (B, K, d), torch.float32, "C")
+    if labels is None:
+        labels = torch.empty((B, N), dtype=torch.int32, device=X.device)
+    if mindist is None:
+        mindist = torch.empty((B, N), dtype=torch.float32, device=X.device)
+    objective = torch.empty(B, dtype=torch.float64, device=X.device)
+    check("km_assign_objective", lib().km_assign_objective(_ptr(X), _ptr(C), B, N, K, d, _dtype_code(X),
+                                                           _ptr(labels), _ptr(mindist), _ptr(objective),
+                                                           _stream(stream)))
+    return labels, mindist, objective
 
 
 def assign_dense(X, C, labels=None, mindist=None, stream=None):
@@ -251,7 +269,7 @@ def device_fault(stream=None) -> int:
 
 
 def assign_rescans(stream=None) -> int:
-    """Read and clear the count of fp32 points handed to the exact re-scan (see include/km.h)."""
+    """Read and clear the count of points handed to the exact re-scan (see include/km.h)."""
     n = ctypes.c_int64(0)
     check("km_assign_rescans", lib().km_assign_rescans(ctypes.byref(n), _stream(stream)))
     return int(n.value)

@@ -7,11 +7,12 @@
 //   * dense_argmin_kernel: the second half of the dense assignment -- reads
 //     the score matrix that the tensor-core kernel wrote in its dense mode
 //     (s = x.c - ||c||^2/2, [B, padded K, N] fp32) and takes each point's
-//     argmax (lowest index among equal scores), mindist = ||x||^2 - 2 s.
+//     argmax (lowest index among equal scores), mindist = ||x||^2 - 2 s, with
+//     the fused kernel's certification and exact re-scan of the rest.
 //   * scatter_update_kernel: one thread per (point, coordinate), an fp32
 //     atomic addition into the cluster's sum per coordinate and an integer
 //     one per point into its count: B*N*d + B*N atomics.
-#include "km_internal.cuh"
+#include "certify.cuh"
 
 namespace km {
 namespace {
@@ -19,31 +20,34 @@ namespace {
 constexpr int kArgminThreads = 256;
 
 // One thread per point: column k of the scores is D[b][k][0..N), so the warp's
-// loads of one column are consecutive.  Strict > over ascending k keeps the
-// lowest index among equal scores.
+// loads of one column are consecutive.  The best score (strict > over
+// ascending k keeps the lowest index among equal scores) is certified as in
+// the fused kernel; the rest go to the re-scan list.
 __global__ void __launch_bounds__(kArgminThreads) dense_argmin_kernel(const float* __restrict__ D,
                                                                       const float* __restrict__ xnorm, int64_t N,
                                                                       int64_t K, int64_t Kp,
                                                                       int32_t* __restrict__ labels,
-                                                                      float* __restrict__ mindist) {
+                                                                      float* __restrict__ mindist, RescanList list) {
     pdl_trigger();
     pdl_wait();
     const int64_t b = blockIdx.y;
     const int64_t n = (int64_t)blockIdx.x * kArgminThreads + threadIdx.x;
-    if (n >= N) return;
-    const float* d = D + b * Kp * N + n;
+    const bool valid = n < N;  // every lane stays for the warp-wide listing
     float best = -INFINITY;
     int idx = -1;
+    if (valid) {
+        const float* d = D + b * Kp * N + n;
 #pragma unroll 8
-    for (int64_t k = 0; k < K; ++k) {
-        const float v = d[k * N];
-        if (v > best) {
-            best = v;
-            idx = (int)k;
+        for (int64_t k = 0; k < K; ++k) {
+            const float v = d[k * N];
+            if (v > best) {
+                best = v;
+                idx = (int)k;
+            }
         }
     }
-    labels[b * N + n] = idx;
-    if (mindist) mindist[b * N + n] = fmaxf(fmaf(-2.f, best, xnorm[b * N + n]), 0.f);
+    certify_best(list, list.cmax[b], b, N, n, valid, best, idx, valid ? xnorm[b * N + n] : 0.f, labels, mindist,
+                      threadIdx.x & 31);
 }
 
 template <typename T>
@@ -72,9 +76,10 @@ __global__ void __launch_bounds__(256) scatter_update_kernel(const T* __restrict
 }  // namespace
 
 cudaError_t launch_dense_argmin(const float* D, const float* xnorm, int64_t B, int64_t N, int64_t K, int32_t* labels,
-                                float* mindist, cudaStream_t st) {
+                                float* mindist, const RescanList& list, cudaStream_t st) {
+    if (!list.cmax || !list.count || !list.rows) return cudaErrorInvalidValue;
     return launch_kernel(dense_argmin_kernel, dim3((unsigned)ceil_div(N, kArgminThreads), (unsigned)B),
-                         dim3(kArgminThreads), 0, st, D, xnorm, N, K, padded_k(K), labels, mindist);
+                         dim3(kArgminThreads), 0, st, D, xnorm, N, K, padded_k(K), labels, mindist, list);
 }
 
 cudaError_t launch_scatter_update(const void* X, int dtype, const int32_t* labels, int64_t B, int64_t N, int64_t K,

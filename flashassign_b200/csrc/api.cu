@@ -195,97 +195,122 @@ bool uses_tc(int dtype, int64_t d) {
                            : assign_tf32_supported(d);
 }
 
-// Scratch of a tensor-core assignment: the prepared centroids and, for fp32,
-// the per-batch list of points left to the exact re-scan.
+// Scratch of a tensor-core assignment: the prepared centroids and the lists of
+// points left to the exact re-scan.  The list counters come in two sets of
+// `lists` entries used in turn: an assignment appends to one set while its
+// re-scan zeroes the other, ready for the next assignment, so that no memset
+// sits between the kernels of an iteration.
 struct TcScratch {
     PreparedC prep;
-    int32_t* flag_count = nullptr;  // [B]
-    int32_t* flag_rows = nullptr;   // [B, list_rows / B]
-    // batch b alone (the chunk pipeline assigns one batch at a time; its list
-    // and counter serve every chunk in turn)
+    int32_t* flag_count = nullptr;  // [2, lists]
+    int32_t* flag_rows = nullptr;   // [lists, cap]
+    int64_t lists = 0, cap = 0;
+    int parity = 0;                 // the counter set the next assignment appends to
+    // batch b alone: its prepared centroids; the chunk pipeline (one batch at a
+    // time, lists == 1) keeps the single list, which serves every chunk in turn
     TcScratch batch(int64_t b, int64_t K, int64_t d, int dtype) const {
         TcScratch t = *this;
         const int64_t Kp = padded_k(K);
         if (dtype == KM_F16) {
             t.prep.chat = static_cast<__half*>(prep.chat) + b * K * d;
-            t.prep.cext = static_cast<__half*>(prep.cext) + b * Kp * 16;
+            t.prep.cext = static_cast<__half*>(prep.cext) + b * Kp * kNormPieces;
         } else {
             t.prep.chat = static_cast<float*>(prep.chat) + b * K * 2 * d;
             t.prep.cext = static_cast<float*>(prep.cext) + b * Kp * 8;
-            t.prep.cmax = prep.cmax + b;
         }
+        t.prep.cmax = prep.cmax + b;
         return t;
     }
 };
 
 // Takes the tensor-core scratch for B batches of K centroids from `s`, with
-// room for list_rows listed points (fp32), and zeroes the norm bound.
-km_status alloc_tc(Scratch& s, int dtype, int64_t B, int64_t K, int64_t d, int64_t list_rows, cudaStream_t st,
-                   TcScratch* out) {
+// `lists` re-scan lists of `cap` rows, and zeroes the norm bound and the list
+// counters.
+km_status alloc_tc(Scratch& s, int dtype, int64_t B, int64_t K, int64_t d, int64_t lists, int64_t cap,
+                   cudaStream_t st, TcScratch* out) {
     const int64_t Kp = padded_k(K);
     if (dtype == KM_F16) {
         __half *chat = nullptr, *cext = nullptr;
         KM_TRY(s.get(&chat, (size_t)(B * K * d), "rounded centroids"));
-        KM_TRY(s.get(&cext, (size_t)(B * Kp * 16), "centroid norm slices"));
+        KM_TRY(s.get(&cext, (size_t)(B * Kp * kNormPieces), "centroid norm slices"));
         out->prep.chat = chat;
         out->prep.cext = cext;
-        return KM_OK;
+    } else {
+        float *chat = nullptr, *cext = nullptr;
+        KM_TRY(s.get(&chat, (size_t)(B * K * 2 * d), "centroid heads and tails"));
+        KM_TRY(s.get(&cext, (size_t)(B * Kp * 8), "centroid norm pieces"));
+        out->prep.chat = chat;
+        out->prep.cext = cext;
     }
-    float *chat = nullptr, *cext = nullptr;
-    KM_TRY(s.get(&chat, (size_t)(B * K * 2 * d), "centroid heads and tails"));
-    KM_TRY(s.get(&cext, (size_t)(B * Kp * 8), "centroid norm pieces"));
     KM_TRY(s.get(&out->prep.cmax, (size_t)B, "centroid norm bound"));
-    KM_TRY(s.get(&out->flag_count, (size_t)B, "re-scan counters"));
-    KM_TRY(s.get(&out->flag_rows, (size_t)list_rows, "re-scan lists"));
-    out->prep.chat = chat;
-    out->prep.cext = cext;
-    return launched(cudaMemsetAsync(out->prep.cmax, 0, sizeof(float) * (size_t)B, st), "zero norm bound");
+    KM_TRY(s.get(&out->flag_count, (size_t)(2 * lists), "re-scan counters"));
+    KM_TRY(s.get(&out->flag_rows, (size_t)(lists * cap), "re-scan lists"));
+    out->lists = lists;
+    out->cap = cap;
+    out->parity = 0;
+    KM_TRY(launched(cudaMemsetAsync(out->prep.cmax, 0, sizeof(float) * (size_t)B, st), "zero norm bound"));
+    return launched(cudaMemsetAsync(out->flag_count, 0, sizeof(int32_t) * (size_t)(2 * lists), st),
+                    "zero re-scan counters");
+}
+
+// The re-scan list of the next assignment with `tc` (counter set tc->parity).
+RescanList rescan_list(const TcScratch& tc, int dtype, int64_t d) {
+    RescanList L;
+    L.cmax = tc.prep.cmax;
+    L.count = tc.flag_count + tc.parity * tc.lists;
+    L.rows = tc.flag_rows;
+    L.cap = tc.cap;
+    L.total = rescan_word();
+    if (dtype == KM_F16) L.set_fp16(d);
+    return L;
 }
 
 // The assignment for one iteration, given prepared centroids (tc == nullptr:
-// the CUDA-core kernel).  fp32 on tensor cores is two launches: the tf32
-// kernel, then the exact re-scan of the points it listed.
-km_status run_assign(const void* X, int dtype, const float* C, const TcScratch* tc, int64_t B, int64_t N, int64_t K,
+// the CUDA-core kernel).  On tensor cores it is two launches: the tensor-core
+// kernel, which certifies each point's label from its best two scores and
+// lists the rest, then the exact re-scan of the listed points (which also
+// zeroes the other counter set; tc->parity flips).
+km_status run_assign(const void* X, int dtype, const float* C, TcScratch* tc, int64_t B, int64_t N, int64_t K,
                      int64_t d, int32_t* labels, float* mindist, double* obj_acc, const DeviceInfo& dev,
                      cudaStream_t st, const int32_t* stop = nullptr) {
-    if (tc && dtype == KM_F16 && assign_split_supported(d, dtype)) {
+    if (!tc) {
         PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
-        return launched(launch_assign_split((const __half*)X, static_cast<const __half*>(tc->prep.chat),
-                                            static_cast<const __half*>(tc->prep.cext), B, N, K, d, labels, mindist,
-                                            obj_acc, dev.sms, st, stop),
-                        "assign (tensor cores, points and centroids streamed along d)");
+        return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st, stop),
+                        "assign (CUDA cores)");
     }
-    if (tc && dtype == KM_F16 && assign_wide_supported(d, dtype)) {
-        PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
-        return launched(launch_assign_wide((const __half*)X, static_cast<const __half*>(tc->prep.chat),
-                                           static_cast<const __half*>(tc->prep.cext), B, N, K, d, labels, mindist,
-                                           obj_acc, dev.sms, st, stop),
-                        "assign (tensor cores, d split in chunks)");
+    if (tc->cap < N && obj_acc) {
+        set_error("internal: a re-scan list shorter than a batch cannot carry the objective");
+        return KM_E_INVALID;
     }
-    if (tc && dtype == KM_F16) {
-        PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
-        return launched(launch_assign_tc((const __half*)X, static_cast<const __half*>(tc->prep.chat),
-                                         static_cast<const __half*>(tc->prep.cext), B, N, K, d, labels, mindist,
-                                         obj_acc, dev.sms, st, stop),
-                        "assign (tensor cores)");
+    PhaseScope ph(st, KM_PHASE_ASSIGN, 2);
+    const RescanList L = rescan_list(*tc, dtype, d);
+    int32_t* next = tc->flag_count + (1 - tc->parity) * tc->lists;
+    tc->parity ^= 1;
+    cudaError_t e;
+    const char* what;
+    if (dtype == KM_F16) {
+        const __half* Xh = static_cast<const __half*>(X);
+        const __half* chat = static_cast<const __half*>(tc->prep.chat);
+        const __half* cext = static_cast<const __half*>(tc->prep.cext);
+        if (assign_split_supported(d, dtype)) {
+            e = launch_assign_split(Xh, chat, cext, B, N, K, d, labels, mindist, obj_acc, L, dev.sms, st, stop);
+            what = "assign (tensor cores, points and centroids streamed along d)";
+        } else if (assign_wide_supported(d, dtype)) {
+            e = launch_assign_wide(Xh, chat, cext, B, N, K, d, labels, mindist, obj_acc, L, dev.sms, st, stop);
+            what = "assign (tensor cores, d split in chunks)";
+        } else {
+            e = launch_assign_tc(Xh, chat, cext, B, N, K, d, labels, mindist, obj_acc, L, dev.sms, st, stop);
+            what = "assign (tensor cores)";
+        }
+    } else {
+        e = launch_assign_tf32(static_cast<const float*>(X), static_cast<const float*>(tc->prep.chat),
+                               static_cast<const float*>(tc->prep.cext), B, N, K, d, labels, mindist, obj_acc, L,
+                               dev.sms, st, stop);
+        what = "assign (tf32 tensor cores)";
     }
-    if (tc) {
-        PhaseScope ph(st, KM_PHASE_ASSIGN, 2);
-        KM_TRY(launched(cudaMemsetAsync(tc->flag_count, 0, sizeof(int32_t) * (size_t)B, st), "zero re-scan counters"));
-        KM_TRY(launched(launch_assign_tf32((const float*)X, static_cast<const float*>(tc->prep.chat),
-                                           static_cast<const float*>(tc->prep.cext), tc->prep.cmax, B, N, K, d,
-                                           labels, mindist, obj_acc, tc->flag_count, tc->flag_rows, dev.sms, st,
-                                           stop),
-                        "assign (tf32 tensor cores)"));
-        const int blocks = (int)std::max<int64_t>(1, 4 * (int64_t)dev.sms / B);
-        return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st, tc->flag_rows,
-                                           tc->flag_count, blocks, stop),
-                        "assign (exact re-scan of listed points)");
-    }
-    PhaseScope ph(st, KM_PHASE_ASSIGN, 1);
-    return launched(launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, st, nullptr, nullptr, 0,
-                                       stop),
-                    "assign (CUDA cores)");
+    KM_TRY(launched(e, what));
+    return launched(launch_rescan(X, dtype, C, B, N, K, d, labels, mindist, obj_acc, L, dev.sms, st, stop, next),
+                    "assign (exact re-scan of listed points)");
 }
 
 std::atomic<int64_t> g_chunk_rows{0};
@@ -376,7 +401,7 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
         int32_t *lab = nullptr, *a_sorted = nullptr, *sidx = nullptr, *offs = nullptr, *counts = nullptr;
         unsigned char* work = nullptr;
         for (int i = 0; i < kSlots && status == KM_OK; ++i) status = scratch.get(&slot[i], (size_t)(R * d * s), "X slot");
-        if (status == KM_OK && tc) status = alloc_tc(scratch, dtype, B, K, d, R, st, &tcs);
+        if (status == KM_OK && tc) status = alloc_tc(scratch, dtype, B, K, d, 1, R, st, &tcs);
         if (status == KM_OK) status = scratch.get(&sums, (size_t)(B * K * d), "cluster sums");
         if (status == KM_OK) status = scratch.get(&counts, (size_t)(B * K), "cluster counts");
         if (status == KM_OK && objective) status = scratch.get(&obj_acc, (size_t)B, "objective accumulator");
@@ -412,9 +437,10 @@ km_status lloyd_host(const void* X, int64_t B, int64_t N, int64_t K, int64_t d, 
                     KM_TRY(launched(cudaEventRecord(res.ready[si], res.copy), "record chunk ready"));
                     // compute stream
                     KM_TRY(launched(cudaStreamWaitEvent(st, res.ready[si], 0), "wait chunk"));
-                    const TcScratch tcb = tc ? tcs.batch(b, K, d, dtype) : TcScratch();
+                    TcScratch tcb = tc ? tcs.batch(b, K, d, dtype) : TcScratch();
                     KM_TRY(run_assign(slot[si], dtype, C_out + b * K * d, tc ? &tcb : nullptr, 1, rows, K, d, lab,
                                       nullptr, obj_acc ? obj_acc + b : nullptr, dev, st));
+                    tcs.parity = tcb.parity;
                     {
                         PhaseScope ph(st, KM_PHASE_SORT, sort_launches);
                         KM_TRY(launched(launch_sort(lab, 1, rows, K, a_sorted, sidx, nullptr, nullptr, work, st, false),
@@ -474,7 +500,7 @@ km_status lloyd_device(const void* X, int64_t B, int64_t N, int64_t K, int64_t d
     unsigned char* work = nullptr;
     int32_t* stop = nullptr;
     double* shift = nullptr;
-    if (tc) KM_TRY(alloc_tc(scratch, dtype, B, K, d, B * N, st, &tcs));
+    if (tc) KM_TRY(alloc_tc(scratch, dtype, B, K, d, B, N, st, &tcs));
     if (cv) {
         KM_TRY(scratch.get(&stop, 1, "stop flag"));
         KM_TRY(scratch.get(&shift, (size_t)B, "centroid shifts"));
@@ -619,11 +645,43 @@ km_status km_assign(const void* X, const float* C, int64_t B, int64_t N, int64_t
     const bool tc = uses_tc(dtype, d);
     TcScratch tcs;
     if (tc) {
-        KM_TRY(alloc_tc(scratch, dtype, B, K, d, B * N, st, &tcs));
+        KM_TRY(alloc_tc(scratch, dtype, B, K, d, B, N, st, &tcs));
         PhaseScope ph(st, KM_PHASE_PREP, 1);
         KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
     }
     return run_assign(X, dtype, C, tc ? &tcs : nullptr, B, N, K, d, labels, mindist, nullptr, dev, st);
+}
+
+km_status km_assign_objective(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
+                              int32_t* labels, float* mindist, double* objective, void* stream) {
+    g_err[0] = 0;
+    if (!X || !C || !labels || !objective) {
+        set_error("km_assign_objective: X, C, labels and objective must be non-null");
+        return KM_E_INVALID;
+    }
+    KM_TRY(check_shape(B, N, K, d, dtype));
+    if (!aligned(X, 16) || !aligned(C, 16) || !aligned(labels, 4) || (mindist && !aligned(mindist, 4)) ||
+        !aligned(objective, 8)) {
+        set_error("km_assign_objective: X and C must be 16-byte aligned, labels and mindist 4-byte aligned, "
+                  "objective 8-byte aligned");
+        return KM_E_UNSUPPORTED;
+    }
+    DeviceInfo dev;
+    KM_TRY(check_device(&dev));
+    cudaStream_t st = (cudaStream_t)stream;
+    Scratch scratch(st);
+    const bool tc = uses_tc(dtype, d);
+    TcScratch tcs;
+    {
+        PhaseScope ph(st, KM_PHASE_OTHER, 0);
+        KM_TRY(launched(cudaMemsetAsync(objective, 0, sizeof(double) * (size_t)B, st), "zero objective"));
+    }
+    if (tc) {
+        KM_TRY(alloc_tc(scratch, dtype, B, K, d, B, N, st, &tcs));
+        PhaseScope ph(st, KM_PHASE_PREP, 1);
+        KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
+    }
+    return run_assign(X, dtype, C, tc ? &tcs : nullptr, B, N, K, d, labels, mindist, objective, dev, st);
 }
 
 km_status km_sort_labels(const int32_t* labels, int64_t B, int64_t N, int64_t K, int32_t* sorted_idx,
@@ -772,19 +830,23 @@ km_status km_assign_dense(const void* X, const float* C, int64_t B, int64_t N, i
     Scratch scratch(st);
     TcScratch tcs;
     float *dense = nullptr, *xnorm = nullptr;
-    KM_TRY(alloc_tc(scratch, dtype, B, K, d, 0, st, &tcs));
+    KM_TRY(alloc_tc(scratch, dtype, B, K, d, B, N, st, &tcs));
     KM_TRY(scratch.get(&dense, (size_t)(B * N * padded_k(K)), "dense score matrix"));
     KM_TRY(scratch.get(&xnorm, (size_t)(B * N), "point norms"));
     {
         PhaseScope ph(st, KM_PHASE_PREP, 1);
         KM_TRY(launched(launch_prep_centroids(C, B, K, d, dtype, tcs.prep, st), "centroid preparation"));
     }
-    PhaseScope ph(st, KM_PHASE_ASSIGN, 2);
+    PhaseScope ph(st, KM_PHASE_ASSIGN, 3);
     KM_TRY(launched(launch_assign_tc_dense((const __half*)X, static_cast<const __half*>(tcs.prep.chat),
                                            static_cast<const __half*>(tcs.prep.cext), B, N, K, d, dense, xnorm,
                                            dev.sms, st),
                     "dense scores (tensor cores)"));
-    return launched(launch_dense_argmin(dense, xnorm, B, N, K, labels, mindist, st), "argmin over the dense scores");
+    const RescanList L = rescan_list(tcs, dtype, d);
+    KM_TRY(launched(launch_dense_argmin(dense, xnorm, B, N, K, labels, mindist, L, st),
+                    "argmin over the dense scores"));
+    return launched(launch_rescan(X, dtype, C, B, N, K, d, labels, mindist, nullptr, L, dev.sms, st),
+                    "assign (exact re-scan of listed points)");
 }
 
 km_status km_update_scatter(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d,

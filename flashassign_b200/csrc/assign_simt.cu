@@ -4,10 +4,9 @@
 // distances never leaving registers -- computed with direct differences
 // sum_j (x_j - c_j)^2 in fp32.
 //
-// It serves the shapes the tensor-core kernels do not take (fp16 with
-// d < 64 or d > 128, fp32 with d not a multiple of 32 or d > 128), and, in
-// list mode, re-scans exactly the fp32 points that the tf32 tensor-core
-// kernel could not resolve (listed per batch).  Each thread owns one point;
+// It serves the shapes the tensor-core kernels do not take (fp16 with d < 64
+// or d not a multiple of 64 above 128, fp32 with d not a multiple of 32 or
+// d > 128).  Each thread owns one point;
 // centroids and a 32-wide slice of the block's points are staged in shared
 // memory, so the loop is a register-blocked [128 points x 32 centroids] tile.
 #include "km_internal.cuh"
@@ -26,13 +25,10 @@ __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ float to_f<__half>(__half v) { return __half2float(v); }
 
-// Points of batch b: rows [0, N) (list == nullptr), or the list_count[b]
-// rows list[b * N + r] (list mode).  Blocks stride over the points.
+// Points of batch b: rows [0, N); blocks stride over them.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restrict__ X, const float* __restrict__ C,
                                                                int64_t N, int64_t K, int64_t d,
-                                                               const int32_t* __restrict__ list,
-                                                               const int32_t* __restrict__ list_count,
                                                                int32_t* __restrict__ labels,
                                                                float* __restrict__ mindist,
                                                                double* __restrict__ obj_acc,
@@ -46,12 +42,12 @@ __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restri
     const int64_t b = blockIdx.y;
     const T* Xb = X + b * N * d;
     const float* Cb = C + b * K * d;
-    const int64_t count = list ? (int64_t)list_count[b] : N;
+    const int64_t count = N;
 
     for (int64_t i0 = (int64_t)blockIdx.x * kThreads; i0 < count; i0 += (int64_t)gridDim.x * kThreads) {
         __syncthreads();  // the previous round's readers of rows[] are done
         const bool mine = i0 + threadIdx.x < count;
-        rows[threadIdx.x] = !mine ? -1 : list ? (int64_t)list[b * N + i0 + threadIdx.x] : i0 + threadIdx.x;
+        rows[threadIdx.x] = mine ? i0 + threadIdx.x : -1;
         float best = INFINITY;
         int32_t arg = -1;
         for (int64_t k0 = 0; k0 < K; k0 += kTileK) {
@@ -110,16 +106,13 @@ __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restri
 }  // namespace
 
 cudaError_t launch_assign_simt(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
-                               int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st, const int32_t* list,
-                               const int32_t* list_count, int max_blocks, const int32_t* stop) {
-    int64_t gx = ceil_div(N, kThreads);
-    if (list && max_blocks > 0 && gx > max_blocks) gx = max_blocks;
-    const dim3 grid((unsigned)gx, (unsigned)B);
+                               int32_t* labels, float* mindist, double* obj_acc, cudaStream_t st, const int32_t* stop) {
+    const dim3 grid((unsigned)ceil_div(N, kThreads), (unsigned)B);
     if (dtype == KM_F16)
         return launch_kernel(assign_simt_kernel<__half>, grid, dim3(kThreads), 0, st, (const __half*)X, C, N, K, d,
-                             list, list_count, labels, mindist, obj_acc, stop);
-    return launch_kernel(assign_simt_kernel<float>, grid, dim3(kThreads), 0, st, (const float*)X, C, N, K, d, list,
-                         list_count, labels, mindist, obj_acc, stop);
+                             labels, mindist, obj_acc, stop);
+    return launch_kernel(assign_simt_kernel<float>, grid, dim3(kThreads), 0, st, (const float*)X, C, N, K, d, labels,
+                         mindist, obj_acc, stop);
 }
 
 }  // namespace km

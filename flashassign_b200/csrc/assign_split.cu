@@ -21,7 +21,9 @@
 // Layout per CTA pair (cluster of 2, tcgen05.mma.cta_group::2, kind::f16,
 // M=256, N=256, K=16), the score arithmetic of the other fp16 kernels (the
 // -||c||^2/2 term folded in as one more K=16 step of fp16 pieces against a
-// ones slice, so s = x.c - ||c||^2/2 and the epilogue tracks maxima):
+// slice of power-of-two weights, so s = x.c - ||c||^2/2 and the epilogue
+// tracks the best two scores of each point, whose gap certifies its label,
+// certify.cuh):
 //   * stages: [128 points x 64 fp16] + 2 x [128 centroids x 64 fp16], all
 //     128-byte swizzled, 48 KB per CTA, 4 stages;
 //   * norm slices of both tiles ride with a pass's last chunk into one of two
@@ -33,6 +35,7 @@
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records a fault code in the device fault word, stops issuing work, frees
 // its TMEM and returns.
+#include "certify.cuh"
 #include "tc_ptx.cuh"
 
 namespace km {
@@ -60,8 +63,8 @@ constexpr int kStageBytes = 3 * kBoxBytes;                          // points, t
 constexpr int kStageOff = 0;
 constexpr int kExtOff = kStageOff + kStages * kStageBytes;          // 2 slots x 2 tiles of norm pieces
 constexpr int kOnesOff = kExtOff + 2 * kAccSets * kExtBytes;
-constexpr int kMergeOff = kOnesOff + kExtBytes;                     // 2 slots x 128 rows x (score, label)
-constexpr int kMergeBytes = 2 * kRows * 8;
+constexpr int kMergeOff = kOnesOff + kExtBytes;                     // 2 slots x 128 rows x (best, second, label)
+constexpr int kMergeBytes = 2 * kRows * 12;
 constexpr int kBarOff = kMergeOff + kMergeBytes;
 // c_full[4], c_empty[4], acc_full[2], acc_empty[2], m_full[2], m_empty[2]
 constexpr int kNumBars = 2 * kStages + 2 * kAccSets + 4;
@@ -93,6 +96,7 @@ struct Params {
     double* obj_acc;      // [B] running sum of minimum distances, nullable
     const int32_t* stop;  // nullable: when *stop, the launch does nothing
     int32_t* fault;
+    RescanList list;      // the points left to the exact re-scan
 };
 
 // Sum of squares of rows n0 + 0..31 of batch b (rows past N give 0): the warp
@@ -139,8 +143,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t bar_m_full = bar_acc_empty + 8 * kAccSets, bar_m_empty = bar_m_full + 16;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + kNumBars * 8 + 4);
-    float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                 // [2][128]
-    int* merge_label = reinterpret_cast<int*>(smem + kMergeOff + kMergeBytes / 2);  // [2][128]
+    float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                // [2][128]
+    float* merge_second = reinterpret_cast<float*>(smem + kMergeOff + 8 * kRows);  // [2][128]
+    int* merge_label = reinterpret_cast<int*>(smem + kMergeOff + 16 * kRows);      // [2][128]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cta_rank();  // 0: leader CTA of the pair (issues the MMAs)
@@ -161,11 +166,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // the points' extra K slice: all ones (any layout of it reads as ones)
-    for (int i = threadIdx.x; i < kExtBytes / 16; i += kThreads) {
-        const uint32_t one2 = 0x3C003C00u;  // two fp16 1.0
-        reinterpret_cast<uint4*>(smem + kOnesOff)[i] = make_uint4(one2, one2, one2, one2);
-    }
+    // the points' extra K slice: the norm pieces' weights, the same in both
+    // 16-byte halves of every row (so the 32-byte swizzle leaves it as it is)
+    for (int i = threadIdx.x; i < kExtBytes / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem + kOnesOff)[i] =
+            make_uint4(kNormWeightW01, kNormWeightW23, kNormWeightW45, kNormWeightW67);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes visible to the MMA
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -289,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int nq = (u - b * upb) * kUnitRows + (int)rank * kRows + q * 32;  // this warp's first row
             // ||x||^2 of the warp's 32 rows (half 0), while the first pass is in the tensor pipe
             const float xnorm = h == 0 ? row_norms(P.X, b, P.N, P.d, nq, lane) : 0.f;
-            float best = -INFINITY;
+            float best = -INFINITY, second = -INFINITY;
             int label = -1;  // column of the running best
             for (int p = 0; p < P.passes && ok; ++p) {
                 const int tiles = 2 * p + 1 < P.ktiles ? 2 : 1;
@@ -306,58 +311,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
                     const int kt = 2 * p + s;
 #pragma unroll
-                    for (int g = 0; g < kPartCols / 32; ++g) {
-                        const float* w = v + 32 * g;
-                        float ga = max3(w[0], w[1], w[2]), gb = max3(w[3], w[4], w[5]);
-#pragma unroll
-                        for (int t = 6; t < 30; t += 4) {
-                            ga = max3(ga, w[t], w[t + 1]);
-                            gb = max3(gb, w[t + 2], w[t + 3]);
-                        }
-                        const float gmax = max3(max3(ga, w[30], w[31]), gb, gb);
-                        const bool better = gmax > best;  // strict: an earlier group keeps ties
-                        if (__any_sync(0xffffffffu, better)) {
-                            // the first column of the group holding its maximum
-                            int j0 = 31;
-#pragma unroll
-                            for (int j = 31; j >= 0; --j) j0 = (w[j] == gmax) ? j : j0;
-                            if (better) {
-                                best = gmax;
-                                label = kt * kTileK + h * kPartCols + g * 32 + j0;
-                            }
-                        }
-                    }
+                    for (int g = 0; g < kPartCols / 32; ++g)
+                        top2_group(v + 32 * g, kt * kTileK + h * kPartCols + g * 32, best, second, label);
                 }
             }
             if (!ok) break;
-            // join the column halves of each row (larger score, then lower
-            // index) through a double-buffered shared slot with bounded handoffs
+            // join the column halves of each row (the best two scores, the lower
+            // index on equal ones) through a double-buffered shared slot with
+            // bounded handoffs, then certify and write
             const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
             if (h == 1) {
                 if (!(ok = mbar_wait(bar_m_empty + 8 * ms, mph ^ 1, abort_flag, P.fault))) break;
                 merge_score[ms * kRows + row] = best;
+                merge_second[ms * kRows + row] = second;
                 merge_label[ms * kRows + row] = label;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_m_full + 8 * ms);
             } else {
                 if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
                 const float ob = merge_score[ms * kRows + row];
+                const float os = merge_second[ms * kRows + row];
                 const int ol = merge_label[ms * kRows + row];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
-                if (ob > best || (ob == best && ol >= 0 && (label < 0 || ol < label))) {
-                    best = ob;
-                    label = ol;
-                }
+                top2_join(best, second, label, ob, os, ol);  // this half holds the lower columns
                 const int n = nq + lane;
-                const float md = fmaxf(fmaf(-2.f, best, xnorm), 0.f);
-                if (n < P.N) {
-                    const int64_t o = (int64_t)b * P.N + n;
-                    P.labels[o] = label;
-                    if (P.mindist) P.mindist[o] = md;
-                }
-                if (P.obj_acc) {  // the objective: this warp's 32 rows, one atomic per warp
-                    double part = n < P.N ? (double)md : 0.0;
+                double part = certify_top2(P.list, P.list.cmax[b], b, P.N, n, n < P.N, best, second, label, xnorm,
+                                                P.labels, P.mindist, lane);
+                if (P.obj_acc) {  // the objective: this warp's certified rows, one atomic per warp
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
                     if (lane == 0) atomicAdd(P.obj_acc + b, part);
@@ -384,9 +365,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 bool assign_split_supported(int64_t d, int dtype) { return dtype == KM_F16 && d > 512 && d % 64 == 0; }
 
 cudaError_t launch_assign_split(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N,
-                                int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms,
-                                cudaStream_t st, const int32_t* stop) {
+                                int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
+                                const RescanList& list, int sms, cudaStream_t st, const int32_t* stop) {
     if (!assign_split_supported(d, KM_F16)) return cudaErrorNotSupported;
+    if (!list.cmax || !list.count || !list.rows) return cudaErrorInvalidValue;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, 2, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mc, chat, 2, B, K, d, kBoxK, kHalfTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -407,6 +389,7 @@ cudaError_t launch_assign_split(const __half* X, const __half* chat, const __hal
     P.obj_acc = obj_acc;
     P.stop = stop;
     P.fault = fault_word();
+    P.list = list;
     static std::atomic<int> pair_cache[kMaxDevices];
     const int max_pairs = co_resident_pairs((const void*)assign_split_kernel, kThreads, kSmemBytes, sms, pair_cache);
     P.pairs = P.units < max_pairs ? P.units : max_pairs;

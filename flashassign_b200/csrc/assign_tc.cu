@@ -13,8 +13,9 @@
 //     argmin_k ||x - c_k||^2 = argmax_k s.  The whole score comes out of the
 //     tensor cores: each point row gets one extra 16-wide K slice of ones and
 //     each centroid row the matching slice holding -||c||^2/2 split into fp16
-//     pieces (exact to ~2^-33 relative), so one more K=16 MMA step adds the
-//     norm term in fp32 and the epilogue only tracks maxima.
+//     pieces against power-of-two weights on the points' side
+//     (norm_piece_weight), so one more K=16 MMA step adds the norm term in
+//     fp32 and the epilogue only tracks maxima.
 //   * CTA pairs (a cluster of 2) run tcgen05.mma.cta_group::2 with M=256,
 //     N=256, K=16: each CTA stages its own 128 point rows and its own half
 //     (128) of each 256-centroid tile, so every instruction runs at the full
@@ -49,9 +50,11 @@
 //     summed from the staged X tile and the X buffer is released while the
 //     unit's other tiles run (two X buffers then suffice); at the unit's end
 //     the two column slices are joined (larger score, then lower index), and
-//     labels, mindist = ||x||^2 - 2 * best and the objective (one atomic per
-//     unit) are written.  Three X buffers with the release at the unit's end
-//     left room for only three centroid stages: 5% slower at K = 1024.
+//     each point whose label the scores' error bound certifies (certify.cuh)
+//     gets its label and mindist = ||x||^2 - 2 * best, and adds to the
+//     objective (one atomic per unit); the others are listed for the exact
+//     re-scan.  Three X buffers with the release at the unit's end left room
+//     for only three centroid stages: 5% slower at K = 1024.
 //   * Measured on B200: at the 1 kW power cap the SM clock settles near
 //     1.4 GHz (K = 4096) to 1.7 GHz (K = 1024) and a tile costs ~1.1 us of
 //     wall time either way: the kernel runs at the power limit, so fewer
@@ -59,6 +62,7 @@
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records a fault code in the device fault word, stops issuing work, frees
 // its TMEM and returns.
+#include "certify.cuh"
 #include "tc_ptx.cuh"
 
 namespace km {
@@ -128,6 +132,7 @@ struct Params {
     float* xnorm;     // dense mode: [B, N] ||x||^2
     const int32_t* stop;  // nullable: when *stop, the launch does nothing
     int32_t* fault;
+    RescanList list;      // the points left to the exact re-scan
 };
 
 // kDense (the dense-distance ablation): the same MMA pipeline, but every
@@ -180,11 +185,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // the points' extra K slice: all ones (any layout of it reads as ones)
-    for (int i = threadIdx.x; i < kExtBytes / 16; i += kThreads) {
-        const uint32_t one2 = 0x3C003C00u;  // two fp16 1.0
-        reinterpret_cast<uint4*>(smem + kAOnesOff)[i] = make_uint4(one2, one2, one2, one2);
-    }
+    // the points' extra K slice: the norm pieces' weights, the same in both
+    // 16-byte halves of every row (so the 32-byte swizzle leaves it as it is)
+    for (int i = threadIdx.x; i < kExtBytes / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem + kAOnesOff)[i] =
+            make_uint4(kNormWeightW01, kNormWeightW23, kNormWeightW45, kNormWeightW67);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes visible to the MMA
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -401,6 +406,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t ms = it_x & 1, mph = (it_x >> 1) & 1;
             const int b = u / upb;
             const int n0 = (u - b * upb) * kUnitRows + (int)rank * kRows;
+            float cmax2 = 0.f;  // the batch's norm bound, loaded while the unit runs
+            if constexpr (!kDense) cmax2 = P.list.cmax[b];
             // ||x||^2 as soon as the unit's first tile of MMAs has completed
             // (its X tile is then in place in both CTAs); the X buffer is
             // released right after, while the unit's other tiles run
@@ -436,34 +443,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
             double obj = 0.0;
             if constexpr (!kDense) {
+                float fb[kRows / 32];
+                int fl[kRows / 32];
 #pragma unroll
                 for (int rq = 0; rq < kRows / 32; ++rq) {
                     const int r = rq * 32 + lane;
-                    float fb = merge_score[((int)ms * kColParts) * kRows + r];
-                    int fl = merge_label[((int)ms * kColParts) * kRows + r];
+                    fb[rq] = merge_score[((int)ms * kColParts) * kRows + r];
+                    fl[rq] = merge_label[((int)ms * kColParts) * kRows + r];
 #pragma unroll
                     for (int part = 1; part < kColParts; ++part) {
                         const int slot = ((int)ms * kColParts + part) * kRows + r;
                         const float ob = merge_score[slot];
                         const int ol = merge_label[slot];
-                        if (ob > fb || (ob == fb && ol >= 0 && (fl < 0 || ol < fl))) {
-                            fb = ob;
-                            fl = ol;
+                        if (ob > fb[rq] || (ob == fb[rq] && ol >= 0 && (fl[rq] < 0 || ol < fl[rq]))) {
+                            fb[rq] = ob;
+                            fl[rq] = ol;
                         }
                     }
-                    const float md = fmaxf(fmaf(-2.f, fb, xn[rq]), 0.f);
-                    const int n = n0 + r;
-                    if (n < P.N) {
-                        const int64_t o = (int64_t)b * P.N + n;
-                        P.labels[o] = fl;
-                        if (P.mindist) P.mindist[o] = md;
-                        obj += (double)md;
-                    }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);  // the slot is read: the epilogue may refill it
+#pragma unroll
+                for (int rq = 0; rq < kRows / 32; ++rq) {
+                    const int n = n0 + rq * 32 + lane;
+                    obj += certify_best(P.list, cmax2, b, P.N, n, n < P.N, fb[rq], fl[rq], xn[rq], P.labels,
+                                             P.mindist, lane);
+                }
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
-            if (!kDense && P.obj_acc) {  // the objective of the unit's 128 rows, one atomic
+            if (!kDense && P.obj_acc) {  // the objective of the unit's certified rows, one atomic
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) obj += __shfl_xor_sync(0xffffffffu, obj, o);
                 if (lane == 0) atomicAdd(P.obj_acc + b, obj);
@@ -491,8 +501,8 @@ bool assign_tc_supported(int64_t d, int dtype) { return dtype == KM_F16 && d >= 
 
 template <bool kDense>
 cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
-                      int64_t d, int32_t* labels, float* mindist, double* obj_acc, float* dense, float* xnorm, int sms,
-                      cudaStream_t st, const int32_t* stop) {
+                      int64_t d, int32_t* labels, float* mindist, double* obj_acc, const RescanList& list, float* dense,
+                      float* xnorm, int sms, cudaStream_t st, const int32_t* stop) {
     if (!assign_tc_supported(d, KM_F16)) return cudaErrorNotSupported;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, 2, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -517,6 +527,7 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
     P.xnorm = xnorm;
     P.stop = stop;
     P.fault = fault_word();
+    P.list = list;
     static std::atomic<int> pair_cache[kMaxDevices];  // per instantiation
     const int max_pairs = co_resident_pairs((const void*)assign_tc_kernel<kDense>, kThreads, kSmemBytes, sms, pair_cache);
     P.pairs = P.units < max_pairs ? P.units : max_pairs;
@@ -525,14 +536,17 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
 }
 
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
-                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, int sms, cudaStream_t st,
-                             const int32_t* stop) {
-    return launch_tc<false>(X, chat, cext, B, N, K, d, labels, mindist, obj_acc, nullptr, nullptr, sms, st, stop);
+                             int64_t d, int32_t* labels, float* mindist, double* obj_acc, const RescanList& list,
+                             int sms, cudaStream_t st, const int32_t* stop) {
+    if (!list.cmax || !list.count || !list.rows) return cudaErrorInvalidValue;
+    return launch_tc<false>(X, chat, cext, B, N, K, d, labels, mindist, obj_acc, list, nullptr, nullptr, sms, st,
+                            stop);
 }
 
 cudaError_t launch_assign_tc_dense(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N,
                                    int64_t K, int64_t d, float* dense, float* xnorm, int sms, cudaStream_t st) {
-    return launch_tc<true>(X, chat, cext, B, N, K, d, nullptr, nullptr, nullptr, dense, xnorm, sms, st, nullptr);
+    return launch_tc<true>(X, chat, cext, B, N, K, d, nullptr, nullptr, nullptr, RescanList(), dense, xnorm, sms, st,
+                           nullptr);
 }
 
 }  // namespace km

@@ -143,8 +143,9 @@ struct Params {
     float* mindist;
     double* obj_acc;      // [B] running sum of minimum distances of the resolved points, nullable
     int32_t* flag_count;  // [B] points listed for the exact re-scan (zero on entry)
-    int32_t* flag_rows;   // [B, N] their indices within the batch
-    unsigned long long* rescans;  // running total of listed points (observability)
+    int32_t* flag_rows;   // [B, list_cap] their indices within the batch
+    int64_t list_cap;     // a count above it makes the re-scan take the whole batch
+    unsigned long long* rescans;  // running total of listed points (observability, nullable)
     const int32_t* stop;  // nullable: when *stop, the launch does nothing
     int32_t* fault;
 };
@@ -404,10 +405,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     int base = 0;
                     if (lane == 0) {
                         base = atomicAdd(P.flag_count + b, __popc(mask));
-                        atomicAdd(P.rescans, (unsigned long long)__popc(mask));
+                        if (P.rescans) atomicAdd(P.rescans, (unsigned long long)__popc(mask));
                     }
                     base = __shfl_sync(0xffffffffu, base, 0);
-                    if (listed) P.flag_rows[(int64_t)b * P.N + base + __popc(mask & ((1u << lane) - 1u))] = n;
+                    const int pos = base + __popc(mask & ((1u << lane) - 1u));
+                    if (listed && pos < P.list_cap) P.flag_rows[(int64_t)b * P.list_cap + pos] = n;
                 }
             }
         }
@@ -430,11 +432,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 bool assign_tf32_supported(int64_t d) { return d >= 32 && d <= 128 && d % 32 == 0; }
 
-cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float* cext, const float* cmax, int64_t B,
-                               int64_t N, int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
-                               int32_t* flag_count, int32_t* flag_rows, int sms, cudaStream_t st,
-                               const int32_t* stop) {
+cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float* cext, int64_t B, int64_t N,
+                               int64_t K, int64_t d, int32_t* labels, float* mindist, double* obj_acc,
+                               const RescanList& list, int sms, cudaStream_t st, const int32_t* stop) {
     if (!assign_tf32_supported(d)) return cudaErrorNotSupported;
+    if (!list.cmax || !list.count || !list.rows) return cudaErrorInvalidValue;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, 4, B, N, d, kBoxF, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mc, csplit, 4, B, K, 2 * d, kBoxF, kHalfTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -448,13 +450,14 @@ cudaError_t launch_assign_tf32(const float* X, const float* csplit, const float*
     P.units = B * P.units_per_batch;
     P.ktiles = (int)ceil_div(K, kTileK);
     P.boxes = (int)(d / kBoxF);
-    P.cmax = cmax;
+    P.cmax = list.cmax;
     P.labels = labels;
     P.mindist = mindist;
     P.obj_acc = obj_acc;
-    P.flag_count = flag_count;
-    P.flag_rows = flag_rows;
-    P.rescans = rescan_word();
+    P.flag_count = list.count;
+    P.flag_rows = list.rows;
+    P.list_cap = list.cap;
+    P.rescans = list.total;
     P.stop = stop;
     P.fault = fault_word();
     static std::atomic<int> pair_cache[kMaxDevices];

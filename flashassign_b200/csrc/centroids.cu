@@ -24,25 +24,33 @@ __device__ __forceinline__ double warp_sum(double v) {
 }
 
 // The centroid's norm slice for the fp16 tensor-core assignment: 16 fp16
-// values whose sum is -v to within ~2^-33 relative (greedy pieces, each the
-// nearest fp16 to what is left, clamped to the fp16 range), stored as two
-// 16-byte vectors.
-__device__ __forceinline__ void write_norm_slice(__half* out, double v) {
+// pieces p_j with sum_j w_j p_j = -v, w_j = norm_piece_weight(j), stored as
+// two 16-byte vectors.  Greedy from the largest weight down: each piece is the
+// fp16 nearest to what is left divided by its weight (clamped to the fp16
+// range; a piece that would be subnormal is left at 0, so nothing depends on
+// how the tensor cores treat subnormal inputs).  Returns false when the
+// remainder is not within 2^-30 of v (plus 2^-27): v beyond the pieces' range.
+__device__ __forceinline__ bool write_norm_slice(__half* out, double v) {
     double r = -v;
-    uint32_t w[8];
+    unsigned short bits[kNormPieces];
+    // positions in decreasing weight: 2^15 at 0-4 and 8-12, 1 at 5, 6, 13, 14, 2^-13 at 7 and 15
+    constexpr int kOrder[kNormPieces] = {0, 1, 2, 3, 4, 8, 9, 10, 11, 12, 5, 6, 13, 14, 7, 15};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        __half p[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // once r is 0 every further piece is 0
-            const double c = fmin(fmax(r, -65504.0), 65504.0);
-            p[h] = __float2half_rn((float)c);
-            r -= (double)__half2float(p[h]);
-        }
-        w[i] = (uint32_t)__half_as_ushort(p[0]) | ((uint32_t)__half_as_ushort(p[1]) << 16);
+    for (int i = 0; i < kNormPieces; ++i) {
+        const int j = kOrder[i];
+        const double w = (double)norm_piece_weight(j);
+        const double q = fmin(fmax(r / w, -65504.0), 65504.0);
+        __half p = __float2half_rn((float)q);
+        if (fabsf(__half2float(p)) < 0x1p-14f) p = __float2half(0.f);
+        bits[j] = __half_as_ushort(p);
+        r -= w * (double)__half2float(p);
     }
-    reinterpret_cast<uint4*>(out)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    reinterpret_cast<uint4*>(out)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    uint32_t wd[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wd[i] = (uint32_t)bits[2 * i] | ((uint32_t)bits[2 * i + 1] << 16);
+    reinterpret_cast<uint4*>(out)[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    reinterpret_cast<uint4*>(out)[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+    return fabs(r) <= 0x1p-30 * fabs(v) + 0x1p-27;
 }
 
 // tf32 head of an fp32 value: its low 13 mantissa bits cleared (exact in tf32).
@@ -63,16 +71,18 @@ __device__ __forceinline__ void write_norm_pieces_tf32(float* out, double v) {
 }
 
 // Everything the assignment needs of one centroid row, from the warp's sum of
-// squares `acc` (lane 0 writes): the norm slice, and for fp32 the running
-// bound of max_k ||c_k||^2 (non-negative floats order like their bit patterns).
+// squares `acc` (lane 0 writes): the norm slice, and the running bound of
+// max_k ||c_k||^2 (non-negative floats order like their bit patterns; +inf
+// when an fp16 norm slice cannot hold the norm).
 __device__ __forceinline__ void write_row_norm(const PreparedC& p, int dtype, int64_t b, int64_t slice_row,
                                                double acc) {
-    if (dtype == KM_F16) {
-        write_norm_slice(static_cast<__half*>(p.cext) + slice_row * 16, 0.5 * acc);
-    } else {
+    bool ok = true;
+    if (dtype == KM_F16)
+        ok = write_norm_slice(static_cast<__half*>(p.cext) + slice_row * kNormPieces, 0.5 * acc);
+    else
         write_norm_pieces_tf32(static_cast<float*>(p.cext) + slice_row * 8, 0.5 * acc);
-        atomicMax(reinterpret_cast<int*>(p.cmax + b), __float_as_int((float)(acc * (1.0 + 1e-6))));
-    }
+    if (p.cmax)
+        atomicMax(reinterpret_cast<int*>(p.cmax + b), ok ? __float_as_int((float)(acc * (1.0 + 1e-6))) : 0x7F800000);
 }
 
 // One warp per centroid row of [B, Kp]: fp16 rounds C (chat) and writes the

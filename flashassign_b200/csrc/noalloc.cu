@@ -5,7 +5,9 @@
 // allocate: a framework that reserved the whole device for its own pool, or
 // a latency-critical loop that must not enter the allocator (which can
 // synchronise and take locks).  This variant runs the same kernels with that
-// scratch in one fixed array compiled into the library instead.
+// scratch in one fixed array compiled into the library instead: the
+// centroid preparation, the tensor-core assignment (fp16, or fp32 on tf32)
+// and the exact re-scan of the points it could not certify.
 //
 // The array is a file-scope __device__ object, so every GPU that loads the
 // library holds kNoAllocScratchBytes of it until the process exits.  Host
@@ -15,6 +17,7 @@
 // entry point runs on it.
 #include "km_internal.cuh"
 
+#include <algorithm>
 #include <mutex>
 
 namespace km {
@@ -84,36 +87,69 @@ extern "C" km_status km_assign_noalloc(const void* X, const float* C, int64_t B,
         return KM_E_UNSUPPORTED;
     }
     cudaStream_t stm = (cudaStream_t)stream;
-    const bool tc = dtype == KM_F16 && (assign_tc_supported(d, dtype) || assign_wide_supported(d, dtype) ||
-                                        assign_split_supported(d, dtype));
+    const bool tc = dtype == KM_F16 ? (assign_tc_supported(d, dtype) || assign_wide_supported(d, dtype) ||
+                                       assign_split_supported(d, dtype))
+                                    : assign_tf32_supported(d);
     if (!tc) {  // the CUDA-core kernel reads C directly and needs no scratch
         cudaError_t e = launch_assign_simt(X, dtype, C, B, N, K, d, labels, mindist, nullptr, stm);
         return e == cudaSuccess ? KM_OK : cuda_error(e, "km_assign_noalloc: assign (CUDA cores)");
     }
-    const size_t chat_bytes = round_up(sizeof(__half) * (size_t)(B * K * d), 256);
-    const size_t cext_bytes = sizeof(__half) * (size_t)(B * padded_k(K) * 16);
-    if (chat_bytes + cext_bytes > kNoAllocScratchBytes) {
-        set_error("km_assign_noalloc: needs %zu bytes of scratch (2*B*K*d + 32*B*ceil(K/256)*256), above the "
-                  "fixed %zu-byte array; use km_assign",
-                  chat_bytes + cext_bytes, kNoAllocScratchBytes);
+    // the array holds, in order: the prepared centroids (fp16: rounded rows and
+    // norm slices; fp32: tf32 heads and tails and norm pieces), the per-batch
+    // norm bound, the re-scan counters, and as many re-scan rows per batch as
+    // fit (up to N; a batch whose list overflows is re-scanned whole)
+    const int64_t Kp = padded_k(K);
+    const size_t chat_bytes =
+        round_up((dtype == KM_F16 ? sizeof(__half) : 2 * sizeof(float)) * (size_t)(B * K * d), 256);
+    const size_t cext_bytes =
+        round_up(dtype == KM_F16 ? sizeof(__half) * (size_t)(B * Kp * kNormPieces) : sizeof(float) * (size_t)(B * Kp * 8),
+                 256);
+    const size_t fixed = chat_bytes + cext_bytes + round_up(sizeof(float) * (size_t)B, 256) +
+                         round_up(sizeof(int32_t) * (size_t)B, 256);
+    if (fixed > kNoAllocScratchBytes) {
+        set_error("km_assign_noalloc: needs %zu bytes of scratch for the prepared centroids (fp16: 2*B*K*d + "
+                  "32*B*ceil(K/256)*256; fp32: 8*B*K*d + 32*B*ceil(K/256)*256; plus 8*B), above the fixed %zu-byte "
+                  "array; use km_assign",
+                  fixed, kNoAllocScratchBytes);
         return KM_E_UNSUPPORTED;
     }
     void* base = nullptr;
     if ((st = scratch_address(dev.device, &base)) != KM_OK) return st;
-    __half* chat = static_cast<__half*>(base);
-    __half* cext = reinterpret_cast<__half*>(static_cast<unsigned char*>(base) + chat_bytes);
-    // every element of both scratch regions that the assignment reads is written here first
+    unsigned char* p = static_cast<unsigned char*>(base);
     PreparedC prep;
-    prep.chat = chat;
-    prep.cext = cext;
-    cudaError_t e = launch_prep_centroids(C, B, K, d, dtype, prep, stm);
+    prep.chat = p;
+    prep.cext = p + chat_bytes;
+    prep.cmax = reinterpret_cast<float*>(p + chat_bytes + cext_bytes);
+    RescanList L;
+    L.cmax = prep.cmax;
+    L.count = reinterpret_cast<int32_t*>(p + chat_bytes + cext_bytes + round_up(sizeof(float) * (size_t)B, 256));
+    L.rows = reinterpret_cast<int32_t*>(p + fixed);
+    L.cap = std::min<int64_t>(N, (int64_t)((kNoAllocScratchBytes - fixed) / (sizeof(int32_t) * (size_t)B)));
+    L.total = rescan_word();
+    if (dtype == KM_F16) L.set_fp16(d);
+    // the bound and the counters must start at zero; every other element that
+    // the kernels read is written first by the preparation or the assignment
+    cudaError_t e = cudaMemsetAsync(prep.cmax, 0, sizeof(float) * (size_t)B, stm);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L.count, 0, sizeof(int32_t) * (size_t)B, stm);
+    if (e != cudaSuccess) return cuda_error(e, "km_assign_noalloc: clear the scratch's counters");
+    e = launch_prep_centroids(C, B, K, d, dtype, prep, stm);
     if (e != cudaSuccess) return cuda_error(e, "km_assign_noalloc: centroid preparation");
-    const __half* Xh = static_cast<const __half*>(X);
-    if (assign_split_supported(d, dtype))
-        e = launch_assign_split(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms, stm);
-    else if (assign_wide_supported(d, dtype))
-        e = launch_assign_wide(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms, stm);
-    else
-        e = launch_assign_tc(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, dev.sms, stm);
-    return e == cudaSuccess ? KM_OK : cuda_error(e, "km_assign_noalloc: assign (tensor cores)");
+    if (dtype == KM_F16) {
+        const __half* Xh = static_cast<const __half*>(X);
+        const __half* chat = static_cast<const __half*>(prep.chat);
+        const __half* cext = static_cast<const __half*>(prep.cext);
+        if (assign_split_supported(d, dtype))
+            e = launch_assign_split(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, L, dev.sms, stm);
+        else if (assign_wide_supported(d, dtype))
+            e = launch_assign_wide(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, L, dev.sms, stm);
+        else
+            e = launch_assign_tc(Xh, chat, cext, B, N, K, d, labels, mindist, nullptr, L, dev.sms, stm);
+    } else {
+        e = launch_assign_tf32(static_cast<const float*>(X), static_cast<const float*>(prep.chat),
+                               static_cast<const float*>(prep.cext), B, N, K, d, labels, mindist, nullptr, L, dev.sms,
+                               stm);
+    }
+    if (e != cudaSuccess) return cuda_error(e, "km_assign_noalloc: assign (tensor cores)");
+    e = launch_rescan(X, dtype, C, B, N, K, d, labels, mindist, nullptr, L, dev.sms, stm);
+    return e == cudaSuccess ? KM_OK : cuda_error(e, "km_assign_noalloc: exact re-scan of listed points");
 }

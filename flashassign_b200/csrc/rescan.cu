@@ -1,0 +1,258 @@
+// The exact re-scan of the points that a tensor-core assignment could not
+// certify (near ties, duplicate centroids, data far from the origin, fp16
+// norms beyond the folded term's range): for each listed point the nearest
+// centroid under direct differences sum_j (x_j - c_j)^2 in fp32, lowest index
+// on ties -- the FlashAssign recurrence of the papernotes.org "Flash-KMeans"
+// page (关键设计 1) without the norm expansion, so no cancellation.
+//
+// The list is short (a few points per batch, often none), so the kernel is
+// built for latency: a thread-block cluster takes 32 listed points of one
+// batch at a time and splits the batch's centroids among its CTAs; in a CTA,
+// lane p of every warp holds point p and each warp a slice of the CTA's
+// centroids; the warps' results are joined in shared memory and the CTAs'
+// through distributed shared memory by CTA 0, which writes the label, mindist
+// and the objective share.  The distance of each (point, centroid) is summed
+// over ascending dimensions, as the CUDA-core assignment kernel sums it.
+#include "km_internal.cuh"
+
+#include <algorithm>
+#include <atomic>
+
+namespace km {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kPoints = 32;                 // points per chunk, one per lane
+constexpr int kPerWarp = 8;                 // centroids per warp per block
+constexpr int kBlockK = kWarps * kPerWarp;  // centroids per CTA per block (64)
+constexpr int kSlice = 32;                  // dimensions per staged slice
+constexpr int kClusterMax = 16;             // non-portable on sm_100, checked placeable
+
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__half>(__half v) { return __half2float(v); }
+
+__device__ __forceinline__ uint32_t cl_rank() {
+    uint32_t r;
+    asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cl_size() {
+    uint32_t r;
+    asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cl_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// (distance, index) of point `lane` in CTA `rank`'s result slots
+__device__ __forceinline__ void ld_peer(const float* d_local, const int* k_local, uint32_t rank, float& dv, int& kv) {
+    uint32_t da = (uint32_t)__cvta_generic_to_shared(d_local), ka = (uint32_t)__cvta_generic_to_shared(k_local);
+    asm volatile("mapa.shared::cluster.u32 %0, %0, %1;" : "+r"(da) : "r"(rank));
+    asm volatile("mapa.shared::cluster.u32 %0, %0, %1;" : "+r"(ka) : "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(dv) : "r"(da) : "memory");
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(kv) : "r"(ka) : "memory");
+}
+// Whether (d, k) is nearer than (bd, bk): a smaller distance, or an equal one at a lower index.
+__device__ __forceinline__ bool nearer(float d, int k, float bd, int bk) {
+    return k >= 0 && (bk < 0 || d < bd || (d == bd && k < bk));
+}
+
+// grid = (cluster size * clusters per batch, B); each cluster takes the
+// chunks c, c + clusters, ... of its batch's list (the whole batch when its
+// count exceeds the capacity: the list overflowed).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) rescan_kernel(const T* __restrict__ X, const float* __restrict__ C,
+                                                          int64_t N, int64_t K, int64_t d,
+                                                          const int32_t* __restrict__ list,
+                                                          const int32_t* __restrict__ list_count, int64_t cap,
+                                                          int32_t* __restrict__ reset, int32_t* __restrict__ labels,
+                                                          float* __restrict__ mindist, double* __restrict__ obj_acc,
+                                                          const int32_t* __restrict__ stop) {
+    pdl_trigger();
+    pdl_wait();
+    if (stop && *stop) return;  // read by every CTA of the cluster alike
+    __shared__ float xs[kPoints][kSlice + 1];
+    __shared__ float cs[kBlockK][kSlice + 1];
+    __shared__ float red_d[kWarps][kPoints];
+    __shared__ int red_k[kWarps][kPoints];
+    __shared__ float res_d[kPoints];
+    __shared__ int res_k[kPoints];
+    __shared__ int64_t rows[kPoints];
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t b = blockIdx.y;
+    const uint32_t rank = cl_rank(), csize = cl_size();
+    const int64_t cluster = blockIdx.x / csize, clusters = gridDim.x / csize;
+    if (reset && cluster == 0 && rank == 0 && threadIdx.x == 0) reset[b] = 0;
+    const int64_t listed = list_count[b];
+    const bool whole = listed > cap;
+    const int64_t npts = whole ? N : listed;
+    const int64_t chunks = (npts + kPoints - 1) / kPoints;
+    const int64_t per_cta = (K + csize - 1) / csize;
+    const int64_t k_lo = (int64_t)rank * per_cta, k_hi = k_lo + per_cta < K ? k_lo + per_cta : K;
+    const T* Xb = X + b * N * d;
+    const float* Cb = C + b * K * d;
+
+    for (int64_t ch = cluster; ch < chunks; ch += clusters) {
+        if (threadIdx.x < kPoints) {
+            const int64_t p = ch * kPoints + threadIdx.x;
+            rows[threadIdx.x] = p >= npts ? -1 : whole ? p : (int64_t)list[b * cap + p];
+        }
+        __syncthreads();
+        float best = INFINITY;
+        int bk = -1;
+        for (int64_t kb = k_lo; kb < k_hi; kb += kBlockK) {
+            float acc[kPerWarp];
+#pragma unroll
+            for (int c = 0; c < kPerWarp; ++c) acc[c] = 0.f;
+            for (int64_t j0 = 0; j0 < d; j0 += kSlice) {
+                for (int t = threadIdx.x; t < kPoints * kSlice; t += kThreads) {
+                    const int r = t / kSlice, j = t % kSlice;
+                    const int64_t gi = rows[r], gj = j0 + j;
+                    xs[r][j] = (gi >= 0 && gj < d) ? to_f<T>(Xb[gi * d + gj]) : 0.f;
+                }
+                for (int t = threadIdx.x; t < kBlockK * kSlice; t += kThreads) {
+                    const int r = t / kSlice, j = t % kSlice;
+                    const int64_t gk = kb + r, gj = j0 + j;
+                    float v = (gk < k_hi && gj < d) ? Cb[gk * d + gj] : 0.f;
+                    if (sizeof(T) == 2) v = __half2float(__float2half_rn(v));  // the centroids as the assignment sees them
+                    cs[r][j] = v;
+                }
+                __syncthreads();
+#pragma unroll 8
+                for (int j = 0; j < kSlice; ++j) {
+                    const float xv = xs[lane][j];
+#pragma unroll
+                    for (int c = 0; c < kPerWarp; ++c) {
+                        const float diff = xv - cs[warp * kPerWarp + c][j];
+                        acc[c] = fmaf(diff, diff, acc[c]);
+                    }
+                }
+                __syncthreads();
+            }
+#pragma unroll
+            for (int c = 0; c < kPerWarp; ++c) {
+                const int64_t k = kb + warp * kPerWarp + c;
+                if (k < k_hi && acc[c] < best) {  // ascending k within the warp: strict keeps the lowest
+                    best = acc[c];
+                    bk = (int)k;
+                }
+            }
+        }
+        // this CTA's nearest centroid of each point: join the warps
+        red_d[warp][lane] = best;
+        red_k[warp][lane] = bk;
+        __syncthreads();
+        if (warp == 0) {
+            float bd = red_d[0][lane];
+            int kk = red_k[0][lane];
+            for (int w = 1; w < kWarps; ++w)
+                if (nearer(red_d[w][lane], red_k[w][lane], bd, kk)) {
+                    bd = red_d[w][lane];
+                    kk = red_k[w][lane];
+                }
+            res_d[lane] = bd;
+            res_k[lane] = kk;
+        }
+        cl_sync();  // every CTA's result is visible to the cluster
+        if (rank == 0 && warp == 0) {
+            float bd = res_d[lane];
+            int kk = res_k[lane];
+            for (uint32_t q = 1; q < csize; ++q) {
+                float dv;
+                int kv;
+                ld_peer(&res_d[lane], &res_k[lane], q, dv, kv);
+                if (nearer(dv, kv, bd, kk)) {
+                    bd = dv;
+                    kk = kv;
+                }
+            }
+            const int64_t i = rows[lane];
+            if (i >= 0) {
+                labels[b * N + i] = kk;
+                if (mindist) mindist[b * N + i] = bd;
+            }
+            if (obj_acc) {  // the listed points' share of the objective: one atomic per chunk
+                double part = i >= 0 ? (double)bd : 0.0;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                if (lane == 0 && part != 0.0) atomicAdd(obj_acc + b, part);
+            }
+        }
+        cl_sync();  // no CTA refills its result slots while CTA 0 may still read them
+    }
+}
+
+// The cluster size: 16 CTAs when such clusters can be placed on this device
+// (checked once per device), else 8.
+int cluster_ctas() {
+    static std::atomic<int> state[64];  // per device: 0 unknown, else the size
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 8;
+    }
+    int s = state[dev].load(std::memory_order_acquire);
+    if (s == 0) {
+        bool ok = cudaFuncSetAttribute(rescan_kernel<__half>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                      cudaSuccess &&
+                  cudaFuncSetAttribute(rescan_kernel<float>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                      cudaSuccess;
+        for (int which = 0; ok && which < 2; ++which) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(kClusterMax, 1, 1);
+            cfg.blockDim = dim3(kThreads, 1, 1);
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = kClusterMax;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            ok = (which == 0 ? cudaOccupancyMaxActiveClusters(&n, rescan_kernel<__half>, &cfg)
+                             : cudaOccupancyMaxActiveClusters(&n, rescan_kernel<float>, &cfg)) == cudaSuccess &&
+                 n >= 1;
+        }
+        if (!ok) cudaGetLastError();
+        s = ok ? kClusterMax : 8;
+        state[dev].store(s, std::memory_order_release);
+    }
+    return s;
+}
+
+}  // namespace
+
+cudaError_t launch_rescan(const void* X, int dtype, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
+                          int32_t* labels, float* mindist, double* obj_acc, const RescanList& list, int sms,
+                          cudaStream_t st, const int32_t* stop, int32_t* reset) {
+    if (!list.count || !list.rows) return cudaErrorInvalidValue;
+    const int cs = cluster_ctas();
+    // enough clusters per batch to fill the GPU about twice when the lists are long
+    const int64_t per_batch = std::max<int64_t>(1, std::min<int64_t>(ceil_div(N, kPoints), 2 * sms / (cs * B)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(cs * per_batch), (unsigned)B, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    if (dtype == KM_F16)
+        return cudaLaunchKernelEx(&cfg, rescan_kernel<__half>, (const __half*)X, C, N, K, d, (const int32_t*)list.rows,
+                                  (const int32_t*)list.count, list.cap, reset, labels, mindist, obj_acc, stop);
+    return cudaLaunchKernelEx(&cfg, rescan_kernel<float>, (const float*)X, C, N, K, d, (const int32_t*)list.rows,
+                              (const int32_t*)list.count, list.cap, reset, labels, mindist, obj_acc, stop);
+}
+
+}  // namespace km

@@ -74,11 +74,17 @@ typedef enum {
  *     article, "Usándolo"): on the tensor cores, points and centroids both
  *     streamed in 64-dimension chunks, each point chunk meeting 512 centroids;
  *   - fp32, d in {32, 64, 96, 128}: on the tensor cores from tf32 head/tail
- *     splits of both operands (three products); a point whose best two scores
- *     lie within the split's error bound is re-scanned exactly on the CUDA
- *     cores, so every label is the exact argmin up to fp32 rounding (see
- *     km_assign_rescans);
+ *     splits of both operands (three products);
  *   - other shapes: direct differences sum_j (x_j - c_j)^2 on the CUDA cores.
+ * On the tensor-core paths each point's label is certified against the
+ * rounding-error bound of its scores, from its best score (fp16, d <= 128) or
+ * its best two scores (wider fp16, fp32); a point that is not certified (near
+ * ties, near-duplicate centroids, data far from the origin, fp16 centroid
+ * norms beyond the folded norm term's range of ~3.4e10) is re-scanned exactly
+ * on the CUDA cores (see km_assign_rescans).  So every fp32 label is the exact argmin up
+ * to fp32 rounding, and every fp16 label is the exact argmin unless the two
+ * smallest exact distances d1 <= d2 of the point satisfy d2 - d1 < 1e-3 d2,
+ * in which case its distance is within 1e-3 d2 of d1.
  *   X       [B, N, d] dtype, device.     C [B, K, d] fp32, device.
  *   labels  [B, N] int32, device, written.
  *   mindist [B, N] fp32, device, written; may be NULL.
@@ -172,13 +178,18 @@ KM_API km_status km_lloyd_tol(const void* X, const float* C_init, int64_t B, int
  * e.g. a framework that has reserved the device's memory for its own pool,
  * or a latency-critical loop that must not enter the allocator, which can
  * synchronise and take locks.  Same arguments, results and kernels as
- * km_assign; the scratch (fp16 centroids and their norm slices) lives in one
- * fixed array of km_assign_noalloc_limit() bytes (16 MiB) compiled into the
- * library, which every GPU that loads the library holds until exit.
- *   - Needs 2*B*K*d + 32*B*ceil(K/256)*256 bytes for fp16 inputs on the
- *     tensor-core paths (64 <= d <= 128, or d a multiple of 64 above 128;
- *     none otherwise); larger problems return
- *     KM_E_UNSUPPORTED with the sizes in km_last_error().
+ * km_assign; the scratch (the prepared centroids, their norm bound, and the
+ * list of points left to the exact re-scan) lives in one fixed array of
+ * km_assign_noalloc_limit() bytes (16 MiB) compiled into the library, which
+ * every GPU that loads the library holds until exit.
+ *   - The prepared centroids need 2*B*K*d (fp16) or 8*B*K*d (fp32) bytes plus
+ *     32*B*ceil(K/256)*256 and 8*B on the tensor-core paths (fp16 with
+ *     64 <= d <= 128 or d a multiple of 64 above 128; fp32 with d in
+ *     {32, 64, 96, 128}; nothing otherwise); larger problems return
+ *     KM_E_UNSUPPORTED with the sizes in km_last_error().  The rest of the
+ *     array holds the re-scan lists; a batch with more listed points than fit
+ *     is re-scanned whole (same labels; its mindist then all from the CUDA
+ *     cores).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -202,6 +213,15 @@ KM_API size_t km_assign_noalloc_limit(void);
  */
 KM_API km_status km_update_sums(const void* X, const int32_t* labels, int64_t B, int64_t N, int64_t K, int64_t d,
                                 int dtype, float* sums, int32_t* counts, void* stream);
+
+/*
+ * km_assign that also returns, per batch, the objective of the assignment it
+ * made: objective[b] = sum_i mindist[b][i] (fp64, device, [B], 8-byte
+ * aligned, written), accumulated by the assignment kernels themselves (the
+ * sharded loop adds it over the shards).  Other arguments as km_assign.
+ */
+KM_API km_status km_assign_objective(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d,
+                                     int dtype, int32_t* labels, float* mindist, double* objective, void* stream);
 KM_API km_status km_finalize(const float* sums, const int32_t* counts, int64_t B, int64_t K, int64_t d, float* C_out,
                              void* stream);
 
@@ -216,7 +236,8 @@ KM_API km_status km_finalize(const float* sums, const int32_t* counts, int64_t B
  * scratch matrix in HBM (K' = K rounded up to 256; 4*B*N*K' bytes, taken with
  * cudaMallocAsync: KM_E_NOMEM when it does not fit), then a second kernel
  * reads it back and takes each point's argmax (lowest index among equal
- * scores).  fp16 points with 64 <= d <= 128 only (else KM_E_UNSUPPORTED).
+ * scores), certified and re-scanned as in km_assign.  fp16 points with
+ * 64 <= d <= 128 only (else KM_E_UNSUPPORTED).
  * Arguments as km_assign.
  */
 KM_API km_status km_assign_dense(const void* X, const float* C, int64_t B, int64_t N, int64_t K, int64_t d, int dtype,
@@ -282,11 +303,11 @@ KM_API km_status km_device_fault(int32_t* code, void* stream);
 
 /*
  * Reads and clears the number of points, on the current device, that the
- * fp32 tensor-core assignment could not resolve within its error bound and
+ * tensor-core assignments could not certify within their error bound and
  * handed to the exact CUDA-core re-scan since the last call (near ties,
- * duplicate centroids, data far from the origin).  Not a result of the
- * method -- an observability counter for its numerics; 0 on fp16 and
- * CUDA-core paths.  Synchronises `stream`.
+ * duplicate centroids, data far from the origin, fp16 norms beyond the
+ * folded term's range).  Not a result of the method -- an observability
+ * counter for its numerics; 0 on the CUDA-core paths.  Synchronises `stream`.
  */
 KM_API km_status km_assign_rescans(int64_t* count, void* stream);
 

@@ -79,6 +79,7 @@ def test_update_and_sort_and_lloyd_reject_nulls():
     assert L.km_lloyd_tol(FAKE, FAKE, 1, 10, 2, 16, 0, 0, 0.0, FAKE, FAKE, None, FAKE, None) == 1
     assert L.km_assign_dense(None, FAKE, 1, 10, 2, 64, 1, FAKE, None, None) == 1
     assert L.km_update_scatter(FAKE, None, 1, 10, 2, 16, 0, FAKE, FAKE, FAKE, None) == 1
+    assert L.km_assign_objective(FAKE, FAKE, 1, 10, 2, 16, 0, FAKE, None, None, None) == 1
 
 
 def test_binding_raises_with_detail():

@@ -130,6 +130,86 @@ def test_fp32_tensor_cores_exact_where_the_gap_is_clear_far_from_the_origin():
     check_labels(X, C, lab, md)
 
 
+FP16_TC_WIDTHS = [64, 128, 256, 512, 1024, 4096]  # the d <= 128, wide and split-D tensor-core kernels
+
+
+def _far_mixture(rng, B, N, ncomp, d, offset, spread, sigma):
+    """Points of a Gaussian mixture whose centres sit at `offset` + spread * N(0,1) per coordinate."""
+    centres = offset + spread * rng.standard_normal((B, ncomp, d))
+    comp = rng.integers(0, ncomp, (B, N))
+    X = (np.take_along_axis(centres, comp[..., None], axis=1) + sigma * rng.standard_normal((B, N, d)))
+    return X.astype(np.float16), centres
+
+
+@pytest.mark.parametrize("d", FP16_TC_WIDTHS)
+def test_fp16_large_norms_fold_exactly(d):
+    # ||c||^2 of several million, far past what 16 unit-weight fp16 pieces of -||c||^2/2 can hold
+    # (~2.1e6), on data the tensor cores can certify: for d <= 128 (certified from the best score)
+    # points spread widely around their centres, for wider points (certified from the best two
+    # scores) tight clusters far apart; almost every label comes from the tensor cores
+    rng = np.random.default_rng(80 + d)
+    B, N, K = 2, (1000 if d <= 512 else 300), (300 if d <= 512 else 60)
+    offset = float(np.sqrt(6e6 / d))
+    spread, sigma = (offset / 2, offset / 4) if d <= 128 else (offset / 10, 1.0)
+    X, centres = _far_mixture(rng, B, N, K, d, offset, spread, sigma)
+    C = (centres + 0.5 * rng.standard_normal(centres.shape)).astype(np.float32)
+    assert (np.square(C.astype(np.float16).astype(np.float64)).sum(-1) > 4e6).all()
+    km.assign_rescans()
+    lab, md = run_assign(X, C)
+    listed = km.assign_rescans()
+    check_labels(X, C, lab, md)
+    assert listed < 0.05 * B * N, f"{listed} of {B * N} points went to the exact re-scan"
+
+
+@pytest.mark.parametrize("d", [128, 1024])
+def test_fp16_norms_beyond_the_folded_range_are_rescanned_exactly(d):
+    # ||c||^2 / 2 above the folded term's ~1.7e10: every point of the batch goes to the exact
+    # CUDA-core re-scan, none gets a truncated score
+    rng = np.random.default_rng(90 + d)
+    B, N, K = 2, 400, 50
+    offset = float(np.sqrt(6e10 / d))
+    X, centres = _far_mixture(rng, B, N, K, d, offset, offset / 10, offset / 100)
+    C = (centres + offset / 100 * rng.standard_normal(centres.shape)).astype(np.float32)
+    assert (np.square(C.astype(np.float16).astype(np.float64)).sum(-1) > 3.5e10).all()
+    km.assign_rescans()
+    lab, md = run_assign(X, C)
+    assert km.assign_rescans() == B * N
+    check_labels(X, C, lab, md)
+
+
+@pytest.mark.parametrize("d", FP16_TC_WIDTHS)
+def test_fp16_tensor_cores_exact_where_the_gap_is_clear_far_from_the_origin(d):
+    # the fp16 twin of the fp32 test above: ||x||^2 and ||c||^2 dwarf the distances, so the
+    # expansion cancels; labels must be exact wherever the relative top-2 gap is >= 1e-3
+    rng = np.random.default_rng(78 + d)
+    B, N, K = 2, (3000 if d <= 512 else 800), (200 if d <= 512 else 80)
+    centres = rng.standard_normal((B, 40, d)) + 4.0
+    X = (centres[:, rng.integers(0, 40, N)] + 0.05 * rng.standard_normal((B, N, d))).astype(np.float16)
+    C = X[:, rng.choice(N, K, replace=False)].astype(np.float32)
+    km.assign_rescans()
+    lab, md = run_assign(X, C)
+    listed = km.assign_rescans()
+    check_labels(X, C, lab, md)
+    print(f"d={d}: {listed} of {B * N} points re-scanned")
+
+
+@pytest.mark.parametrize("d", [128, 256, 1024])
+def test_fp16_duplicate_centroids_resolve_to_the_lowest_index(d):
+    # every centroid twice, 100 columns apart (some pairs in one 32-column group, most not): the
+    # duplicates' scores are equal bit for bit, and the label must be the lower index as in the
+    # oracle, whether the tensor cores certify the point or the exact re-scan takes it
+    rng = np.random.default_rng(31 + d)
+    B, N, K = 2, 2000, 200
+    X = rng.standard_normal((B, N, d)).astype(np.float16)
+    base = rng.standard_normal((B, K // 2, d)).astype(np.float32)
+    C = np.concatenate([base, base], axis=1)
+    C[:, 1::7] = C[:, 0::7][:, :C[:, 1::7].shape[1]]  # and some neighbours equal inside a group
+    lab, md = run_assign(X, C)
+    ref, d1, d2 = oracle.assign(X, C)
+    assert np.array_equal(lab, ref)
+    check_labels(X, C, lab, md)
+
+
 def test_assign_single_centroid_and_far_centroids():
     rng = np.random.default_rng(12)
     X = rng.standard_normal((2, 300, 128)).astype(np.float16)
@@ -437,6 +517,50 @@ def test_lloyd_tol_stops_when_the_centroids_settle_and_equals_plain_iterations(d
     _, C_next, _ = km.lloyd(Xg, C, 1)
     torch.cuda.synchronize()
     assert (_shift(C_next.cpu().numpy(), C.cpu().numpy()) <= 10 * tol).all()
+    assert km.device_fault() == 0
+
+
+@pytest.mark.parametrize("dt,d,K", [("f16", 128, 60), ("f32", 64, 40), ("f16", 1024, 30)])
+def test_lloyd_tol_stops_where_the_oracle_does_in_lock_step(dt, d, K):
+    """The stopping rule against the oracle: iteration by iteration the oracle takes the GPU's
+    centroids, checks that iteration's labels and update, and computes the shift of its own
+    update; the loop must stop after the first iteration whose shift is within tol in every
+    batch (oracle.lloyd_tol's rule), for a tol chosen away from every shift of the run."""
+    w = synth.small(B=2, N=3000, d=d, K=K, dtype=dt, ncomp=K, sigma=0.3, seed=4200 + d + K)
+    X = synth.points(w)
+    C0 = synth.init_centroids(w, X)
+    Xg = cuda(X)
+    Cs, shifts, labs = [C0], [], []
+    for t in range(12):
+        lab, C_next, _ = km.lloyd(Xg, cuda(Cs[-1]), 1)
+        torch.cuda.synchronize()
+        lab, C_next = lab.cpu().numpy(), C_next.cpu().numpy()
+        check_labels(X, Cs[-1], lab)
+        C_ref = check_centroids(X, lab, Cs[-1], C_next)
+        shifts.append(_shift(C_ref, Cs[-1]))  # the oracle's update of the GPU's centroids
+        labs.append(lab)
+        Cs.append(C_next)
+    S = np.array([s.max() for s in shifts])  # a batch stops the loop only with every other batch
+    # a tolerance a factor of 3 away from every shift up to the stop it causes, stopping after >= 2 iterations
+    best = None
+    for i in range(1, len(S) - 1):
+        tol = float(np.sqrt(S[i] * S[i + 1])) if S[i + 1] > 0 else S[i] / 9
+        T = next((t + 1 for t, s in enumerate(S) if s <= tol), None)
+        if T is None or T < 2 or tol <= 0:
+            continue
+        margin = min(abs(np.log(max(S[t], 1e-300) / tol)) for t in range(T))
+        if best is None or margin > best[2]:
+            best = (tol, T, margin)
+    assert best is not None and best[2] > np.log(3), f"no well-separated tolerance in shifts {S}"
+    tol, T, _ = best
+    lab_g, C_g, obj_g, n = km.lloyd_tol(Xg, cuda(C0), 12, tol)
+    torch.cuda.synchronize()
+    assert int(n.item()) == T, (int(n.item()), T, S, tol)
+    # its last labels match the oracle from the centroids before them, and its centroids those
+    # of the replay (checked against the oracle above; the two runs may differ in the last bits,
+    # where fp32 atomics add partial sums in another order)
+    check_labels(X, Cs[T - 1], lab_g.cpu().numpy())
+    np.testing.assert_allclose(C_g.cpu().numpy(), Cs[T], rtol=1e-4, atol=1e-6)
     assert km.device_fault() == 0
 
 

@@ -30,7 +30,8 @@ def noalloc(X, C, labels, mindist):
                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("dtype,d", [("f16", 128), ("f16", 96), ("f32", 16), ("f16", 256), ("f16", 1024)])
+@pytest.mark.parametrize("dtype,d", [("f16", 128), ("f16", 96), ("f32", 16), ("f32", 128), ("f16", 256),
+                                     ("f16", 1024)])
 def test_noalloc_matches_km_assign_on_two_calls_in_a_row(dtype, d):
     w = synth.small(B=3, N=2500, d=d, K=300, dtype=dtype, seed=777 + d)
     X = torch.from_numpy(synth.points(w)).cuda()
@@ -51,7 +52,7 @@ def test_noalloc_matches_km_assign_on_two_calls_in_a_row(dtype, d):
 def test_noalloc_rejects_problems_above_its_fixed_scratch():
     limit = km.lib().km_assign_noalloc_limit()
     assert limit == 16 << 20
-    B, K, d = 4, 32768, 128          # 2*B*K*d bytes = 32 MiB > 16 MiB
+    B, K, d = 4, 32768, 128          # 2*B*K*d bytes = 32 MiB > 16 MiB (fp16)
     X = torch.zeros((B, 256, d), dtype=torch.float16, device="cuda")
     C = torch.zeros((B, K, d), dtype=torch.float32, device="cuda")
     lab = torch.empty((B, 256), dtype=torch.int32, device="cuda")
