@@ -30,10 +30,9 @@ METRIC = "ms per Lloyd iter at B32·N65536·K1024·d128 fp16; assign/update % of
 UNIT = "ms/iter"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic of one launch on this workload (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu
-# captures summarised in profiles/assign_tc_kernel_b32_n65536_k1024_d128_f16.md and
-# profiles/update_kernel_b32_n65536_k1024_d128_f16.md, each valid only for the kernel source it was
-# taken on (sha1 of the .cu file); reported as null once that source changes.
+# DRAM traffic of one launch on this workload (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
+# capture of the assignment and of the update kernel, each valid only for the kernel sources it was
+# taken on (sha1 of each file); reported as null once one of them changes.
 ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "d275abe8a25de3841bb772b7c87659bb4b1d4ae0",
                             "tc_ptx.cuh": "cb7d62f9e816a6a9f946b8e125aa3e97e31fcd8e",
                             "km_internal.cuh": "a3d2b21c0f460ec27ddcc9a9b01915cf4424ca40"},
@@ -105,8 +104,11 @@ def work(w):
     flops_assign = 2.0 * B * N * K * d
     bytes_assign = B * N * (d * s + 8) + B * K * (d * s + 4)
     bytes_update = B * N * (d * s + 8) + 2 * B * K * d * 4 + 4 * B * K
-    passes = 2 if K > 256 else 1
-    bytes_sort = passes * B * N * 16 + B * N * 4
+    # the label sort: one pass (a thread-block cluster per batch) for batches of up to 65,536 labels
+    # below 1024 clusters, else LSD radix passes of at most 8 bits; 16 bytes per key and pass
+    bits = max(1, (K - 1).bit_length())
+    passes = 1 if (N <= 65536 and K <= 1024) else -(-bits // 8)
+    bytes_sort = passes * B * N * 16
     bytes_finalize = B * K * d * (4 + 4 + s) + B * K * 8
     return dict(flops_assign=flops_assign, bytes_assign=bytes_assign, bytes_update=bytes_update,
                 bytes_sort=bytes_sort, bytes_finalize=bytes_finalize)
@@ -157,73 +159,100 @@ class ClockSampler:
 
 # ---- CPU oracle baseline ----
 
-def cpu_oracle_ms_per_iter(w, X, C, rows: int):
-    """Time the oracle's assign + update over `rows` points of batch 0; extrapolate to one full iteration."""
-    import numpy as np
-    import oracle
-    sample_X = np.ascontiguousarray(X[:1, :rows])
-    t0 = time.perf_counter()
-    lab, _, _ = oracle.assign(sample_X, C[:1])
-    oracle.update(sample_X, lab, C[:1])
-    dt = time.perf_counter() - t0
-    scale = (w.B * w.N) / rows
-    return dt * scale * 1e3, dt, oracle.threads()
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
-def cpu_oracle_baseline(w, X, C, target_s: float = 12.0):
-    """The oracle's assign + update on a bounded sample of about `target_s` seconds: whole batches when
-    one batch fits in the budget (the whole workload when all do), else leading rows of batch 0.
-    Returns (ms per full iteration, seconds measured, threads, description of the sample)."""
-    import numpy as np
+def oracle_iteration(X, C):
+    """The oracle's assignment and update of the given problems (what one Lloyd iteration computes):
+    returns (seconds, labels, d1, d2)."""
     import oracle
-    probe = min(2048, w.N)
-    _, dt_probe, _ = cpu_oracle_ms_per_iter(w, X, C, probe)
-    fit = target_s * probe / max(dt_probe, 1e-9)
-    if fit >= w.N:
-        nb = int(min(w.B, fit // w.N))
-        sample_X, sample_C, rows = X[:nb], C[:nb], nb * w.N
-        what = (f"the whole iteration ({nb} of {w.B} problems)" if nb == w.B else
-                f"{nb} of the {w.B} problems, extrapolated x{w.B / nb:g}")
-    else:
-        rows = max(probe, int(fit))
-        sample_X, sample_C = np.ascontiguousarray(X[:1, :rows]), C[:1]
-        what = f"{rows} of the {w.B * w.N} points (batch 0), extrapolated x{w.B * w.N / rows:.1f}"
     t0 = time.perf_counter()
-    lab, _, _ = oracle.assign(sample_X, sample_C)
-    oracle.update(sample_X, lab, sample_C)
-    dt = time.perf_counter() - t0
-    ms = dt * 1e3 * (w.B * w.N) / rows
-    return ms, dt, oracle.threads(), f"oracle assign+update (K={w.K}, d={w.d}) on {what}: {dt:.2f} s measured"
+    lab, d1, d2 = oracle.assign(X, C)
+    oracle.update(X, lab, C)
+    return time.perf_counter() - t0, lab, d1, d2
+
+
+def oracle_problems(w, target_s: float) -> int:
+    """How many whole problems of the workload the oracle iterates in about target_s seconds (at least
+    one), from a timed probe of 2048 rows of one problem."""
+    import numpy as np
+    import synth
+    rows = min(2048, w.N)
+    Xp = synth.points(w.with_(B=1), 0, rows)
+    Cp = Xp[:, np.random.default_rng(0).choice(rows, min(w.K, rows), replace=False)].astype(np.float32)
+    if Cp.shape[1] < w.K:
+        Cp = np.concatenate([Cp] * (-(-w.K // Cp.shape[1])), axis=1)[:, :w.K].copy()
+    dt, *_ = oracle_iteration(Xp, Cp)
+    per_problem = dt * w.N / rows
+    return int(max(1, min(w.B, target_s // max(per_problem, 1e-9))))
+
+
+def cpu_sample_text(w, nb: int, dt: float) -> str:
+    part = "the whole iteration" if nb == w.B else f"{nb} of the {w.B} problems, scaled x{w.B / nb:g} to all {w.B}"
+    return (f"oracle assign+update (plain C++, fp64, K={w.K}, d={w.d}) of whole problems: {part}; "
+            f"{dt:.2f} s measured on {cpu_model()}")
 
 
 def run_reference(args, w):
-    """The oracle arm: plain C++ CPU Lloyd on bounded samples of the same workload."""
-    import numpy as np
+    """The oracle arm: the plain C++ CPU Lloyd iteration (assign + update) of the workload's problems, each
+    timed step the same whole problems as the cpu_baseline leg of the other arm (all of them when they
+    fit in about 12 s), measured; warm-up steps run one problem."""
     import synth
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    rows = min(16384, w.N)
-    wx = w.with_(B=1)
-    X = synth.points(wx, 0, rows)  # batch 0, first rows: same distribution as the full workload
-    rng = np.random.default_rng(0)
-    C = X[:, rng.choice(rows, w.K, replace=False)].astype(np.float32)
+    import oracle
+    nb = oracle_problems(w, 12.0)
+    wx = w.with_(B=nb)
+    X = synth.points(wx)
+    C = synth.init_centroids(wx, X)
+    for _ in range(args.warmup):
+        oracle_iteration(X[:1], C[:1])
     times = []
-    for i in range(args.warmup + args.steps):
-        ms, dt, cores = cpu_oracle_ms_per_iter(w, X, C, rows)
-        if i >= args.warmup:
-            times.append(ms)
-    v = statistics.mean(times)
-    sample = (f"each step: oracle assign+update of {rows} of the {w.B * w.N} points (batch 0) against all "
-              f"K={w.K} centroids, extrapolated linearly to the full iteration")
+    for _ in range(args.steps):
+        dt, *_ = oracle_iteration(X, C)
+        times.append(dt)
+    v = statistics.mean(times) * 1e3 * w.B / nb
     out = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-           "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "parallelism": "replicas"},
-           "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+           "config": bench_config(w, args.gpus),
+           "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                            "cpu": cpu_model(), "sample": cpu_sample_text(w, nb, statistics.mean(times))},
            "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0
+
+
+def bench_config(w, world: int) -> dict:
+    return {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "global_problems": w.B * world,
+            "parallelism": f"replicas{world}",
+            "l2": f"inputs larger than L2 (X is {w.B * w.N * w.d * w.elem_bytes / 2**20:.0f} MiB)"}
+
+
+def parity_report(w, X_host, C_host, gpu_labels, nb: int):
+    """The oracle's iteration of the first nb problems at the GPU's current centroids, timed (the CPU
+    baseline), and compared with the GPU's assignment there: labels must equal the oracle's at every
+    point whose relative top-2 gap (d2 - d1) / d2 is at least 1e-3 (fp16) or 1e-5 (fp32); the points
+    below it (near ties, where either label is allowed) are counted."""
+    import numpy as np
+    Xs, Cs = np.ascontiguousarray(X_host[:nb]), np.ascontiguousarray(C_host[:nb])
+    dt, lab, d1, d2 = oracle_iteration(Xs, Cs)
+    tau = 1e-3 if w.dtype == "f16" else 1e-5
+    gap = (d2 - d1) / np.maximum(d2, np.finfo(np.float64).tiny)
+    clear = gap >= tau
+    g = gpu_labels[:nb]
+    return dt, {"checked_points": int(lab.size), "near_tie_points": int((~clear).sum()),
+                "label_mismatches_at_clear_points": int((clear & (g != lab)).sum()),
+                "label_mismatches_at_near_ties": int((~clear & (g != lab)).sum()), "tau": tau}
 
 
 def run_ablations(w, X, C, labels, stream, calls: int = 3):
@@ -420,6 +449,10 @@ def run_ours(args, w):
                "d2h_bytes_per_step": int(lab_h.numel() * 4 + C_h.numel() * 4),
                "path": "km_lloyd(iters=1) on X in pinned host memory (chunked copies overlapped with the "
                        "kernels, labels written back to pinned host memory); C copied in and out"}
+    # the assignment at the run's final centroids, for the parity report against the oracle
+    lab_final, _ = km.assign(X, C)
+    torch.cuda.synchronize()
+    rescans = km.assign_rescans()
     ablations = None
     if not args.no_ablations and w.dtype == "f16":
         ablations = run_ablations(w, X, C, labels, stream)
@@ -442,50 +475,55 @@ def run_ours(args, w):
     t_other = phases["other"][0] / args.steps
     tflops = wk["flops_assign"] / (t_assign * 1e-3) / 1e12
     upd_gbs = wk["bytes_update"] / (t_update * 1e-3) / 1e9
-    # fp16 dense rate equals bf16.  The assignment is timed inside a long loop of back-to-back
-    # iterations that runs at the 1 kW power cap (sw_power_cap in the clock record; the SM clock
-    # settles near 1.4-1.7 GHz), so its denominator is the sustained GEMM figure; the burst figure
-    # is reported beside it.
-    peak_tf = peaks["bf16_tflops_sustained"]
-    peak_burst = peaks["bf16_tflops"]
+    # fp16 dense rate equals bf16.  The timed region is short (tens of milliseconds), so the
+    # denominator is the burst GEMM figure; the sustained (power-capped, seconds-long) figure is
+    # reported beside it.
+    peak_tf = peaks["bf16_tflops"]
+    peak_sus = peaks["bf16_tflops_sustained"]
     peak_bw = peaks["hbm_gbs"]
-    t_roof_burst = (max(wk["flops_assign"] / (peak_burst * 1e12), wk["bytes_assign"] / (peak_bw * 1e9)) +
-                    (wk["bytes_update"] + wk["bytes_sort"] + wk["bytes_finalize"]) / (peak_bw * 1e9)) * 1e3
+    t_roof_sus = (max(wk["flops_assign"] / (peak_sus * 1e12), wk["bytes_assign"] / (peak_bw * 1e9)) +
+                  (wk["bytes_update"] + wk["bytes_sort"] + wk["bytes_finalize"]) / (peak_bw * 1e9)) * 1e3
     t_roof = (max(wk["flops_assign"] / (peak_tf * 1e12), wk["bytes_assign"] / (peak_bw * 1e9)) +
               (wk["bytes_update"] + wk["bytes_sort"] + wk["bytes_finalize"]) / (peak_bw * 1e9)) * 1e3
     launches = sum(c for _, c in phases.values())
 
-    cpu = None
+    cpu = parity = None
     if not args.no_cpu and world == 1:
-        ms_cpu, dt, cores, what = cpu_oracle_baseline(w, X_host, C_init)
-        cpu = {"value": round(ms_cpu, 1), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": what}
+        import oracle
+        nb = oracle_problems(w, 12.0)
+        dt, parity = parity_report(w, X_host, C.cpu().numpy(), lab_final.cpu().numpy(), nb)
+        cpu = {"value": round(dt * 1e3 * w.B / nb, 1), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+               "cpu": cpu_model(), "sample": cpu_sample_text(w, nb, dt)}
+        parity["rescanned_points"] = rescans
+        parity["note"] = ("km_assign at the run's final centroids against the oracle's assignment of the same "
+                          "problems (the CPU baseline's run)")
 
     out = {
         "metric": METRIC, "value": round(ms_iter, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_iter, 4), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "N": w.N, "K": w.K, "d": w.d, "global_problems": w.B * world,
-                   "parallelism": f"replicas{world}",
-                   "l2": f"inputs larger than L2 (X is {w.B * w.N * w.d * w.elem_bytes / 2**20:.0f} MiB)"},
+        "config": bench_config(w, world),
         "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(tflops / peak_tf, 4), "traffic": traffic_for(ASSIGN_TRAFFIC, w.name),
                      "kernel": assign_kernel_name(w),
-                     "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate equals bf16); the kernel runs "
-                                    f"inside a long power-capped loop",
-                     "frac_of_burst_peak": round(tflops / peak_burst, 4), "burst_peak": peak_burst,
+                     "peak_source": f"{peak_src} bf16 burst (fp16 dense rate equals bf16)",
+                     "frac_of_sustained_peak": round(tflops / peak_sus, 4), "sustained_peak": peak_sus,
                      "ms_per_launch": round(t_assign, 4)},
         "roofline_update": {"bound": "hbm", "achieved": round(upd_gbs, 1), "peak": peak_bw, "unit": "GB/s",
                             "frac": round(upd_gbs / peak_bw, 4), "kernel": "update_kernel",
                             "traffic": traffic_for(UPDATE_TRAFFIC, w.name),
                             "ms_per_launch": round(t_update, 4), "peak_source": peak_src},
         "iteration_roofline": {"ms": round(t_roof, 4), "frac": round(t_roof / ms_iter, 4),
-                               "frac_with_burst_tensor_peak": round(t_roof_burst / ms_iter, 4)},
+                               "frac_with_sustained_tensor_peak": round(t_roof_sus / ms_iter, 4),
+                               "bytes": {k: v for k, v in wk.items() if k.startswith("bytes")},
+                               "flops_assign": wk["flops_assign"]},
         "phases_ms_per_iter": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
         "traced_ms_per_iter": round(traced_ms_iter, 4),
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "parity": parity,
         "ablations": ablations,
         "convergence": convergence,
         "device_fault": fault,

@@ -8,9 +8,10 @@ sums (fp32 [B,K,d]) and counts (int32 [B,K]) over the ranks, and every rank fina
 centroids.  The assignment needs no exchange (each point only meets the centroids), so the only
 traffic per iteration is 4*B*K*(d+1) bytes per rank, independent of N.
 
-The step functions are those of the library (`flashassign_b200.assign`, `update_sums`,
+The step functions are those of the library (`flashassign_b200.assign_objective`, `update_sums`,
 `finalize`) unless `ops` supplies others with the same signatures (the multi-process tests run the
-exchange logic on CPU ranks that way).  Every rank takes the same collective steps in the same order.
+exchange logic on CPU ranks that way); this module only moves their results between the ranks.
+Every rank takes the same collective steps in the same order.
 """
 from __future__ import annotations
 
@@ -20,8 +21,8 @@ from typing import Callable
 
 @dataclass(frozen=True)
 class Ops:
-    """The three per-rank steps: assign(X, C) -> (labels, mindist); update_sums(X, labels, K) ->
-    (sums, counts); finalize(sums, counts, C_prev) -> C_new."""
+    """The three per-rank steps: assign(X, C) -> (labels, objective [B] fp64 of this shard);
+    update_sums(X, labels, K) -> (sums, counts); finalize(sums, counts, C_prev) -> C_new."""
     assign: Callable
     update_sums: Callable
     finalize: Callable
@@ -29,7 +30,12 @@ class Ops:
 
 def library_ops() -> Ops:
     import flashassign_b200 as km
-    return Ops(assign=km.assign, update_sums=km.update_sums, finalize=km.finalize)
+
+    def assign(X, C):
+        labels, _, objective = km.assign_objective(X, C)
+        return labels, objective
+
+    return Ops(assign=assign, update_sums=km.update_sums, finalize=km.finalize)
 
 
 def lloyd_sharded(X_local, C_init, iters: int, group=None, ops: Ops | None = None):
@@ -46,9 +52,8 @@ def lloyd_sharded(X_local, C_init, iters: int, group=None, ops: Ops | None = Non
     objective = []
     labels = None
     for _ in range(iters):
-        labels, mindist = ops.assign(X_local, C)
+        labels, obj = ops.assign(X_local, C)
         sums, counts = ops.update_sums(X_local, labels, K)
-        obj = mindist.to(torch.float64).sum(dim=1)
         dist.all_reduce(sums, group=group)
         dist.all_reduce(counts, group=group)
         dist.all_reduce(obj, group=group)

@@ -85,3 +85,40 @@ def test_pageable_host_memory_is_rejected():
     with pytest.raises(km.KMError) as e:
         km.lloyd(X, C, 1, labels=torch.empty((1, 256), dtype=torch.int32).pin_memory())
     assert e.value.status == 2
+
+
+def test_host_pipeline_deadline_returns_timeout_then_recovers(monkeypatch):
+    """The pipeline's bounded host wait (KM_HOST_TIMEOUT_S): a deadline far shorter than the work makes
+    km_lloyd return KM_E_TIMEOUT instead of blocking; the work it enqueued still completes on the
+    stream, the scratch goes back to the pool, and the next call succeeds with the same results.
+    Host-side only: nothing on the GPU waits for anything that does not come."""
+    w = synth.small(B=2, N=200000, d=128, K=256, dtype="f16", ncomp=256, seed=47)
+    X = synth.points(w)
+    C0 = torch.from_numpy(synth.init_centroids(w, X)).cuda()
+    Xh = pinned(X)
+    lab_h = torch.empty((w.B, w.N), dtype=torch.int32).pin_memory()
+    km.lib().km_set_chunk_rows(25000)  # 8 chunks per batch
+    lab_ref, C_ref, _ = km.lloyd(Xh, C0, 2, labels=lab_h)
+    torch.cuda.synchronize()
+    lab_ref = lab_ref.clone()
+    km.lib().km_release_cached()
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+
+    monkeypatch.setenv("KM_HOST_TIMEOUT_S", "0.000001")
+    lab2 = torch.empty_like(lab_h).pin_memory()
+    with pytest.raises(km.KMError) as e:
+        km.lloyd(Xh, C0, 2, labels=lab2)
+    assert e.value.status == 5  # KM_E_TIMEOUT
+    assert b"still running" in km.lib().km_last_error()
+    torch.cuda.synchronize()  # the enqueued work completes
+    monkeypatch.delenv("KM_HOST_TIMEOUT_S")
+    assert km.device_fault() == 0
+    km.lib().km_release_cached()
+    torch.cuda.synchronize()
+    assert abs(torch.cuda.mem_get_info()[0] - free0) <= 8 << 20  # nothing kept beyond the pool's slack
+
+    lab3, C3, _ = km.lloyd(Xh, C0, 2, labels=torch.empty_like(lab_h).pin_memory())
+    torch.cuda.synchronize()
+    assert torch.equal(lab3, lab_ref)
+    torch.testing.assert_close(C3, C_ref, rtol=1e-5, atol=1e-6)

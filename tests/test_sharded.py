@@ -31,7 +31,7 @@ def _oracle_ops() -> Ops:
     def assign(X, C):
         B, N, _ = X.shape
         lab, d1, _ = oracle.assign(X.numpy(), C.numpy())
-        return torch.from_numpy(lab.reshape(B, N)), torch.from_numpy(d1.reshape(B, N))
+        return torch.from_numpy(lab.reshape(B, N)), torch.from_numpy(d1.reshape(B, N).sum(axis=1))
 
     def update_sums(X, labels, K):
         B, _, d = X.shape
