@@ -450,6 +450,7 @@ def run_ours(args, w):
                "path": "km_lloyd(iters=1) on X in pinned host memory (chunked copies overlapped with the "
                        "kernels, labels written back to pinned host memory); C copied in and out"}
     # the assignment at the run's final centroids, for the parity report against the oracle
+    km.assign_rescans()  # clear the count of the runs above
     lab_final, _ = km.assign(X, C)
     torch.cuda.synchronize()
     rescans = km.assign_rescans()

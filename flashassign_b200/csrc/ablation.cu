@@ -21,8 +21,8 @@ constexpr int kArgminThreads = 256;
 
 // One thread per point: column k of the scores is D[b][k][0..N), so the warp's
 // loads of one column are consecutive.  The best score (strict > over
-// ascending k keeps the lowest index among equal scores) is certified as in
-// the fused kernel; the rest go to the re-scan list.
+// ascending k keeps the lowest index among equal scores) and the second best
+// certify the label as in the fused kernel; the rest go to the re-scan list.
 __global__ void __launch_bounds__(kArgminThreads) dense_argmin_kernel(const float* __restrict__ D,
                                                                       const float* __restrict__ xnorm, int64_t N,
                                                                       int64_t K, int64_t Kp,
@@ -33,21 +33,22 @@ __global__ void __launch_bounds__(kArgminThreads) dense_argmin_kernel(const floa
     const int64_t b = blockIdx.y;
     const int64_t n = (int64_t)blockIdx.x * kArgminThreads + threadIdx.x;
     const bool valid = n < N;  // every lane stays for the warp-wide listing
-    float best = -INFINITY;
+    float best = -INFINITY, second = -INFINITY;
     int idx = -1;
     if (valid) {
         const float* d = D + b * Kp * N + n;
 #pragma unroll 8
         for (int64_t k = 0; k < K; ++k) {
             const float v = d[k * N];
+            second = fmaxf(second, fminf(best, v));
             if (v > best) {
                 best = v;
                 idx = (int)k;
             }
         }
     }
-    certify_best(list, list.cmax[b], b, N, n, valid, best, idx, valid ? xnorm[b * N + n] : 0.f, labels, mindist,
-                      threadIdx.x & 31);
+    certify_top2(list, list.cmax[b], b, N, n, valid, best, second, idx, valid ? xnorm[b * N + n] : 0.f, labels,
+                 mindist, threadIdx.x & 31);
 }
 
 template <typename T>

@@ -98,8 +98,9 @@ constexpr int kCOff = kXOff + kXBytes;
 constexpr int kCStageBytes = kMaxBoxes * kCBoxBytes + kCExtBytes;  // 36 KB: centroid boxes + norm slice
 constexpr int kCBytes = kCStages * kCStageBytes;                    // 144 KB
 constexpr int kAOnesOff = kCOff + kCBytes;                          // 4 KB of ones (the points' extra slice)
-constexpr int kMergeOff = kAOnesOff + kExtBytes;                    // 2 slots x 2 halves x 128 rows x (score, label)
-constexpr int kMergeBytes = 2 * kColParts * kRows * 8;
+constexpr int kMergeOff = kAOnesOff + kExtBytes;  // 2 slots x 2 halves x 128 rows x (best, second, label)
+constexpr int kMergeSlots = 2 * kColParts * kRows;
+constexpr int kMergeBytes = kMergeSlots * 12;
 constexpr int kBarOff = kMergeOff + kMergeBytes;
 // x_full/x_empty, c_full/c_empty, acc_full/acc_empty, merge handoff (2 slots x full/empty), x_used
 constexpr int kNumBars = 2 * kXBufs + 2 * kCStages + 2 * kAccSets + 4 + kXBufs;
@@ -157,8 +158,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t bar_x_used = bar_m_empty + 16;  // a unit's first tile of MMAs has completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBarOff + kNumBars * 8 + 4);
-    float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                 // [2][parts][128]
-    int* merge_label = reinterpret_cast<int*>(smem + kMergeOff + kMergeBytes / 2);  // [2][parts][128]
+    float* merge_score = reinterpret_cast<float*>(smem + kMergeOff);                      // [2][parts][128]
+    float* merge_second = reinterpret_cast<float*>(smem + kMergeOff + 4 * kMergeSlots);  // [2][parts][128]
+    int* merge_label = reinterpret_cast<int*>(smem + kMergeOff + 8 * kMergeSlots);       // [2][parts][128]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cta_rank();         // 0: leader CTA of the pair (issues the MMAs)
@@ -327,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         bool ok = true;
         const int units = (int)n_units, pairs = (int)P.pairs;  // < 2^23: 32-bit counters
         for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
-            float best = -INFINITY;
+            float best = -INFINITY, second = -INFINITY;
             int label = -1;    // column of the running best
             for (int kt = 0; kt < P.ktiles; ++kt, ++it_a) {
                 const uint32_t s = it_a % kAccSets;
@@ -353,29 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         for (int j = 0; j < kPartCols; ++j) out[(int64_t)j * P.N] = v[j];
                     }
                 } else {
-#pragma unroll
-                  for (int g = 0; g < kPartCols / 32; ++g) {
-                      const float* w = v + 32 * g;
-                      // two interleaved 3-input chains: few live temporaries
-                      float ga = max3(w[0], w[1], w[2]), gb = max3(w[3], w[4], w[5]);
-#pragma unroll
-                      for (int t = 6; t < 30; t += 4) {
-                          ga = max3(ga, w[t], w[t + 1]);
-                          gb = max3(gb, w[t + 2], w[t + 3]);
-                      }
-                      const float gmax = max3(max3(ga, w[30], w[31]), gb, gb);
-                      const bool better = gmax > best;  // strict: an earlier group keeps ties
-                      if (__any_sync(0xffffffffu, better)) {
-                          // the first column of the group holding its maximum
-                          int j0 = 31;
-#pragma unroll
-                          for (int j = 31; j >= 0; --j) j0 = (w[j] == gmax) ? j : j0;
-                          if (better) {
-                              best = gmax;
-                              label = kt * kTileK + h * kPartCols + g * 32 + j0;
-                          }
-                      }
-                  }
+                    top2_tile<kPartCols / 32>(v, kt * kTileK + h * kPartCols, best, second, label);
                 }
             }
             if (!ok) break;
@@ -385,6 +365,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if constexpr (!kDense) {
                 const int slot = ((int)ms * kColParts + h) * kRows + row;
                 merge_score[slot] = best;
+                merge_second[slot] = second;
                 merge_label[slot] = label;
             }
             __syncwarp();
@@ -443,22 +424,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
             double obj = 0.0;
             if constexpr (!kDense) {
-                float fb[kRows / 32];
+                float fb[kRows / 32], fs[kRows / 32];
                 int fl[kRows / 32];
 #pragma unroll
                 for (int rq = 0; rq < kRows / 32; ++rq) {
                     const int r = rq * 32 + lane;
-                    fb[rq] = merge_score[((int)ms * kColParts) * kRows + r];
-                    fl[rq] = merge_label[((int)ms * kColParts) * kRows + r];
+                    const int s0 = ((int)ms * kColParts) * kRows + r;
+                    fb[rq] = merge_score[s0];
+                    fs[rq] = merge_second[s0];
+                    fl[rq] = merge_label[s0];
 #pragma unroll
-                    for (int part = 1; part < kColParts; ++part) {
+                    for (int part = 1; part < kColParts; ++part) {  // slice 0 holds the lower columns
                         const int slot = ((int)ms * kColParts + part) * kRows + r;
-                        const float ob = merge_score[slot];
-                        const int ol = merge_label[slot];
-                        if (ob > fb[rq] || (ob == fb[rq] && ol >= 0 && (fl[rq] < 0 || ol < fl[rq]))) {
-                            fb[rq] = ob;
-                            fl[rq] = ol;
-                        }
+                        top2_join(fb[rq], fs[rq], fl[rq], merge_score[slot], merge_second[slot], merge_label[slot]);
                     }
                 }
                 __syncwarp();
@@ -466,8 +444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int rq = 0; rq < kRows / 32; ++rq) {
                     const int n = n0 + rq * 32 + lane;
-                    obj += certify_best(P.list, cmax2, b, P.N, n, n < P.N, fb[rq], fl[rq], xn[rq], P.labels,
-                                             P.mindist, lane);
+                    obj += certify_top2(P.list, cmax2, b, P.N, n, n < P.N, fb[rq], fs[rq], fl[rq], xn[rq], P.labels,
+                                        P.mindist, lane);
                 }
             } else {
                 __syncwarp();

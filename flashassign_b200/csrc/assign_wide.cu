@@ -268,9 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
-#pragma unroll
-                for (int g = 0; g < kPartCols / 32; ++g)
-                    top2_group(v + 32 * g, kt * kTileK + h * kPartCols + g * 32, best, second, label);
+top2_tile<kPartCols / 32>(v, kt * kTileK + h * kPartCols, best, second, label);
                 if (kt == 0) {
                     // The MMA has consumed this unit's X tile, so it is in place.
                     // ||x||^2 from it (half 0 of each row; the swizzle permutes
