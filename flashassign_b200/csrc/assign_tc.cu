@@ -337,14 +337,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 __syncwarp();  // tcgen05.ld below is warp-collective
                 tc_fence_after();
                 const uint32_t tcol = tmem_base + ((uint32_t)(q * 32) << 16) + s * kTileK + h * kPartCols;
-                // this warp's 128 columns in one load; the accumulator is handed
-                // back as soon as they are in registers, before their arithmetic
-                float v[kPartCols];
-                tmem_ld128(tcol, v);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
                 if constexpr (kDense) {
+                    // this warp's 128 columns in one load, the accumulator handed back at once
+                    float v[kPartCols];
+                    tmem_ld128(tcol, v);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
                     const int upb = (int)P.units_per_batch;
                     const int b = u / upb;
                     const int n = (u - b * upb) * kUnitRows + (int)rank * kRows + row;
@@ -355,7 +354,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         for (int j = 0; j < kPartCols; ++j) out[(int64_t)j * P.N] = v[j];
                     }
                 } else {
-                    top2_tile<kPartCols / 32>(v, kt * kTileK + h * kPartCols, best, second, label);
+                    // this warp's 128 columns in two loads of 64: the second is in flight
+                    // while the first half is reduced; the accumulator is handed back
+                    // once both are in registers
+                    uint32_t ra[kPartCols / 2], rb[kPartCols / 2];
+                    tmem_ld64_issue(tcol, ra);
+                    tmem_wait64(ra);
+                    tmem_ld64_issue(tcol + kPartCols / 2, rb);
+                    {
+                        float va[kPartCols / 2];
+#pragma unroll
+                        for (int j = 0; j < kPartCols / 2; ++j) va[j] = __uint_as_float(ra[j]);
+                        top2_tile<kPartCols / 64>(va, kt * kTileK + h * kPartCols, best, second, label);
+                    }
+                    tmem_wait64(rb);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
+                    float vb[kPartCols / 2];
+#pragma unroll
+                    for (int j = 0; j < kPartCols / 2; ++j) vb[j] = __uint_as_float(rb[j]);
+                    top2_tile<kPartCols / 64>(vb, kt * kTileK + h * kPartCols + kPartCols / 2, best, second, label);
                 }
             }
             if (!ok) break;
