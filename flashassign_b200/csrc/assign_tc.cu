@@ -89,6 +89,7 @@ constexpr int kMergeWarp = 11;                  // joins the halves, ||x||^2, ou
 constexpr int kEpiWarps = 8;                    // at most 3 warps per SMSP: up to 168 registers each
 constexpr int kColParts = kEpiWarps / 4;        // warps per TMEM lane quarter, each with a column slice
 constexpr int kPartCols = kTileK / kColParts;   // 128 columns of each tile per epilogue warp
+static_assert(kPartCols == 128, "the epilogue reduces 128-column slices (grid_rows, grid_top2)");
 constexpr uint32_t kTmemCols = 512;
 
 // shared memory map (offsets from a 1024-byte aligned base)
@@ -358,6 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     // while the first half is reduced; the accumulator is handed back
                     // once both are in registers
                     uint32_t ra[kPartCols / 2], rb[kPartCols / 2];
+                    float R[8], M[16];
                     tmem_ld64_issue(tcol, ra);
                     tmem_wait64(ra);
                     tmem_ld64_issue(tcol + kPartCols / 2, rb);
@@ -365,7 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         float va[kPartCols / 2];
 #pragma unroll
                         for (int j = 0; j < kPartCols / 2; ++j) va[j] = __uint_as_float(ra[j]);
-                        top2_tile<kPartCols / 64>(va, kt * kTileK + h * kPartCols, best, second, label);
+                        grid_rows<false>(va, R, M);
                     }
                     tmem_wait64(rb);
                     tc_fence_before();
@@ -374,7 +376,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     float vb[kPartCols / 2];
 #pragma unroll
                     for (int j = 0; j < kPartCols / 2; ++j) vb[j] = __uint_as_float(rb[j]);
-                    top2_tile<kPartCols / 64>(vb, kt * kTileK + h * kPartCols + kPartCols / 2, best, second, label);
+                    grid_rows<true>(vb, R, M);
+                    grid_top2(R, M, kt * kTileK + h * kPartCols, best, second, label);
                 }
             }
             if (!ok) break;

@@ -53,6 +53,7 @@ constexpr int kEpiWarp0 = 2;
 constexpr int kEpiWarps = 8;
 constexpr int kColParts = 2;                    // column halves per TMEM lane quarter
 constexpr int kPartCols = kTileK / kColParts;   // 128 columns of each tile per epilogue warp
+static_assert(kPartCols == 128, "the epilogue reduces 128-column slices (grid_rows, grid_top2)");
 constexpr uint32_t kTmemCols = 512;
 
 // shared memory map (offsets from a 1024-byte aligned base)
@@ -268,7 +269,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
-top2_tile<kPartCols / 32>(v, kt * kTileK + h * kPartCols, best, second, label);
+                top2_slice128(v, kt * kTileK + h * kPartCols, best, second, label);
                 if (kt == 0) {
                     // The MMA has consumed this unit's X tile, so it is in place.
                     // ||x||^2 from it (half 0 of each row; the swizzle permutes

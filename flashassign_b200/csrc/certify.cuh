@@ -15,12 +15,15 @@
 //     exact argmin o is at most 4e farther from the point than o, the exact
 //     second-smallest distance then exceeds 4e / tau, the exact relative
 //     top-2 gap of such a point is below tau, and the label is within tau d2
-//     of the smallest distance -- exact up to the label tolerance.
+//     of the smallest distance -- exact up to the label tolerance; a point
+//     whose best two scores are equal is never certified this way (its
+//     label would be a matter of index order, which the reductions leave to
+//     the re-scan).
 // The second test alone, made from the best score (d1 in place of d2), would
 // spare the second-best score but not cover a point lying on the centroid of
 // a one-member cluster (d1 = 0), which Lloyd iterations keep producing.  The
 // points neither test covers
-// (near ties, data far from the origin, norms beyond the folded term's range,
+// (near and exact ties, data far from the origin, norms beyond the folded term's range,
 // where the bound is +inf) are listed for the exact re-scan on the CUDA cores
 // (rescan.cu).
 #pragma once
@@ -35,75 +38,93 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// The best, the second-best (with multiplicity) and the index of the best of
-// one group of 32 scores w[0..31] of this lane's row, without branches.
-//
-// The group is read as a 4 x 8 grid (row r = w[8r .. 8r+7], column c =
-// w[c], w[8+c], w[16+c], w[24+c]).  Any element other than the maximum lies
-// in another grid row or another grid column than the maximum, so the
-// group's second-best value (with multiplicity: equal to the best when the
-// best occurs twice) is the larger of the second-largest row maximum and the
-// second-largest column maximum -- 12 maxima of 32 values instead of a scan.
-// The index is the lowest grid row and lowest grid column that reach the
-// maximum: the maximum's column when it occurs once (a repeated maximum has
-// g2 == g1, and the caller resolves it to its first column).
-__device__ __forceinline__ void group_top2(const float* w, float& g1, float& g2, int& gi) {
-    float R[4], M[8];
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-        R[r] = fmax3(fmax3(w[8 * r], w[8 * r + 1], w[8 * r + 2]), fmax3(w[8 * r + 3], w[8 * r + 4], w[8 * r + 5]),
-                     fmaxf(w[8 * r + 6], w[8 * r + 7]));
-#pragma unroll
-    for (int c = 0; c < 8; ++c) M[c] = fmax3(w[c], w[8 + c], fmaxf(w[16 + c], w[24 + c]));
-    const float ra = fmaxf(R[0], R[1]), rb = fmaxf(R[2], R[3]);
-    g1 = fmaxf(ra, rb);
-    const float r2 = fmax3(fminf(ra, rb), fminf(R[0], R[1]), fminf(R[2], R[3]));
-    const float ca = fmaxf(M[0], M[1]), cb = fmaxf(M[2], M[3]), cc = fmaxf(M[4], M[5]), cd = fmaxf(M[6], M[7]);
-    const float sab = fmax3(fminf(ca, cb), fminf(M[0], M[1]), fminf(M[2], M[3]));
-    const float scd = fmax3(fminf(cc, cd), fminf(M[4], M[5]), fminf(M[6], M[7]));
-    g2 = fmaxf(r2, fmax3(fminf(fmaxf(ca, cb), fmaxf(cc, cd)), sab, scd));
-    int rs = 3, cs = 7;
-    rs = R[2] == g1 ? 2 : rs;
-    rs = R[1] == g1 ? 1 : rs;
-    rs = R[0] == g1 ? 0 : rs;
-#pragma unroll
-    for (int c = 6; c >= 0; --c) cs = M[c] == g1 ? c : cs;
-    gi = 8 * rs + cs;
+__device__ __forceinline__ float fmax4(float a, float b, float c, float d) { return fmax3(a, b, fmaxf(c, d)); }
+
+// The largest of w[0..15] in eight instructions.
+__device__ __forceinline__ float max16(const float* w) {
+    const float a = fmax3(w[0], w[1], w[2]), b = fmax3(w[3], w[4], w[5]), c = fmax3(w[6], w[7], w[8]);
+    const float d = fmax3(w[9], w[10], w[11]), e = fmax3(w[12], w[13], w[14]);
+    return fmaxf(fmax3(a, b, c), fmax3(d, e, w[15]));
 }
 
-// A tile slice of kGroups * 32 scores v[] (columns col0 ...) folded into the
-// running (best, second, label): every group's (best, second, index) first,
-// with no branch between them, then the groups in ascending order (strict
-// improvement: an earlier group keeps an equal score).
-template <int kGroups>
-__device__ __forceinline__ void top2_tile(const float* v, int col0, float& best, float& second, int& label) {
-    float g1[kGroups], g2[kGroups];
-    int gi[kGroups];
+// The second-largest of four values, with multiplicity (equal to the largest
+// when it occurs twice): the smaller of the two pair maxima or the larger of
+// the two pair minima.
+__device__ __forceinline__ float second4(float a, float b, float c, float d) {
+    return fmax3(fminf(fmaxf(a, b), fmaxf(c, d)), fminf(a, b), fminf(c, d));
+}
+
+// 1.0f where a == b, else 0.0f: the comparison's outcome as a number, so that
+// the index below is summed on the FMA pipe rather than selected on the ALU
+// pipe, which the reduction already fills.
+__device__ __forceinline__ float eqf(float a, float b) {
+    float r;
+    asm("set.eq.f32.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// Top-2 of a 128-column slice of one row (scores v[0..127] of this lane's
+// point), read as an 8 x 16 grid: grid row r = v[16r .. 16r+15], grid column
+// c = v[c], v[16+c], ..., v[112+c].  Any score other than the maximum lies
+// in another grid row or another grid column than the maximum, so the
+// second-best score (with multiplicity) is the larger of the second-largest
+// row maximum and the second-largest column maximum; the rows and columns
+// cost about one instruction per score, and the two second-largest values
+// are taken the same way on the 8 row maxima (a 2 x 4 grid) and the 16
+// column maxima (a 4 x 4 grid).  When the maximum is unique, exactly one row
+// maximum and one column maximum (and one of each at the next level) equal
+// it, and their positions sum to its column; a repeated maximum leaves
+// second == best, which the certificate never accepts, so such a point goes
+// to the exact re-scan, which resolves the tie to the lowest index.
+//
+// grid_rows covers half of the grid, 64 scores (the first half: rows 0-3;
+// the second: rows 4-7), so that a kernel can reduce one half while the other
+// is still being loaded; grid_top2 then folds the slice (columns col0 ...)
+// into the running (best, second, label) of the point, an earlier slice
+// keeping an equal score.
+template <bool kSecondHalf>
+__device__ __forceinline__ void grid_rows(const float* v, float (&R)[8], float (&M)[16]) {
 #pragma unroll
-    for (int g = 0; g < kGroups; ++g) group_top2(v + 32 * g, g1[g], g2[g], gi[g]);
-    // a maximum held by two columns of a group (duplicate centroids, exact ties): its first column
-    bool tie = false;
+    for (int r = 0; r < 4; ++r) R[(kSecondHalf ? 4 : 0) + r] = max16(v + 16 * r);
 #pragma unroll
-    for (int g = 0; g < kGroups; ++g) tie = tie || (g2[g] == g1[g] && g1[g] > -INFINITY);
-    if (__any_sync(0xffffffffu, tie)) {
+    for (int c = 0; c < 16; ++c)
+        M[c] = kSecondHalf ? fmax3(fmax3(M[c], v[c], v[16 + c]), v[32 + c], v[48 + c])
+                           : fmax4(v[c], v[16 + c], v[32 + c], v[48 + c]);
+}
+
+__device__ __forceinline__ void grid_top2(const float (&R)[8], const float (&M)[16], int col0, float& best,
+                                          float& second, int& label) {
+    const float ra = fmax4(R[0], R[1], R[2], R[3]), rb = fmax4(R[4], R[5], R[6], R[7]);
+    const float g1 = fmaxf(ra, rb);
+    float Q[4], Nr[4], Nc[4];  // column maxima of the row maxima; row and column maxima of the column maxima
 #pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-            if (g2[g] == g1[g]) {
-                const float* w = v + 32 * g;
-                int j0 = 31;
-#pragma unroll
-                for (int j = 31; j >= 0; --j) j0 = (w[j] == g1[g]) ? j : j0;
-                gi[g] = j0;
-            }
-        }
+    for (int i = 0; i < 4; ++i) {
+        Q[i] = fmaxf(R[i], R[4 + i]);
+        Nr[i] = fmax4(M[4 * i], M[4 * i + 1], M[4 * i + 2], M[4 * i + 3]);
+        Nc[i] = fmax4(M[i], M[4 + i], M[8 + i], M[12 + i]);
     }
+    const float g2 = fmax3(fminf(ra, rb), fmaxf(second4(Q[0], Q[1], Q[2], Q[3]), second4(Nr[0], Nr[1], Nr[2], Nr[3])),
+                           second4(Nc[0], Nc[1], Nc[2], Nc[3]));
+    // column of the maximum = 16 (4 [rb] + i[Q]) + 4 i[Nr] + i[Nc], summed from 2^23 so that its bits
+    // are 0x4B000000 + the column
+    float acc = fmaf(eqf(rb, g1), 64.f, 0x1p23f);
 #pragma unroll
-    for (int g = 0; g < kGroups; ++g) {
-        const bool better = g1[g] > best;
-        label = better ? col0 + 32 * g + gi[g] : label;
-        second = fmax3(fminf(best, g1[g]), second, g2[g]);
-        best = fmaxf(best, g1[g]);
+    for (int i = 1; i < 4; ++i) {
+        acc = fmaf(eqf(Q[i], g1), 16.f * i, acc);
+        acc = fmaf(eqf(Nr[i], g1), 4.f * i, acc);
+        acc = fmaf(eqf(Nc[i], g1), (float)i, acc);
     }
+    label = g1 > best ? __float_as_int(acc) + (col0 - 0x4B000000) : label;
+    second = fmax3(fminf(best, g1), second, g2);
+    best = fmaxf(best, g1);
+}
+
+// grid_rows and grid_top2 over a slice that is all in registers.
+__device__ __forceinline__ void top2_slice128(const float* v, int col0, float& best, float& second, int& label) {
+    float R[8], M[16];
+    grid_rows<false>(v, R, M);
+    grid_rows<true>(v + 64, R, M);
+    grid_top2(R, M, col0, best, second, label);
 }
 
 // Joins two partial results of one row; (best, second, label) holds the lower
@@ -128,7 +149,7 @@ __device__ __forceinline__ double certify_top2(const RescanList& L, float cmax2,
                                                int32_t* __restrict__ labels, float* __restrict__ mindist, int lane) {
     const float e = L.err * fmaf(0.5f, xnorm, cmax2);  // >= err (||x|| cmax + cmax^2/2)
     const float d2 = fmaf(-2.f, second, xnorm);
-    const bool certified = best - second > 2.f * e || d2 > fmaf(L.c_x, xnorm, L.c_c * cmax2);
+    const bool certified = best - second > 2.f * e || (best > second && d2 > fmaf(L.c_x, xnorm, L.c_c * cmax2));
     const bool listed = valid && !certified;
     const float md = fmaxf(fmaf(-2.f, best, xnorm), 0.f);
     if (valid && certified) {
