@@ -206,6 +206,10 @@ struct TcScratch {
     int32_t* flag_rows = nullptr;   // [lists, cap]
     int64_t lists = 0, cap = 0;
     int parity = 0;                 // the counter set the next assignment appends to
+    // ||x||^2 of every point ([B, N], nullable): the first assignment of a
+    // loop over the same X writes it, the later ones read it
+    float* xnorm = nullptr;
+    bool xnorm_valid = false;
     // batch b alone: its prepared centroids; the chunk pipeline (one batch at a
     // time, lists == 1) keeps the single list, which serves every chunk in turn
     TcScratch batch(int64_t b, int64_t K, int64_t d, int dtype) const {
@@ -219,6 +223,8 @@ struct TcScratch {
             t.prep.cext = static_cast<float*>(prep.cext) + b * Kp * 8;
         }
         t.prep.cmax = prep.cmax + b;
+        t.xnorm = nullptr;  // the norms are kept for whole loops over all batches only
+        t.xnorm_valid = false;
         return t;
     }
 };
@@ -299,7 +305,10 @@ km_status run_assign(const void* X, int dtype, const float* C, TcScratch* tc, in
             e = launch_assign_wide(Xh, chat, cext, B, N, K, d, labels, mindist, obj_acc, L, dev.sms, st, stop);
             what = "assign (tensor cores, d split in chunks)";
         } else {
-            e = launch_assign_tc(Xh, chat, cext, B, N, K, d, labels, mindist, obj_acc, L, dev.sms, st, stop);
+            const bool have = tc->xnorm && tc->xnorm_valid;
+            e = launch_assign_tc(Xh, chat, cext, B, N, K, d, labels, mindist, obj_acc, L, dev.sms, st, stop,
+                                 have ? tc->xnorm : nullptr, have ? nullptr : tc->xnorm);
+            tc->xnorm_valid = tc->xnorm != nullptr;
             what = "assign (tensor cores)";
         }
     } else {
@@ -501,6 +510,8 @@ km_status lloyd_device(const void* X, int64_t B, int64_t N, int64_t K, int64_t d
     int32_t* stop = nullptr;
     double* shift = nullptr;
     if (tc) KM_TRY(alloc_tc(scratch, dtype, B, K, d, B, N, st, &tcs));
+    if (tc && dtype == KM_F16 && assign_tc_supported(d, dtype))  // X is the same in every iteration
+        KM_TRY(scratch.get(&tcs.xnorm, (size_t)(B * N), "point norms"));
     if (cv) {
         KM_TRY(scratch.get(&stop, 1, "stop flag"));
         KM_TRY(scratch.get(&shift, (size_t)B, "centroid shifts"));

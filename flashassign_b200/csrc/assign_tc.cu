@@ -131,7 +131,8 @@ struct Params {
     float* mindist;
     double* obj_acc;  // [B] running sum of minimum distances, nullable
     float* dense;     // dense mode: [B, padded K, N] scores, written instead of reduced
-    float* xnorm;     // dense mode: [B, N] ||x||^2
+    float* xnorm;     // [B, N] ||x||^2, written when non-null (always in dense mode)
+    const float* xnorm_in;  // [B, N] ||x||^2 of these points from an earlier launch (nullable): read, not computed
     const int32_t* stop;  // nullable: when *stop, the launch does nothing
     int32_t* fault;
     RescanList list;      // the points left to the exact re-scan
@@ -170,7 +171,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kXBufs; ++i) {
             mbar_init(bar_x_full + 8 * i, 1);               // leader: its expect_tx; bytes from both CTAs
-            mbar_init(bar_x_empty + 8 * i, 3);              // both issuers' end-of-unit commits + the merge warp
+            // both issuers' end-of-unit commits, and the merge warp once it has
+            // read ||x||^2 from the buffer (not when the norms are given)
+            mbar_init(bar_x_empty + 8 * i, P.xnorm_in ? 2 : 3);
         }
         for (int i = 0; i < kCStages; ++i) {
             mbar_init(bar_c_full + 8 * i, 1);
@@ -311,7 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                   1u);
                     if (release_c) umma_commit_pair(bar_c_empty + 8 * cs);
                     umma_commit_pair(bar_acc_full + 8 * s);
-                    if (kt == 0) umma_commit_pair(bar_x_used + 8 * xb);  // the unit's X tile is in place
+                    if (kt == 0 && !P.xnorm_in) umma_commit_pair(bar_x_used + 8 * xb);  // the unit's X tile is in place
                 }
                 if (ok) umma_commit_pair(bar_x_empty + 8 * xb);
             }
@@ -355,29 +358,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         for (int j = 0; j < kPartCols; ++j) out[(int64_t)j * P.N] = v[j];
                     }
                 } else {
-                    // this warp's 128 columns in two loads of 64: the second is in flight
-                    // while the first half is reduced; the accumulator is handed back
-                    // once both are in registers
-                    uint32_t ra[kPartCols / 2], rb[kPartCols / 2];
-                    float R[8], M[16];
-                    tmem_ld64_issue(tcol, ra);
-                    tmem_wait64(ra);
-                    tmem_ld64_issue(tcol + kPartCols / 2, rb);
-                    {
-                        float va[kPartCols / 2];
-#pragma unroll
-                        for (int j = 0; j < kPartCols / 2; ++j) va[j] = __uint_as_float(ra[j]);
-                        grid_rows<false>(va, R, M);
-                    }
-                    tmem_wait64(rb);
+                    // this warp's 128 columns in one load; the accumulator is handed
+                    // back as soon as they are in registers, and reduced after
+                    float v[kPartCols];
+                    tmem_ld128(tcol, v);
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8 * s);
-                    float vb[kPartCols / 2];
-#pragma unroll
-                    for (int j = 0; j < kPartCols / 2; ++j) vb[j] = __uint_as_float(rb[j]);
-                    grid_rows<true>(vb, R, M);
-                    grid_top2(R, M, kt * kTileK + h * kPartCols, best, second, label);
+                    top2_slice128(v, kt * kTileK + h * kPartCols, best, second, label);
                 }
             }
             if (!ok) break;
@@ -411,37 +399,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int n0 = (u - b * upb) * kUnitRows + (int)rank * kRows;
             float cmax2 = 0.f;  // the batch's norm bound, loaded while the unit runs
             if constexpr (!kDense) cmax2 = P.list.cmax[b];
-            // ||x||^2 as soon as the unit's first tile of MMAs has completed
-            // (its X tile is then in place in both CTAs); the X buffer is
-            // released right after, while the unit's other tiles run
-            if (!(ok = mbar_wait(bar_x_used + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
             float xn[kRows / 32];
+            if (P.xnorm_in) {
+                // given: loaded now, used at the unit's end (the X buffer is the issuers' alone)
 #pragma unroll
-            for (int rq = 0; rq < kRows / 32; ++rq) {
-                const int r = rq * 32 + lane;
-                float xnorm = 0.f;
-                for (int kb = 0; kb < boxes; ++kb) {
-                    const uint4* rowp =
-                        reinterpret_cast<const uint4*>(smem + kXOff + (xb * kMaxBoxes + kb) * kBoxBytes + r * 128);
+                for (int rq = 0; rq < kRows / 32; ++rq) {
+                    const int n = n0 + rq * 32 + lane;
+                    xn[rq] = n < P.N ? P.xnorm_in[(int64_t)b * P.N + n] : 0.f;
+                }
+            } else {
+                // ||x||^2 as soon as the unit's first tile of MMAs has completed
+                // (its X tile is then in place in both CTAs); the X buffer is
+                // released right after, while the unit's other tiles run
+                if (!(ok = mbar_wait(bar_x_used + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
 #pragma unroll
-                    for (int cch = 0; cch < 8; ++cch) {
-                        const uint4 xv = rowp[(cch + lane) & 7];  // lanes start on different banks
-                        const __half2* hh = reinterpret_cast<const __half2*>(&xv);
+                for (int rq = 0; rq < kRows / 32; ++rq) {
+                    const int r = rq * 32 + lane;
+                    float xnorm = 0.f;
+                    for (int kb = 0; kb < boxes; ++kb) {
+                        const uint4* rowp =
+                            reinterpret_cast<const uint4*>(smem + kXOff + (xb * kMaxBoxes + kb) * kBoxBytes + r * 128);
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const float2 f = __half22float2(hh[t]);
-                            xnorm = fmaf(f.x, f.x, xnorm);
-                            xnorm = fmaf(f.y, f.y, xnorm);
+                        for (int cch = 0; cch < 8; ++cch) {
+                            const uint4 xv = rowp[(cch + lane) & 7];  // lanes start on different banks
+                            const __half2* hh = reinterpret_cast<const __half2*>(&xv);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const float2 f = __half22float2(hh[t]);
+                                xnorm = fmaf(f.x, f.x, xnorm);
+                                xnorm = fmaf(f.y, f.y, xnorm);
+                            }
                         }
                     }
+                    xn[rq] = xnorm;
+                    if (P.xnorm && n0 + r < P.N) P.xnorm[(int64_t)b * P.N + n0 + r] = xnorm;
                 }
-                xn[rq] = xnorm;
-                if constexpr (kDense) {
-                    if (n0 + r < P.N) P.xnorm[(int64_t)b * P.N + n0 + r] = xnorm;
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);
             // the unit's results, once every epilogue warp has posted its column slice
             if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
             double obj = 0.0;
@@ -502,7 +497,7 @@ bool assign_tc_supported(int64_t d, int dtype) { return dtype == KM_F16 && d >= 
 template <bool kDense>
 cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
                       int64_t d, int32_t* labels, float* mindist, double* obj_acc, const RescanList& list, float* dense,
-                      float* xnorm, int sms, cudaStream_t st, const int32_t* stop) {
+                      float* xnorm, const float* xnorm_in, int sms, cudaStream_t st, const int32_t* stop) {
     if (!assign_tc_supported(d, KM_F16)) return cudaErrorNotSupported;
     CUtensorMap mx, mc, me;
     if (!make_map(&mx, X, 2, B, N, d, kBoxK, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -525,6 +520,7 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
     P.obj_acc = obj_acc;
     P.dense = dense;
     P.xnorm = xnorm;
+    P.xnorm_in = xnorm_in;
     P.stop = stop;
     P.fault = fault_word();
     P.list = list;
@@ -537,16 +533,16 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
 
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
                              int64_t d, int32_t* labels, float* mindist, double* obj_acc, const RescanList& list,
-                             int sms, cudaStream_t st, const int32_t* stop) {
+                             int sms, cudaStream_t st, const int32_t* stop, const float* xnorm_in, float* xnorm_out) {
     if (!list.cmax || !list.count || !list.rows) return cudaErrorInvalidValue;
-    return launch_tc<false>(X, chat, cext, B, N, K, d, labels, mindist, obj_acc, list, nullptr, nullptr, sms, st,
-                            stop);
+    return launch_tc<false>(X, chat, cext, B, N, K, d, labels, mindist, obj_acc, list, nullptr, xnorm_out, xnorm_in,
+                            sms, st, stop);
 }
 
 cudaError_t launch_assign_tc_dense(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N,
                                    int64_t K, int64_t d, float* dense, float* xnorm, int sms, cudaStream_t st) {
-    return launch_tc<true>(X, chat, cext, B, N, K, d, nullptr, nullptr, nullptr, RescanList(), dense, xnorm, sms, st,
-                           nullptr);
+    return launch_tc<true>(X, chat, cext, B, N, K, d, nullptr, nullptr, nullptr, RescanList(), dense, xnorm, nullptr,
+                           sms, st, nullptr);
 }
 
 }  // namespace km

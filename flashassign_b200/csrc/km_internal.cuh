@@ -174,9 +174,14 @@ bool assign_tc_supported(int64_t d, int dtype);
 // Points that the scores' error bound (list.err, list.cmax) does not certify
 // (certify.cuh) are not resolved: they are appended to `list`
 // (its counters zero on entry) for launch_rescan and left out of obj_acc.
+// xnorm_out (nullable, [B, N]) receives ||x||^2 of every point; xnorm_in
+// (nullable) gives them, as an earlier launch on the same X wrote them, so
+// that the kernel reads instead of computing them and releases each X tile
+// as soon as its MMAs are done.
 cudaError_t launch_assign_tc(const __half* X, const __half* chat, const __half* cext, int64_t B, int64_t N, int64_t K,
                              int64_t d, int32_t* labels, float* mindist, double* obj_acc, const RescanList& list,
-                             int sms, cudaStream_t st, const int32_t* stop = nullptr);
+                             int sms, cudaStream_t st, const int32_t* stop = nullptr,
+                             const float* xnorm_in = nullptr, float* xnorm_out = nullptr);
 
 // Tensor-core assignment of wide fp16 points (128 < d <= 512, d % 64 == 0):
 // the centroid tiles stream in 64-dimension chunks, the points stay resident.
