@@ -88,6 +88,7 @@ constexpr int kMmaWarpB = 10;                   // second issuer, on another SMS
 constexpr int kMergeWarp = 11;                  // joins the halves, ||x||^2, outputs (warps go in fours: no extra registers)
 constexpr int kEpiWarps = 8;                    // at most 3 warps per SMSP: up to 168 registers each
 constexpr int kColParts = kEpiWarps / 4;        // warps per TMEM lane quarter, each with a column slice
+constexpr int kMaxKSteps = kMaxBoxes * kBoxK / 16;  // K=16 MMA steps of the widest points (d = 128)
 constexpr int kPartCols = kTileK / kColParts;   // 128 columns of each tile per epilogue warp
 static_assert(kPartCols == 128, "the epilogue reduces 128-column slices (grid_rows, grid_top2)");
 constexpr uint32_t kTmemCols = 512;
@@ -223,17 +224,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // lane 16 streams the units' X tiles (a unit ahead, so HBM latency is
         // hidden behind a whole unit of MMAs); lane 0 streams the centroid
         // tiles and their norm slices through the 4-stage ring.
+        const int units = (int)n_units, pairs = (int)P.pairs, upb = (int)P.units_per_batch;  // < 2^23
         if (lane == 16) {
             uint32_t it_x = 0;
-            for (int64_t u = pair; u < n_units; u += P.pairs, ++it_x) {
-                const int b = (int)(u / P.units_per_batch);
-                const int n0 = (int)((u % P.units_per_batch) * kUnitRows) + (int)rank * kRows;
+            int b = (int)pair / upb, r = (int)pair % upb;  // unit u's batch and index in it, carried along
+            for (int u = (int)pair; u < units; u += pairs, ++it_x) {
+                const int n0 = r * kUnitRows + (int)rank * kRows;
                 const uint32_t xb = it_x % kXBufs;
                 if (!mbar_wait(bar_x_empty + 8 * xb, ((it_x / kXBufs) & 1) ^ 1, abort_flag, P.fault)) break;
                 if (rank == 0) mbar_expect_tx(bar_x_full + 8 * xb, x_bytes_pair);
                 const uint32_t xfull_leader = map_to_rank(bar_x_full + 8 * xb, 0);
                 for (int kb = 0; kb < boxes; ++kb)
                     tma_load_pair(x_base + (xb * kMaxBoxes + kb) * kBoxBytes, &tmap_x, kb * kBoxK, n0, b, xfull_leader);
+                r += pairs;
+                if (r >= upb) {
+                    b += r / upb;
+                    r %= upb;
+                }
             }
         } else if (lane == 0) {
             // Resident mode (an even number of tiles, at most one per stage): tile
@@ -244,8 +251,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t it_c = 0, ep = 0;
             int prev_b = -1;
             bool ok = true;
-            for (int64_t u = pair; u < n_units && ok; u += P.pairs) {
-                const int b = (int)(u / P.units_per_batch);
+            for (int u = (int)pair; u < units && ok; u += pairs) {
+                const int b = u / upb;
                 if (P.resident) {
                     if (b == prev_b) continue;  // this batch's tiles are in place
                     if (prev_b >= 0) ++ep;
@@ -275,20 +282,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t mine = warp == 1 ? 0u : 1u;
         if (rank == 0 && lane == 0) {
             uint32_t it_x = 0, it_c = 0, it_a = 0, ep = 0;
-            int prev_b = -1;
             bool ok = true;
-            for (int64_t u = pair; u < n_units && ok; u += P.pairs, ++it_x) {
-                const uint32_t xb = it_x % kXBufs;
-                const int b = (int)(u / P.units_per_batch);
-                if (P.resident && b != prev_b) {
-                    if (prev_b >= 0) ++ep;
-                    prev_b = b;
+            // 32-bit unit counters (< 2^23), and unit u's batch b and index r in it
+            // carried along as u advances: no division between two units' MMAs
+            const int units = (int)n_units, pairs = (int)P.pairs, upb = (int)P.units_per_batch;
+            int b = (int)pair / upb, r = (int)pair % upb;
+            for (int u = (int)pair; u < units && ok; u += pairs, ++it_x) {
+                int nb = b, nr = r + pairs;  // the next unit's batch and index
+                if (nr >= upb) {
+                    nb += nr / upb;
+                    nr %= upb;
                 }
+                const uint32_t xb = it_x % kXBufs;
                 // resident mode: the stages are released only after the epoch's last unit
                 // (with an even tile count each stage has one issuer, whose commit covers
                 // all of its earlier MMAs on that stage)
-                const bool release_c =
-                    !P.resident || u + P.pairs >= n_units || (int)((u + P.pairs) / P.units_per_batch) != b;
+                const bool release_c = !P.resident || u + pairs >= units || nb != b;
                 if (!(ok = mbar_wait(bar_x_full + 8 * xb, (it_x / kXBufs) & 1, abort_flag, P.fault))) break;
                 const uint64_t a_desc0 = umma_desc_sw128(x_base + xb * kMaxBoxes * kBoxBytes);
                 for (int kt = 0; kt < P.ktiles; ++kt, ++it_c, ++it_a) {
@@ -303,11 +312,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t d_tmem = tmem_base + s * kTileK;
                     const uint32_t stage = c_base + cs * kCStageBytes;
                     const uint64_t b_desc0 = umma_desc_sw128(stage);
-                    for (int ks = 0; ks < P.ksteps; ++ks) {
-                        // start-address field advance (16-byte units): box, then 32 bytes per K=16 step
-                        const uint64_t a_off = (uint64_t)(((ks >> 2) * kBoxBytes + (ks & 3) * 32) >> 4);
-                        const uint64_t b_off = (uint64_t)(((ks >> 2) * kCBoxBytes + (ks & 3) * 32) >> 4);
-                        umma_pair_f16(d_tmem, a_desc0 + a_off, b_desc0 + b_off, ks > 0 ? 1u : 0u);
+                    // unrolled, so that each step's descriptor offsets are immediates: one
+                    // thread issues a tcgen05.mma only about every 100 cycles at best
+#pragma unroll
+                    for (int ks = 0; ks < kMaxKSteps; ++ks) {
+                        if (ks < P.ksteps) {
+                            // start-address field advance (16-byte units): box, then 32 bytes per K=16 step
+                            const uint64_t a_off = (uint64_t)(((ks >> 2) * kBoxBytes + (ks & 3) * 32) >> 4);
+                            const uint64_t b_off = (uint64_t)(((ks >> 2) * kCBoxBytes + (ks & 3) * 32) >> 4);
+                            umma_pair_f16(d_tmem, a_desc0 + a_off, b_desc0 + b_off, ks > 0 ? 1u : 0u);
+                        }
                     }
                     // the norm slice: ones (points) x (-||c||^2/2 pieces) (centroids)
                     umma_pair_f16(d_tmem, umma_desc_sw32(ones_base), umma_desc_sw32(stage + kMaxBoxes * kCBoxBytes),
@@ -317,6 +331,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (kt == 0 && !P.xnorm_in) umma_commit_pair(bar_x_used + 8 * xb);  // the unit's X tile is in place
                 }
                 if (ok) umma_commit_pair(bar_x_empty + 8 * xb);
+                if (P.resident && nb != b) ++ep;  // the next unit starts a new epoch
+                b = nb;
+                r = nr;
             }
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
@@ -511,6 +528,7 @@ cudaError_t launch_tc(const __half* X, const __half* chat, const __half* cext, i
     P.B = B; P.N = N; P.K = K; P.d = d;
     P.units_per_batch = ceil_div(N, kUnitRows);
     P.units = B * P.units_per_batch;
+    if (P.units >= (int64_t(1) << 30)) return cudaErrorInvalidValue;  // the kernel counts units in 32 bits
     P.ktiles = (int)ceil_div(K, kTileK);
     P.ksteps = (int)ceil_div(d, 16);
     P.boxes = (int)ceil_div(d, kBoxK);
