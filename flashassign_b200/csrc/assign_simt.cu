@@ -95,10 +95,10 @@ __global__ void __launch_bounds__(kThreads) assign_simt_kernel(const T* __restri
             if (mindist) mindist[b * N + i] = best;
         }
         if (obj_acc) {  // the objective: one atomic per warp
-            double part = mine ? (double)best : 0.0;
+            float part = mine ? best : 0.f;  // fp32 within the warp, fp64 across
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if ((threadIdx.x & 31) == 0) atomicAdd(obj_acc + b, part);
+            if ((threadIdx.x & 31) == 0) atomicAdd(obj_acc + b, (double)part);
         }
     }
 }

@@ -335,12 +335,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(bar_m_empty + 8 * ms);
                 top2_join(best, second, label, ob, os, ol);  // this half holds the lower columns
                 const int n = nq + lane;
-                double part = certify_top2(P.list, P.list.cmax[b], b, P.N, n, n < P.N, best, second, label, xnorm,
+                float part = certify_top2(P.list, P.list.cmax[b], b, P.N, n, n < P.N, best, second, label, xnorm,
                                                 P.labels, P.mindist, lane);
                 if (P.obj_acc) {  // the objective: this warp's certified rows, one atomic per warp
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-                    if (lane == 0) atomicAdd(P.obj_acc + b, part);
+                    if (lane == 0) atomicAdd(P.obj_acc + b, (double)part);
                 }
             }
         }

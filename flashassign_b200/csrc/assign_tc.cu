@@ -456,7 +456,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             // the unit's results, once every epilogue warp has posted its column slice
             if (!(ok = mbar_wait(bar_m_full + 8 * ms, mph, abort_flag, P.fault))) break;
-            double obj = 0.0;
+            float obj = 0.f;  // the unit's certified rows' share of the objective
             if constexpr (!kDense) {
                 float fb[kRows / 32], fs[kRows / 32];
                 int fl[kRows / 32];
@@ -488,7 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!kDense && P.obj_acc) {  // the objective of the unit's certified rows, one atomic
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) obj += __shfl_xor_sync(0xffffffffu, obj, o);
-                if (lane == 0) atomicAdd(P.obj_acc + b, obj);
+                if (lane == 0) atomicAdd(P.obj_acc + b, (double)obj);
             }
         }
     }

@@ -395,10 +395,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (P.mindist) P.mindist[o64] = md;
                 }
                 if (P.obj_acc) {  // the resolved points' share of the objective: one atomic per warp
-                    double part = (valid && !listed) ? (double)md : 0.0;
+                    float part = (valid && !listed) ? md : 0.f;  // fp32 within the warp, fp64 across
 #pragma unroll
                     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-                    if (lane == 0) atomicAdd(P.obj_acc + b, part);
+                    if (lane == 0) atomicAdd(P.obj_acc + b, (double)part);
                 }
                 const unsigned mask = __ballot_sync(0xffffffffu, listed);
                 if (mask) {

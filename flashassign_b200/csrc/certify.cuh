@@ -140,11 +140,13 @@ __device__ __forceinline__ void top2_join(float& best, float& second, int& label
 // label and mindist = ||x||^2 - 2 best, and its mindist is returned as its
 // share of the objective; the others are listed (one atomic per warp, every
 // lane of the warp calling) and left to the re-scan, which writes all three;
-// 0 is returned for them.  NaN or -inf scores are never certified.  cmax2:
+// 0 is returned for them (the caller sums the shares in fp32 and adds the
+// sum to the fp64 accumulator: fp64 arithmetic in the per-unit path measured
+// ~13% of the iteration).  NaN or -inf scores are never certified.  cmax2:
 // the batch's bound of max_k ||c_k||^2 (+inf: certify nothing); the error
 // bound e is taken as err (||x||^2/2 + cmax^2) >= err (||x|| cmax + cmax^2/2),
 // which needs no square root.
-__device__ __forceinline__ double certify_top2(const RescanList& L, float cmax2, int64_t b, int64_t N, int64_t n,
+__device__ __forceinline__ float certify_top2(const RescanList& L, float cmax2, int64_t b, int64_t N, int64_t n,
                                                bool valid, float best, float second, int label, float xnorm,
                                                int32_t* __restrict__ labels, float* __restrict__ mindist, int lane) {
     const float e = L.err * fmaf(0.5f, xnorm, cmax2);  // >= err (||x|| cmax + cmax^2/2)
@@ -167,7 +169,7 @@ __device__ __forceinline__ double certify_top2(const RescanList& L, float cmax2,
         base = __shfl_sync(0xffffffffu, base, 0) + __popc(mask & ((1u << lane) - 1u));
         if (listed && base < L.cap) L.rows[b * L.cap + base] = (int32_t)n;
     }
-    return (valid && certified) ? (double)md : 0.0;
+    return (valid && certified) ? md : 0.f;
 }
 
 }  // namespace km

@@ -178,10 +178,10 @@ __global__ void __launch_bounds__(kThreads) rescan_kernel(const T* __restrict__ 
                 if (mindist) mindist[b * N + i] = bd;
             }
             if (obj_acc) {  // the listed points' share of the objective: one atomic per chunk
-                double part = i >= 0 ? (double)bd : 0.0;
+                float part = i >= 0 ? bd : 0.f;  // fp32 within the warp, fp64 across
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-                if (lane == 0 && part != 0.0) atomicAdd(obj_acc + b, part);
+                if (lane == 0 && part != 0.f) atomicAdd(obj_acc + b, (double)part);
             }
         }
         cl_sync();  // no CTA refills its result slots while CTA 0 may still read them
