@@ -39,7 +39,8 @@ __device__ __forceinline__ bool write_norm_slice(__half* out, double v) {
     for (int i = 0; i < kNormPieces; ++i) {
         const int j = kOrder[i];
         const double w = (double)norm_piece_weight(j);
-        const double q = fmin(fmax(r / w, -65504.0), 65504.0);
+        // r / w as r times the exact reciprocal of the power-of-two weight: the same value, no division
+        const double q = fmin(fmax(r * (double)(1.f / norm_piece_weight(j)), -65504.0), 65504.0);
         __half p = __float2half_rn((float)q);
         if (fabsf(__half2float(p)) < 0x1p-14f) p = __float2half(0.f);
         bits[j] = __half_as_ushort(p);
