@@ -33,13 +33,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one launch on this workload (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
 # capture of the assignment and of the update kernel, each valid only for the kernel sources it was
 # taken on (sha1 of each file); reported as null once one of them changes.
-ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "e21333f77b5dd8c67c97a16012d3013010082d7d",
+ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "10671a7ed48f4a31cc3298a69624c0f0eca0f020",
                             "tc_ptx.cuh": "1aa5f8cb3f1a62ec39a0c8ebfc993d50a08a4596",
-                            "certify.cuh": "ce618f9d1dffef9afdb4b0865d77c5c3719a3078",
-                            "km_internal.cuh": "4c7b4ebb37a6c6ac9493c00aa8d8d0f6fdd47e32"},
-                  "bytes": 546.466816e6 + 10.963968e6, "workload": "b32_n65536_d128_k1024_f16"}
+                            "certify.cuh": "3ec630ee9ae5990396e6368699568c0d9a21a9f8",
+                            "km_internal.cuh": "5c6937782b4ef766ba3e026a4e95b9c39a1e1f3a"},
+                  "bytes": 546.461184e6 + 18.694144e6, "workload": "b32_n65536_d128_k1024_f16"}
 UPDATE_TRAFFIC = {"files": {"update.cu": "c2925d516164c1f22f495185a00ac7554f0b41ff",
-                            "km_internal.cuh": "4c7b4ebb37a6c6ac9493c00aa8d8d0f6fdd47e32"},
+                            "km_internal.cuh": "5c6937782b4ef766ba3e026a4e95b9c39a1e1f3a"},
                   "bytes": 556.301824e6 + 15.386112e6, "workload": "b32_n65536_d128_k1024_f16"}
 
 
@@ -103,7 +103,10 @@ def work(w):
     s = w.elem_bytes
     B, N, K, d = w.B, w.N, w.K, w.d
     flops_assign = 2.0 * B * N * K * d
-    bytes_assign = B * N * (d * s + 8) + B * K * (d * s + 4)
+    # X, the label and mindist-or-objective share of each point, the centroids and their norm terms; the
+    # fp16 d <= 128 kernel also reads each point's ||x||^2, stored by a loop's first assignment
+    norms = 4 if (w.dtype == "f16" and 64 <= d <= 128 and d % 8 == 0) else 0
+    bytes_assign = B * N * (d * s + 8 + norms) + B * K * (d * s + 4)
     bytes_update = B * N * (d * s + 8) + 2 * B * K * d * 4 + 4 * B * K
     # the label sort: one pass (a thread-block cluster per batch) for batches of up to 65,536 labels
     # below 1024 clusters, else LSD radix passes of at most 8 bits; 16 bytes per key and pass

@@ -188,14 +188,14 @@ __global__ void __launch_bounds__(kThreads) rescan_kernel(const T* __restrict__ 
     }
 }
 
-// The cluster size: 16 CTAs when such clusters can be placed on this device
-// (checked once per device), else 8.
-int cluster_ctas() {
-    static std::atomic<int> state[64];  // per device: 0 unknown, else the size
+// How many clusters of 16 CTAs this device holds at once (checked once per
+// device; 0 when such clusters cannot be placed at all).
+int max_clusters16() {
+    static std::atomic<int> state[64];  // per device: 0 unknown, else 1 + the count
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
-        return 8;
+        return 0;
     }
     int s = state[dev].load(std::memory_order_acquire);
     if (s == 0) {
@@ -203,6 +203,7 @@ int cluster_ctas() {
                       cudaSuccess &&
                   cudaFuncSetAttribute(rescan_kernel<float>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
                       cudaSuccess;
+        int most = 1 << 30;
         for (int which = 0; ok && which < 2; ++which) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(kClusterMax, 1, 1);
@@ -218,12 +219,13 @@ int cluster_ctas() {
             ok = (which == 0 ? cudaOccupancyMaxActiveClusters(&n, rescan_kernel<__half>, &cfg)
                              : cudaOccupancyMaxActiveClusters(&n, rescan_kernel<float>, &cfg)) == cudaSuccess &&
                  n >= 1;
+            most = std::min(most, n);
         }
         if (!ok) cudaGetLastError();
-        s = ok ? kClusterMax : 8;
+        s = 1 + (ok ? most : 0);
         state[dev].store(s, std::memory_order_release);
     }
-    return s;
+    return s - 1;
 }
 
 }  // namespace
@@ -232,9 +234,15 @@ cudaError_t launch_rescan(const void* X, int dtype, const float* C, int64_t B, i
                           int32_t* labels, float* mindist, double* obj_acc, const RescanList& list, int sms,
                           cudaStream_t st, const int32_t* stop, int32_t* reset) {
     if (!list.count || !list.rows) return cudaErrorInvalidValue;
-    const int cs = cluster_ctas();
-    // enough clusters per batch to fill the GPU about twice when the lists are long
-    const int64_t per_batch = std::max<int64_t>(1, std::min<int64_t>(ceil_div(N, kPoints), 2 * sms / (cs * B)));
+    // enough clusters per batch to fill the GPU about twice when the lists are long; clusters of 16
+    // CTAs (the centroids split 16 ways) only while all of them fit on the device at once: a second
+    // wave of clusters costs even a launch whose lists are empty (~6 us for 32 batches)
+    auto per_batch_for = [&](int c) {
+        return std::max<int64_t>(1, std::min<int64_t>(ceil_div(N, kPoints), 2 * sms / (c * B)));
+    };
+    const int most16 = max_clusters16();
+    const int cs = most16 > 0 && B * per_batch_for(kClusterMax) <= most16 ? kClusterMax : 8;
+    const int64_t per_batch = per_batch_for(cs);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(cs * per_batch), (unsigned)B, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
