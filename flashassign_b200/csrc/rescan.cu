@@ -5,14 +5,17 @@
 // on ties -- the FlashAssign recurrence of the papernotes.org "Flash-KMeans"
 // page (关键设计 1) without the norm expansion, so no cancellation.
 //
-// The list is short (a few points per batch, often none), so the kernel is
-// built for latency: a thread-block cluster takes 32 listed points of one
-// batch at a time and splits the batch's centroids among its CTAs; in a CTA,
-// lane p of every warp holds point p and each warp a slice of the CTA's
-// centroids; the warps' results are joined in shared memory and the CTAs'
-// through distributed shared memory by CTA 0, which writes the label, mindist
-// and the objective share.  The distance of each (point, centroid) is summed
-// over ascending dimensions, as the CUDA-core assignment kernel sums it.
+// A thread-block cluster takes 32 listed points of one batch at a time and
+// splits the batch's centroids among its CTAs.  In a CTA, each warp holds 4 of
+// the points and each lane 4 centroids of a 128-centroid block, so that every
+// staged value feeds 16 differences (register tiles of 4 points x 4
+// centroids); the lanes' nearest centroids are joined by shuffles and the
+// CTAs' through distributed shared memory by CTA 0, which writes the label,
+// mindist and the objective share.  The distance of each (point, centroid) is
+// summed over ascending dimensions, as the CUDA-core assignment kernel sums
+// it.  The launch does not know how long the lists are (they are filled on the
+// device): it is sized to fill the GPU when they are long, and a CTA whose
+// batch has nothing listed returns at once.
 #include "km_internal.cuh"
 
 #include <algorithm>
@@ -23,10 +26,13 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kPoints = 32;                 // points per chunk, one per lane
-constexpr int kPerWarp = 8;                 // centroids per warp per block
-constexpr int kBlockK = kWarps * kPerWarp;  // centroids per CTA per block (64)
+constexpr int kPts = 4;                     // points per warp (every lane holds all 4)
+constexpr int kPoints = kWarps * kPts;      // points per chunk (32)
+constexpr int kPerLane = 4;                 // centroids per lane per block
+constexpr int kBlockK = 32 * kPerLane;      // centroids per CTA per block (128)
 constexpr int kSlice = 32;                  // dimensions per staged slice
+constexpr int kXStride = kPoints + 4;       // staged rows, padded (and 16-byte aligned for float4 reads)
+constexpr int kCStride = kBlockK + 4;
 constexpr int kClusterMax = 16;             // non-portable on sm_100, checked placeable
 
 template <typename T>
@@ -76,10 +82,8 @@ __global__ void __launch_bounds__(kThreads) rescan_kernel(const T* __restrict__ 
     pdl_trigger();
     pdl_wait();
     if (stop && *stop) return;  // read by every CTA of the cluster alike
-    __shared__ float xs[kPoints][kSlice + 1];
-    __shared__ float cs[kBlockK][kSlice + 1];
-    __shared__ float red_d[kWarps][kPoints];
-    __shared__ int red_k[kWarps][kPoints];
+    __shared__ __align__(16) float xs[kSlice][kXStride];  // the chunk's points, a slice of dimensions, transposed
+    __shared__ __align__(16) float cs[kSlice][kCStride];  // a block's centroids, the same slice, transposed
     __shared__ float res_d[kPoints];
     __shared__ int res_k[kPoints];
     __shared__ int64_t rows[kPoints];
@@ -104,60 +108,89 @@ __global__ void __launch_bounds__(kThreads) rescan_kernel(const T* __restrict__ 
             rows[threadIdx.x] = p >= npts ? -1 : whole ? p : (int64_t)list[b * cap + p];
         }
         __syncthreads();
-        float best = INFINITY;
-        int bk = -1;
-        for (int64_t kb = k_lo; kb < k_hi; kb += kBlockK) {
-            float acc[kPerWarp];
+        float best[kPts];
+        int bk[kPts];
 #pragma unroll
-            for (int c = 0; c < kPerWarp; ++c) acc[c] = 0.f;
+        for (int i = 0; i < kPts; ++i) {
+            best[i] = INFINITY;
+            bk[i] = -1;
+        }
+        for (int64_t kb = k_lo; kb < k_hi; kb += kBlockK) {
+            float acc[kPts][kPerLane];
+#pragma unroll
+            for (int i = 0; i < kPts; ++i)
+#pragma unroll
+                for (int c = 0; c < kPerLane; ++c) acc[i][c] = 0.f;
             for (int64_t j0 = 0; j0 < d; j0 += kSlice) {
                 for (int t = threadIdx.x; t < kPoints * kSlice; t += kThreads) {
                     const int r = t / kSlice, j = t % kSlice;
                     const int64_t gi = rows[r], gj = j0 + j;
-                    xs[r][j] = (gi >= 0 && gj < d) ? to_f<T>(Xb[gi * d + gj]) : 0.f;
+                    xs[j][r] = (gi >= 0 && gj < d) ? to_f<T>(Xb[gi * d + gj]) : 0.f;
                 }
                 for (int t = threadIdx.x; t < kBlockK * kSlice; t += kThreads) {
                     const int r = t / kSlice, j = t % kSlice;
                     const int64_t gk = kb + r, gj = j0 + j;
                     float v = (gk < k_hi && gj < d) ? Cb[gk * d + gj] : 0.f;
                     if (sizeof(T) == 2) v = __half2float(__float2half_rn(v));  // the centroids as the assignment sees them
-                    cs[r][j] = v;
+                    cs[j][r] = v;
                 }
                 __syncthreads();
 #pragma unroll 8
                 for (int j = 0; j < kSlice; ++j) {
-                    const float xv = xs[lane][j];
+                    const float4 xv = *reinterpret_cast<const float4*>(&xs[j][warp * kPts]);
+                    const float4 cv = *reinterpret_cast<const float4*>(&cs[j][lane * kPerLane]);
+                    const float xa[kPts] = {xv.x, xv.y, xv.z, xv.w}, ca[kPerLane] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-                    for (int c = 0; c < kPerWarp; ++c) {
-                        const float diff = xv - cs[warp * kPerWarp + c][j];
-                        acc[c] = fmaf(diff, diff, acc[c]);
-                    }
+                    for (int i = 0; i < kPts; ++i)
+#pragma unroll
+                        for (int c = 0; c < kPerLane; ++c) {
+                            const float diff = xa[i] - ca[c];
+                            acc[i][c] = fmaf(diff, diff, acc[i][c]);
+                        }
                 }
                 __syncthreads();
             }
+            // each point's nearest centroid of the block: the lane's four (ascending k: strict keeps
+            // the lowest), then across the lanes
 #pragma unroll
-            for (int c = 0; c < kPerWarp; ++c) {
-                const int64_t k = kb + warp * kPerWarp + c;
-                if (k < k_hi && acc[c] < best) {  // ascending k within the warp: strict keeps the lowest
-                    best = acc[c];
-                    bk = (int)k;
+            for (int i = 0; i < kPts; ++i) {
+                float bd = INFINITY;
+                int kk = -1;
+#pragma unroll
+                for (int c = 0; c < kPerLane; ++c) {
+                    const int64_t k = kb + lane * kPerLane + c;
+                    if (k < k_hi && acc[i][c] < bd) {
+                        bd = acc[i][c];
+                        kk = (int)k;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float od = __shfl_xor_sync(0xffffffffu, bd, o);
+                    const int ok = __shfl_xor_sync(0xffffffffu, kk, o);
+                    if (nearer(od, ok, bd, kk)) {
+                        bd = od;
+                        kk = ok;
+                    }
+                }
+                if (nearer(bd, kk, best[i], bk[i])) {
+                    best[i] = bd;
+                    bk[i] = kk;
                 }
             }
         }
-        // this CTA's nearest centroid of each point: join the warps
-        red_d[warp][lane] = best;
-        red_k[warp][lane] = bk;
-        __syncthreads();
-        if (warp == 0) {
-            float bd = red_d[0][lane];
-            int kk = red_k[0][lane];
-            for (int w = 1; w < kWarps; ++w)
-                if (nearer(red_d[w][lane], red_k[w][lane], bd, kk)) {
-                    bd = red_d[w][lane];
-                    kk = red_k[w][lane];
+        // this CTA's nearest centroid of each point (every lane of a warp holds its four)
+        if (lane < kPts) {
+            float rd = best[0];
+            int rk = bk[0];
+#pragma unroll
+            for (int i = 1; i < kPts; ++i)
+                if (lane == i) {
+                    rd = best[i];
+                    rk = bk[i];
                 }
-            res_d[lane] = bd;
-            res_k[lane] = kk;
+            res_d[warp * kPts + lane] = rd;
+            res_k[warp * kPts + lane] = rk;
         }
         cl_sync();  // every CTA's result is visible to the cluster
         if (rank == 0 && warp == 0) {
@@ -234,11 +267,11 @@ cudaError_t launch_rescan(const void* X, int dtype, const float* C, int64_t B, i
                           int32_t* labels, float* mindist, double* obj_acc, const RescanList& list, int sms,
                           cudaStream_t st, const int32_t* stop, int32_t* reset) {
     if (!list.count || !list.rows) return cudaErrorInvalidValue;
-    // enough clusters per batch to fill the GPU about twice when the lists are long; clusters of 16
+    // enough clusters per batch to fill the GPU about four times when the lists are long; clusters of 16
     // CTAs (the centroids split 16 ways) only while all of them fit on the device at once: a second
     // wave of clusters costs even a launch whose lists are empty (~6 us for 32 batches)
     auto per_batch_for = [&](int c) {
-        return std::max<int64_t>(1, std::min<int64_t>(ceil_div(N, kPoints), 2 * sms / (c * B)));
+        return std::max<int64_t>(1, std::min<int64_t>(ceil_div(N, kPoints), 4 * sms / (c * B)));
     };
     const int most16 = max_clusters16();
     const int cs = most16 > 0 && B * per_batch_for(kClusterMax) <= most16 ? kClusterMax : 8;
