@@ -433,21 +433,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (int rq = 0; rq < kRows / 32; ++rq) {
                     const int r = rq * 32 + lane;
                     float xnorm = 0.f;
-                    for (int kb = 0; kb < boxes; ++kb) {
-                        const uint4* rowp =
-                            reinterpret_cast<const uint4*>(smem + kXOff + (xb * kMaxBoxes + kb) * kBoxBytes + r * 128);
-#pragma unroll
-                        for (int cch = 0; cch < 8; ++cch) {
-                            const uint4 xv = rowp[(cch + lane) & 7];  // lanes start on different banks
-                            const __half2* hh = reinterpret_cast<const __half2*>(&xv);
-#pragma unroll
-                            for (int t = 0; t < 4; ++t) {
-                                const float2 f = __half22float2(hh[t]);
-                                xnorm = fmaf(f.x, f.x, xnorm);
-                                xnorm = fmaf(f.y, f.y, xnorm);
-                            }
-                        }
-                    }
+                    for (int kb = 0; kb < boxes; ++kb)
+                        xnorm = add_sq_row_sw128_f16(smem + kXOff + (xb * kMaxBoxes + kb) * kBoxBytes + r * 128, lane,
+                                                     xnorm);
                     xn[rq] = xnorm;
                     if (P.xnorm && n0 + r < P.N) P.xnorm[(int64_t)b * P.N + n0 + r] = xnorm;
                 }

@@ -276,21 +276,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     // 16-byte chunks within a 128-byte row, so each row's bytes
                     // are all in that row); then the buffer may be refilled.
                     if (h == 0) {
-                        for (int kb = 0; kb < boxes; ++kb) {
-                            const uint4* rowp = reinterpret_cast<const uint4*>(
-                                smem + kXOff + (xb * xbuf_boxes + kb) * kBoxBytes + row * 128);
-#pragma unroll
-                            for (int cch = 0; cch < 8; ++cch) {
-                                const uint4 xv = rowp[(cch + lane) & 7];  // lanes start on different banks
-                                const __half2* hh = reinterpret_cast<const __half2*>(&xv);
-#pragma unroll
-                                for (int t = 0; t < 4; ++t) {
-                                    const float2 f = __half22float2(hh[t]);
-                                    xnorm = fmaf(f.x, f.x, xnorm);
-                                    xnorm = fmaf(f.y, f.y, xnorm);
-                                }
-                            }
-                        }
+                        for (int kb = 0; kb < boxes; ++kb)
+                            xnorm = add_sq_row_sw128_f16(smem + kXOff + (xb * xbuf_boxes + kb) * kBoxBytes + row * 128,
+                                                         lane, xnorm);
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_x_empty + 8 * xb);

@@ -94,6 +94,27 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const CUtensorMap* m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
         : "memory");
 }
+// Adds the squares of one 128-byte row of a staged 128B-swizzled fp16 tile
+// (64 values) to acc, in fp32.  The swizzle permutes the row's 16-byte
+// chunks, so the row's values are all in it, in another order; each lane
+// starts at its own chunk so that the rows of a warp start on different
+// banks.  Every caller sums in this order, so a norm is the same number
+// whichever kernel computed it.
+__device__ __forceinline__ float add_sq_row_sw128_f16(const unsigned char* row, int lane, float acc) {
+    const uint4* rowp = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+    for (int cch = 0; cch < 8; ++cch) {
+        const uint4 xv = rowp[(cch + lane) & 7];
+        const __half2* hh = reinterpret_cast<const __half2*>(&xv);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const float2 f = __half22float2(hh[t]);
+            acc = fmaf(f.x, f.x, acc);
+            acc = fmaf(f.y, f.y, acc);
+        }
+    }
+    return acc;
+}
 // UMMA shared-memory descriptors, K-major operands, descriptor version 1.
 //  128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
 //  32-byte swizzle:  rows of 32 bytes (one K=16 fp16 slice), 8-row groups 256 bytes apart.
