@@ -33,7 +33,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one launch on this workload (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
 # capture of the assignment and of the update kernel, each valid only for the kernel sources it was
 # taken on (sha1 of each file); reported as null once one of them changes.
-ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "af09440c8397091e3c49d7ec6b5fca3f1ba2f1ed",
+ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "4aef69159a11d2fb4c430976ebb6eee8a3d57ace",
                             "tc_ptx.cuh": "a536562d7e7b15af8ce19a9bc4897a952f42b80a",
                             "certify.cuh": "3ec630ee9ae5990396e6368699568c0d9a21a9f8",
                             "km_internal.cuh": "5c6937782b4ef766ba3e026a4e95b9c39a1e1f3a"},

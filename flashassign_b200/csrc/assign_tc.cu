@@ -40,25 +40,34 @@
 //     128-column TMEM load, the accumulator released as soon as they are in
 //     registers; warp 11 finishes each unit (below), so that nothing but tile
 //     work sits between two accumulator releases of the epilogue warps.
-//   * Epilogue: per 32-column group, the group maximum (3-input max) is
-//     compared with the running best; only when it improves (in any lane of
-//     the warp) is the group scanned for its first column equal to the
-//     maximum, which becomes the running label.  At the end of a unit each
-//     epilogue warp posts its (score, label) to a double-buffered shared slot.
-//   * Unit finish (warp 11): as soon as the unit's first tile of MMAs has
-//     completed (a commit on a per-buffer barrier), ||x||^2 of each row is
-//     summed from the staged X tile and the X buffer is released while the
-//     unit's other tiles run (two X buffers then suffice); at the unit's end
-//     the two column slices are joined (larger score, then lower index), and
-//     each point whose label the scores' error bound certifies (certify.cuh)
-//     gets its label and mindist = ||x||^2 - 2 * best, and adds to the
-//     objective (one atomic per unit); the others are listed for the exact
+//   * Epilogue: each warp's 128-column slice of a tile is reduced to every
+//     point's best and second-best score as an 8 x 16 grid (row and column
+//     maxima, about 1.5 ALU instructions per score; certify.cuh) and folded
+//     into the running (best, second, label); at the end of a unit each
+//     epilogue warp posts them to a double-buffered shared slot.
+//   * Unit finish (warp 11): ||x||^2 of each row is either read (the later
+//     assignments of a Lloyd loop, from an array the first one wrote), or
+//     summed from the staged X tile as soon as the unit's first tile of MMAs
+//     has completed (a commit on a per-buffer barrier), the X buffer being
+//     released right after; at the unit's end the two column slices are
+//     joined (larger score, then lower index), and each point whose label
+//     the scores' error bound certifies (certify.cuh) gets its label and
+//     mindist = ||x||^2 - 2 * best and adds to the objective (summed in fp32,
+//     one fp64 atomic per unit); the others are listed for the exact
 //     re-scan.  Three X buffers with the release at the unit's end left room
 //     for only three centroid stages: 5% slower at K = 1024.
-//   * Measured on B200: at the 1 kW power cap the SM clock settles near
-//     1.4 GHz (K = 4096) to 1.7 GHz (K = 1024) and a tile costs ~1.1 us of
-//     wall time either way: the kernel runs at the power limit, so fewer
-//     cycles per tile buy a lower clock rather than time.
+//   * The issuers carry their unit and batch counters in 32 bits (a 64-bit
+//     division between two units' MMAs cost 7% at K = 1024) and issue each
+//     tile's K steps unrolled, with immediate descriptor offsets.
+//   * Two accumulator sets bound the rate at K = 1024: tile t+2 starts only
+//     after tile t's MMAs have completed, its TMEM has been read and the
+//     release has reached the issuer (~2900 cycles for two tiles against 2300
+//     of MMA work).  Narrower tiles would give more sets but read the points'
+//     operand twice as often from shared memory (above).
+//   * Measured on B200: in a long loop the 1 kW power cap lowers the SM
+//     clock (~1.6-1.7 GHz at K = 1024 under the profiler, ~1.4 GHz at
+//     K = 4096), so part of any saving in cycles per tile is paid back as a
+//     lower clock.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records a fault code in the device fault word, stops issuing work, frees
 // its TMEM and returns.
