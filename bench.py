@@ -184,9 +184,11 @@ def oracle_iteration(X, C):
     return time.perf_counter() - t0, lab, d1, d2
 
 
-def oracle_problems(w, target_s: float) -> int:
-    """How many whole problems of the workload the oracle iterates in about target_s seconds (at least
-    one), from a timed probe of 2048 rows of one problem."""
+def oracle_sample(w, target_s: float) -> tuple[int, int]:
+    """The part of the workload the oracle iterates in about target_s seconds, from a timed probe of
+    2048 rows of one problem: (nb, rows) = the first nb whole problems (rows = N), or, when one problem
+    takes longer, the first `rows` points of the first problem (the oracle's time grows linearly in the
+    points at a fixed K)."""
     import numpy as np
     import synth
     rows = min(2048, w.N)
@@ -195,13 +197,26 @@ def oracle_problems(w, target_s: float) -> int:
     if Cp.shape[1] < w.K:
         Cp = np.concatenate([Cp] * (-(-w.K // Cp.shape[1])), axis=1)[:, :w.K].copy()
     dt, *_ = oracle_iteration(Xp, Cp)
-    per_problem = dt * w.N / rows
-    return int(max(1, min(w.B, target_s // max(per_problem, 1e-9))))
+    per_row = max(dt / rows, 1e-12)
+    if per_row * w.N <= target_s:
+        return int(max(1, min(w.B, target_s // (per_row * w.N)))), w.N
+    return 1, int(min(w.N, max(rows, target_s // per_row)))
 
 
-def cpu_sample_text(w, nb: int, dt: float) -> str:
-    part = "the whole iteration" if nb == w.B else f"{nb} of the {w.B} problems, scaled x{w.B / nb:g} to all {w.B}"
-    return (f"oracle assign+update (plain C++, fp64, K={w.K}, d={w.d}) of whole problems: {part}; "
+def sample_scale(w, nb: int, rows: int) -> float:
+    """From the sample's oracle time to the whole iteration's."""
+    return (w.B / nb) * (w.N / rows)
+
+
+def cpu_sample_text(w, nb: int, rows: int, dt: float) -> str:
+    if rows < w.N:
+        part = (f"the first {rows} of the {w.N} points of problem 0 against all {w.K} centroids, scaled "
+                f"x{sample_scale(w, nb, rows):.4g} to the whole iteration")
+    elif nb == w.B:
+        part = "whole problems: the whole iteration"
+    else:
+        part = f"whole problems: {nb} of the {w.B} problems, scaled x{w.B / nb:g} to all {w.B}"
+    return (f"oracle assign+update (plain C++, fp64, K={w.K}, d={w.d}) of {part}; "
             f"{dt:.2f} s measured on {cpu_model()}")
 
 
@@ -214,23 +229,27 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     import oracle
-    nb = oracle_problems(w, 12.0)
-    wx = w.with_(B=nb)
-    X = synth.points(wx)
-    C = synth.init_centroids(wx, X)
+    nb, rows = oracle_sample(w, 12.0)
+    if rows == w.N:
+        wx = w.with_(B=nb)
+        X = synth.points(wx)
+        C = synth.init_centroids(wx, X)
+    else:  # the first rows of problem 0, and its first K points as the centroids
+        X = synth.points(w.with_(B=1), 0, rows)
+        C = synth.points(w.with_(B=1), 0, w.K).astype("float32")
     for _ in range(args.warmup):
-        oracle_iteration(X[:1], C[:1])
+        oracle_iteration(X[:1, : min(rows, 2048)], C[:1])
     times = []
     for _ in range(args.steps):
         dt, *_ = oracle_iteration(X, C)
         times.append(dt)
-    v = statistics.mean(times) * 1e3 * w.B / nb
+    v = statistics.mean(times) * 1e3 * sample_scale(w, nb, rows)
     out = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
            "config": bench_config(w, args.gpus),
            "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-                            "cpu": cpu_model(), "sample": cpu_sample_text(w, nb, statistics.mean(times))},
+                            "cpu": cpu_model(), "sample": cpu_sample_text(w, nb, rows, statistics.mean(times))},
            "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0
@@ -242,18 +261,19 @@ def bench_config(w, world: int) -> dict:
             "l2": f"inputs larger than L2 (X is {w.B * w.N * w.d * w.elem_bytes / 2**20:.0f} MiB)"}
 
 
-def parity_report(w, X_host, C_host, gpu_labels, nb: int):
-    """The oracle's iteration of the first nb problems at the GPU's current centroids, timed (the CPU
-    baseline), and compared with the GPU's assignment there: labels must equal the oracle's at every
-    point whose relative top-2 gap (d2 - d1) / d2 is at least 1e-3 (fp16) or 1e-5 (fp32); the points
-    below it (near ties, where either label is allowed) are counted."""
+def parity_report(w, X_host, C_host, gpu_labels, nb: int, rows: int):
+    """The oracle's iteration of the sample (the first nb problems, or the first rows points of problem 0)
+    at the GPU's current centroids, timed (the CPU baseline), and compared with the GPU's assignment
+    there: labels must equal the oracle's at every point whose relative top-2 gap (d2 - d1) / d2 is at
+    least 1e-3 (fp16) or 1e-5 (fp32); the points below it (near ties, where either label is allowed) are
+    counted."""
     import numpy as np
-    Xs, Cs = np.ascontiguousarray(X_host[:nb]), np.ascontiguousarray(C_host[:nb])
+    Xs, Cs = np.ascontiguousarray(X_host[:nb, :rows]), np.ascontiguousarray(C_host[:nb])
     dt, lab, d1, d2 = oracle_iteration(Xs, Cs)
     tau = 1e-3 if w.dtype == "f16" else 1e-5
     gap = (d2 - d1) / np.maximum(d2, np.finfo(np.float64).tiny)
     clear = gap >= tau
-    g = gpu_labels[:nb]
+    g = gpu_labels[:nb, :rows]
     return dt, {"checked_points": int(lab.size), "near_tie_points": int((~clear).sum()),
                 "label_mismatches_at_clear_points": int((clear & (g != lab)).sum()),
                 "label_mismatches_at_near_ties": int((~clear & (g != lab)).sum()), "tau": tau}
@@ -495,10 +515,10 @@ def run_ours(args, w):
     cpu = parity = None
     if not args.no_cpu and world == 1:
         import oracle
-        nb = oracle_problems(w, 12.0)
-        dt, parity = parity_report(w, X_host, C.cpu().numpy(), lab_final.cpu().numpy(), nb)
-        cpu = {"value": round(dt * 1e3 * w.B / nb, 1), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-               "cpu": cpu_model(), "sample": cpu_sample_text(w, nb, dt)}
+        nb, rows = oracle_sample(w, 12.0)
+        dt, parity = parity_report(w, X_host, C.cpu().numpy(), lab_final.cpu().numpy(), nb, rows)
+        cpu = {"value": round(dt * 1e3 * sample_scale(w, nb, rows), 1), "unit": UNIT, "cores": oracle.threads(),
+               "kind": "oracle", "cpu": cpu_model(), "sample": cpu_sample_text(w, nb, rows, dt)}
         parity["rescanned_points"] = rescans
         parity["note"] = ("km_assign at the run's final centroids against the oracle's assignment of the same "
                           "problems (the CPU baseline's run)")
