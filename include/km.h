@@ -77,11 +77,10 @@ typedef enum {
  *     splits of both operands (three products);
  *   - other shapes: direct differences sum_j (x_j - c_j)^2 on the CUDA cores.
  * On the tensor-core paths each point's label is certified against the
- * rounding-error bound of its scores, from its best score (fp16, d <= 128) or
- * its best two scores (wider fp16, fp32); a point that is not certified (near
- * ties, near-duplicate centroids, data far from the origin, fp16 centroid
- * norms beyond the folded norm term's range of ~3.4e10) is re-scanned exactly
- * on the CUDA cores (see km_assign_rescans).  So every fp32 label is the exact argmin up
+ * rounding-error bound of its scores, from its best two scores; a point that
+ * is not certified (near ties, near-duplicate centroids, data far from the
+ * origin, fp16 centroid norms beyond the folded norm term's range of ~3.4e10)
+ * is re-scanned exactly on the CUDA cores (see km_assign_rescans).  So every fp32 label is the exact argmin up
  * to fp32 rounding, and every fp16 label is the exact argmin unless the two
  * smallest exact distances d1 <= d2 of the point satisfy d2 - d1 < 1e-3 d2,
  * in which case its distance is within 1e-3 d2 of d1.
