@@ -34,7 +34,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of the assignment and of the update kernel, each valid only for the kernel sources it was
 # taken on (sha1 of each file); reported as null once one of them changes.
 ASSIGN_TRAFFIC = {"files": {"assign_tc.cu": "4aef69159a11d2fb4c430976ebb6eee8a3d57ace",
-                            "tc_ptx.cuh": "a536562d7e7b15af8ce19a9bc4897a952f42b80a",
+                            "tc_ptx.cuh": "c97cffb6f51a284e71c2f9ae2e507213d09e6c46",
                             "certify.cuh": "3ec630ee9ae5990396e6368699568c0d9a21a9f8",
                             "km_internal.cuh": "5c6937782b4ef766ba3e026a4e95b9c39a1e1f3a"},
                   "bytes": 546.363904e6 + 17.49248e6, "workload": "b32_n65536_d128_k1024_f16"}
